@@ -1,0 +1,9 @@
+"""B200-native fused top-k Mixture-of-Experts layer.
+
+The compute path lives in the CUDA library ``libmoe_b200.so`` (sources in
+``csrc/``, C ABI in ``include/moe_b200.h``); :mod:`moe_layer_top_b200.ops`
+is the thin ctypes binding over it.  The library is loaded on first use and a
+missing or unloadable library raises: there is no CPU fallback.
+"""
+
+__all__ = ["ops", "inputs"]
