@@ -1,0 +1,236 @@
+/*
+ * moe_b200.h -- C ABI of the B200 (sm_100a) fused top-k Mixture-of-Experts layer.
+ *
+ * The layer computes, for every token t of x[T, H]:
+ *
+ *   route   : topk_ids[t, :], topk_weights[t, :] from router logits (softmax
+ *             over E experts, the k largest, renormalised), or given;
+ *   align   : the flat assignments t*topk + j sorted by expert and padded to
+ *             whole blocks of block_m rows (sorted_token_ids, expert_ids);
+ *   GEMM1   : h = x[t] . w13[e]^T  (w13[e] is [2I, H]; gate = rows [0, I),
+ *             up = rows [I, 2I)), held in bf16;
+ *   act     : a2 = bf16(bf16(silu(gate)) * up), re-quantised to FP8 E4M3 per
+ *             (row, 128 columns) with a power-of-two scale on the FP8 path;
+ *   GEMM2   : y[t*topk + j] = topk_weights[t, j] * (a2 . w2[e]^T)  (w2[e] is [H, I]);
+ *   combine : out[t] = sum_j y[t*topk + j].
+ *
+ * Sources: "AWS erklärt zwei Kernel-Optimierungen, die den Durchsatz von
+ * SageMaker AI auf H200 steigern" (kinachrichten.com), sections "Warum
+ * MoE-Kernel so wichtig sind" (fused routing + expert compute) and "Swap-AB"
+ * (weight rows fill the MMA M dimension at decode); the analysis of vLLM PR
+ * #64760 "FP8 MoE down-projection for H200" (blog.secrett2633.cloud), §1.1
+ * (expert-sorted intermediate, sorted_token_ids / num_tokens_post_padded,
+ * block-padded rows) and §1.2 (fused SiLU-mul-FP8 quantisation kernel); and
+ * "Hosting von Qwen auf Blackwell" (perplexity.ai), section "MoE Dispatch -
+ * Combine" (weighted accumulation in the combine).
+ *
+ * Conventions for every entry point:
+ *  - All tensor pointers are DEVICE pointers owned and allocated by the
+ *    caller, row-major and contiguous.  The library allocates no device or
+ *    host memory on these paths and keeps no per-call state.
+ *  - `stream` is a cudaStream_t (NULL = legacy default stream).  Every call
+ *    is asynchronous on it: it enqueues kernels and returns.  No call
+ *    synchronises the device unless its comment says so.
+ *  - Return value: MOE_OK, or a negative MOE_ERR_* code; on error
+ *    moe_last_error_string() (per host thread) describes it.  Arguments are
+ *    validated before anything is enqueued, so an error return means nothing
+ *    was launched (MOE_ERR_CUDA excepted: a launch failed part way).
+ *  - Bad device data (an expert id outside [0, E)) cannot be seen on the
+ *    host: the kernels record it in the workspace status word (see
+ *    moe_read_status) and the outputs of that call are undefined.
+ */
+#ifndef MOE_B200_H_
+#define MOE_B200_H_
+
+#include <stddef.h>
+#include <stdint.h>
+
+#if defined(__GNUC__)
+#define MOE_API __attribute__((visibility("default")))
+#else
+#define MOE_API
+#endif
+
+#ifdef __cplusplus
+extern "C" {
+#endif
+
+/* return codes */
+#define MOE_OK 0
+#define MOE_ERR_INVALID (-1)     /* null pointer, bad shape, misaligned pointer */
+#define MOE_ERR_UNSUPPORTED (-2) /* not an sm_100 device, unsupported combination */
+#define MOE_ERR_WORKSPACE (-3)   /* workspace smaller than moe_workspace_size() */
+#define MOE_ERR_CUDA (-4)        /* a CUDA call or kernel launch failed */
+
+/* device status word codes (moe_read_status) */
+#define MOE_STATUS_OK 0
+#define MOE_STATUS_BAD_EXPERT_ID 1    /* an expert id outside [0, E) */
+#define MOE_STATUS_WAIT_TIMEOUT 0x100 /* a bounded in-kernel wait ran out; low byte = where */
+
+/* weight types */
+#define MOE_DTYPE_BF16 0
+#define MOE_DTYPE_FP8_E4M3 1 /* E4M3 codes + one fp32 scale per 128 x 128 block */
+
+/* tile orientation of the two grouped GEMMs */
+#define MOE_MODE_AUTO 0    /* chosen from the expected tokens per expert */
+#define MOE_MODE_NORMAL 1  /* MMA M = 128 token rows, N = 256 weight rows */
+#define MOE_MODE_SWAP_AB 2 /* MMA M = 128 weight rows, N = block_m token rows */
+
+/* stages of moe_forward_stages, in pipeline order */
+#define MOE_STAGE_ROUTE 0   /* skipped when no router logits are given */
+#define MOE_STAGE_ALIGN 1   /* histogram, scan, stable scatter */
+#define MOE_STAGE_GATHER 2  /* x rows into expert-sorted order (+ FP8 quantisation) */
+#define MOE_STAGE_GEMM1 3   /* gate/up grouped GEMM + fused SiLU*up (+ FP8 requant) */
+#define MOE_STAGE_GEMM2 4   /* down grouped GEMM + routed-weight scatter */
+#define MOE_STAGE_COMBINE 5 /* per-token sum of its topk rows */
+#define MOE_NUM_STAGES 6
+
+/*
+ * Problem description.  T, E, topk, H, I and weight_dtype are required;
+ * mode = MOE_MODE_AUTO and block_m = 0 let the library choose; both are
+ * written back by moe_resolve_problem().
+ * Constraints: T >= 0, 1 <= topk <= E <= 1024, H and I positive multiples of
+ * 128, T * topk < 2^31.
+ */
+typedef struct moe_problem {
+  int32_t T;            /* tokens */
+  int32_t E;            /* experts */
+  int32_t topk;         /* experts per token */
+  int32_t H;            /* hidden size */
+  int32_t I;            /* expert intermediate size */
+  int32_t weight_dtype; /* MOE_DTYPE_* */
+  int32_t mode;         /* MOE_MODE_* */
+  int32_t block_m;      /* rows per expert block: 16, 32 or 64 (swap-AB), 128 (normal); 0 = auto */
+  int32_t renormalize;  /* router: 1 = renormalise the chosen softmax weights (default), 0 = keep them */
+  int32_t reserved[7];  /* must be zero */
+} moe_problem;
+
+/*
+ * Byte offsets of the intermediates inside the workspace (for inspection
+ * by tests and tools; all regions are 256-byte aligned).  A region a call
+ * does not use has offset -1.
+ */
+typedef struct moe_workspace_layout {
+  int64_t status;           /* int32 status word */
+  int64_t topk_ids;         /* int32 [T*topk]      (router output) */
+  int64_t topk_weights;     /* fp32  [T*topk]      (router output) */
+  int64_t sorted_token_ids; /* int32 [capacity] */
+  int64_t expert_ids;       /* int32 [capacity / block_m] */
+  int64_t num_tokens_post_padded; /* int32 */
+  int64_t expert_counts;    /* int32 [E] */
+  int64_t expert_offsets;   /* int32 [E + 1] */
+  int64_t align_scratch;    /* int32 [chunks * E] */
+  int64_t a1;               /* bf16 or E4M3 [capacity, H] x rows in sorted order */
+  int64_t a1_scale;         /* fp32 [H/128, capacity] (FP8 only; K-block major) */
+  int64_t a2;               /* bf16 or E4M3 [capacity, I] activation in sorted order */
+  int64_t a2_scale;         /* fp32 [I/128, capacity] (FP8 only; K-block major) */
+  int64_t y;                /* bf16 [T*topk, H] weighted expert outputs */
+  int64_t total_bytes;
+  int32_t capacity;         /* rows of sorted_token_ids */
+  int32_t block_m;
+  int32_t mode;
+  int32_t align_chunks;
+} moe_workspace_layout;
+
+/* Human-readable description of the last error on this host thread. */
+MOE_API const char* moe_last_error_string(void);
+
+/*
+ * Top-k softmax router ("Warum MoE-Kernel so wichtig sind": token routing).
+ * logits [T, E] fp32 -> topk_ids [T, topk] int32, topk_weights [T, topk] fp32.
+ * Experts are taken by descending logit, equal logits by the lower index;
+ * weights are softmax probabilities (renormalize = 0) or those renormalised
+ * over the chosen experts (renormalize = 1).  One warp per token.
+ */
+MOE_API int moe_route(const float* logits, int32_t T, int32_t E, int32_t topk, int32_t renormalize,
+              int32_t* topk_ids, float* topk_weights, void* stream);
+
+/*
+ * Rows of sorted_token_ids for a problem: an upper bound of
+ * sum_e ceil(count_e / block_m) * block_m, namely
+ * block_m * ceil((T*topk + min(E, T*topk) * (block_m - 1)) / block_m).
+ * Returns -1 on invalid arguments.
+ */
+MOE_API int64_t moe_align_capacity(int32_t T, int32_t topk, int32_t E, int32_t block_m);
+
+/* Scratch bytes moe_align() needs (per-chunk expert histograms). */
+MOE_API size_t moe_align_workspace_size(int32_t T, int32_t topk, int32_t E);
+
+/*
+ * Expert alignment (vLLM PR #64760 analysis, §1.1: sorted_token_ids,
+ * num_tokens_post_padded, one expert per BLOCK_SIZE_M rows).
+ *   topk_ids [T, topk] int32 in [0, E).
+ *   sorted_token_ids [capacity] int32: the flat ids t*topk + j of expert 0,
+ *     then expert 1, ..., each expert's run in ascending flat order and padded
+ *     with the sentinel T*topk to a multiple of block_m; the sentinel also
+ *     fills [num_tokens_post_padded, capacity).
+ *   expert_ids [capacity / block_m] int32: the expert of each used block, -1 after.
+ *   num_tokens_post_padded [1] int32.
+ *   expert_counts [E], expert_offsets [E + 1] int32: may be NULL.
+ *   ws / ws_bytes: scratch of at least moe_align_workspace_size() bytes.
+ * Deterministic: the result is a pure function of topk_ids.
+ */
+MOE_API int moe_align(const int32_t* topk_ids, int32_t T, int32_t topk, int32_t E, int32_t block_m,
+              int32_t* sorted_token_ids, int32_t* expert_ids, int32_t* num_tokens_post_padded,
+              int32_t* expert_counts, int32_t* expert_offsets, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * FP8 weight preparation: w [batches, rows, cols] bf16 -> codes [batches,
+ * rows, cols] E4M3 and scales [batches, rows/128, cols/128] fp32 with, per
+ * 128 x 128 block, scale = max(blockmax, 1e-10) / 448 (fp32) and
+ * code = e4m3(fp32(w / scale)) (round to nearest even, saturating).
+ * rows and cols must be multiples of 128.
+ */
+MOE_API int moe_quantize_weights_fp8(const void* w, int64_t batches, int32_t rows, int32_t cols, uint8_t* codes,
+                             float* scales, void* stream);
+
+/* Fill in mode and block_m when they are left to the library; validates p. */
+MOE_API int moe_resolve_problem(moe_problem* p);
+
+/* Workspace bytes moe_fused_forward needs for p (0 on invalid p). */
+MOE_API size_t moe_workspace_size(const moe_problem* p);
+
+/* Where each intermediate lives inside the workspace for p. */
+MOE_API int moe_get_workspace_layout(const moe_problem* p, moe_workspace_layout* layout);
+
+/*
+ * The fused MoE layer, all stages on `stream`.
+ *   x             [T, H] bf16.
+ *   router_logits [T, E] fp32, or NULL to use topk_ids / topk_weights
+ *                 ([T, topk] int32 / fp32), which are then required.
+ *   w13           [E, 2I, H]: bf16, or E4M3 codes with w13_scale [E, 2I/128, H/128] fp32.
+ *   w2            [E, H, I]:  bf16, or E4M3 codes with w2_scale  [E, H/128, I/128] fp32.
+ *   out           [T, H] bf16.
+ *   ws            device scratch of at least moe_workspace_size(p) bytes,
+ *                 256-byte aligned; the call clears what must start at zero.
+ *                 Two calls that overlap on the device must not share it.
+ * All pointers 16-byte aligned.  T = 0 is a no-op (its buffers may be NULL).
+ */
+MOE_API int moe_fused_forward(const moe_problem* p, const void* x, const float* router_logits, const int32_t* topk_ids,
+                      const float* topk_weights, const void* w13, const void* w2, const float* w13_scale,
+                      const float* w2_scale, void* out, void* ws, size_t ws_bytes, void* stream);
+
+/*
+ * The same pipeline restricted to stages [stage_begin, stage_end) (MOE_STAGE_*),
+ * so that a caller can time or inspect each stage.  Running every range of a
+ * partition in order is exactly moe_fused_forward.
+ */
+MOE_API int moe_forward_stages(const moe_problem* p, const void* x, const float* router_logits, const int32_t* topk_ids,
+                       const float* topk_weights, const void* w13, const void* w2, const float* w13_scale,
+                       const float* w2_scale, void* out, void* ws, size_t ws_bytes, int32_t stage_begin,
+                       int32_t stage_end, void* stream);
+
+/*
+ * Read (and with clear != 0, reset) the device status word of a workspace.
+ * SYNCHRONISES `stream`.  Writes MOE_STATUS_* into *status.
+ */
+MOE_API int moe_read_status(const moe_problem* p, void* ws, int32_t clear, int32_t* status, void* stream);
+
+/* Library version: major * 10000 + minor * 100 + patch. */
+MOE_API int32_t moe_version(void);
+
+#ifdef __cplusplus
+}
+#endif
+
+#endif /* MOE_B200_H_ */

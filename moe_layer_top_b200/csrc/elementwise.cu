@@ -1,0 +1,199 @@
+// Memory-bound helpers of the MoE pipeline: the gather of x into
+// expert-sorted order (with the FP8 per-(row,128) quantisation of the GEMM1
+// input), the top-k combine, and the FP8 128x128 weight quantiser used when
+// weights are prepared.  All move 16-byte vectors per thread.
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+struct alignas(16) bf16x8 {
+  __nv_bfloat162 h[4];
+};
+
+__device__ __forceinline__ void unpack8(const uint4& u, float (&f)[8]) {
+  const bf16x8 b = *reinterpret_cast<const bf16x8*>(&u);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    const float2 t = __bfloat1622float2(b.h[i]);
+    f[2 * i] = t.x;
+    f[2 * i + 1] = t.y;
+  }
+}
+
+__device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
+  bf16x8 b;
+#pragma unroll
+  for (int i = 0; i < 4; ++i) b.h[i] = __floats2bfloat162_rn(f[2 * i], f[2 * i + 1]);
+  return *reinterpret_cast<const uint4*>(&b);
+}
+
+}  // namespace
+
+// ----------------------------------------------------------------------------
+// gather: a1[r] = x[sorted_ids[r] / topk] for r < num_tokens_post_padded
+// (zeros for padding rows).  FP8: per (row, 128 columns) the power-of-two
+// scale of the vLLM PR #64760 analysis §1.2 rule, codes into a1 [cap, H],
+// scales into a1_scale_t [H/128, cap] (K-block major for the GEMM epilogue).
+// A block walks rows; a thread owns 8 consecutive columns, 16 threads one
+// 128-column group.
+// ----------------------------------------------------------------------------
+template <bool FP8>
+__global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* __restrict__ x, int H, int topk,
+                                                     int nflat, const int32_t* __restrict__ sorted_ids,
+                                                     const int32_t* __restrict__ ntpp_ptr, int capacity,
+                                                     void* __restrict__ a1, float* __restrict__ a1_scale_t) {
+  const int ntpp = *ntpp_ptr;
+  const int vecs = H / 8;
+  const int iters = (vecs + blockDim.x - 1) / blockDim.x;
+  for (int row = blockIdx.x; row < ntpp; row += gridDim.x) {
+    const int flat = __ldg(sorted_ids + row);
+    const bool real = flat < nflat;
+    const __nv_bfloat16* src = x + static_cast<size_t>(real ? flat / topk : 0) * H;
+    for (int it = 0; it < iters; ++it) {
+      const int v = it * blockDim.x + threadIdx.x;  // uniform trip count: shuffles below see full warps
+      const bool in = v < vecs;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (in && real) u = __ldg(reinterpret_cast<const uint4*>(src) + v);
+      if constexpr (!FP8) {
+        if (in) reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a1) + static_cast<size_t>(row) * H)[v] = u;
+      } else {
+        float f[8];
+        unpack8(u, f);
+        float amax = 0.f;
+#pragma unroll
+        for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+        for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        const float scale = act_scale_from_amax(amax);
+        const float inv = pow2_recip(scale);
+        uint2 q;
+        q.x = static_cast<uint32_t>(f32x2_to_e4m3x2(f[0] * inv, f[1] * inv)) |
+              (static_cast<uint32_t>(f32x2_to_e4m3x2(f[2] * inv, f[3] * inv)) << 16);
+        q.y = static_cast<uint32_t>(f32x2_to_e4m3x2(f[4] * inv, f[5] * inv)) |
+              (static_cast<uint32_t>(f32x2_to_e4m3x2(f[6] * inv, f[7] * inv)) << 16);
+        if (in) {
+          reinterpret_cast<uint2*>(static_cast<uint8_t*>(a1) + static_cast<size_t>(row) * H)[v] = q;
+          if ((v & 15) == 0) a1_scale_t[static_cast<size_t>(v >> 4) * capacity + row] = scale;
+        }
+      }
+    }
+  }
+}
+
+cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32_t* sorted_ids,
+                          const int32_t* ntpp, int capacity, bool fp8, void* a1, float* a1_scale_t,
+                          cudaStream_t stream) {
+  if (capacity == 0) return cudaSuccess;
+  int blocks = capacity < 148 * 8 ? capacity : 148 * 8;
+  if (fp8)
+    gather_kernel<true><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), H, topk, nflat, sorted_ids,
+                                                    ntpp, capacity, a1, a1_scale_t);
+  else
+    gather_kernel<false><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), H, topk, nflat,
+                                                     sorted_ids, ntpp, capacity, a1, a1_scale_t);
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------
+// combine ("Hosting von Qwen auf Blackwell", "MoE Dispatch - Combine": the
+// weighted accumulation; the weights were applied in the GEMM2 epilogue):
+// out[t, :] = bf16(sum_j y[t*topk + j, :]) in fp32, j ascending.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ y, int T, int topk, int H,
+                                                      __nv_bfloat16* __restrict__ out) {
+  const int vecs = H / 8;
+  const long long total = static_cast<long long>(T) * vecs;
+  for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
+       i += static_cast<long long>(gridDim.x) * blockDim.x) {
+    const long long t = i / vecs;
+    const int v = static_cast<int>(i - t * vecs);
+    float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
+    const uint4* src = reinterpret_cast<const uint4*>(y + static_cast<size_t>(t) * topk * H) + v;
+    for (int j = 0; j < topk; ++j) {
+      float f[8];
+      unpack8(__ldg(src + static_cast<size_t>(j) * vecs), f);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) acc[k] += f[k];
+    }
+    reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[v] = pack8(acc);
+  }
+}
+
+cudaError_t launch_combine(const void* y, int T, int topk, int H, void* out, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const long long total = static_cast<long long>(T) * (H / 8);
+  long long blocks = (total + 255) / 256;
+  if (blocks > 148 * 16) blocks = 148 * 16;
+  combine_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(y), T, topk, H,
+                                                               static_cast<__nv_bfloat16*>(out));
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------
+// weight preparation: one CTA per 128x128 block; thread = half a row (64
+// elements).  scale = max(blockmax, 1e-10) / 448 and code = e4m3(w / scale),
+// both divisions correctly rounded in fp32.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quantize_weights_kernel(const __nv_bfloat16* __restrict__ w, int rows,
+                                                               int cols, uint8_t* __restrict__ codes,
+                                                               float* __restrict__ scales) {
+  __shared__ float warp_max[8];
+  const int nbc = cols / 128, nbr = rows / 128;
+  const long long blk = blockIdx.x;
+  const long long b = blk / (static_cast<long long>(nbr) * nbc);
+  const int rem = static_cast<int>(blk - b * nbr * nbc);
+  const int br = rem / nbc, bc = rem - br * nbc;
+  const int r = threadIdx.x >> 1, half = threadIdx.x & 1;
+  const size_t row_off = (static_cast<size_t>(b) * rows + static_cast<size_t>(br) * 128 + r) * cols +
+                         static_cast<size_t>(bc) * 128 + half * 64;
+  const uint4* src = reinterpret_cast<const uint4*>(w + row_off);
+  float f[64];
+  float amax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) {
+    float t[8];
+    unpack8(__ldg(src + i), t);
+#pragma unroll
+    for (int k = 0; k < 8; ++k) {
+      f[8 * i + k] = t[k];
+      amax = fmaxf(amax, fabsf(t[k]));
+    }
+  }
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+  if ((threadIdx.x & 31) == 0) warp_max[threadIdx.x >> 5] = amax;
+  __syncthreads();
+  float bmax = 0.f;
+#pragma unroll
+  for (int i = 0; i < 8; ++i) bmax = fmaxf(bmax, warp_max[i]);
+  const float scale = __fdiv_rn(fmaxf(bmax, 1e-10f), 448.0f);
+  uint4* dst = reinterpret_cast<uint4*>(codes + row_off);
+#pragma unroll
+  for (int i = 0; i < 4; ++i) {
+    uint32_t wds[4];
+#pragma unroll
+    for (int j = 0; j < 4; ++j) {
+      const int k = 16 * i + 4 * j;
+      wds[j] = static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(f[k], scale), __fdiv_rn(f[k + 1], scale))) |
+               (static_cast<uint32_t>(f32x2_to_e4m3x2(__fdiv_rn(f[k + 2], scale), __fdiv_rn(f[k + 3], scale)))
+                << 16);
+    }
+    dst[i] = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+  }
+  if (threadIdx.x == 0) scales[blk] = scale;
+}
+
+cudaError_t launch_quantize_weights(const void* w, long long batches, int rows, int cols, uint8_t* codes,
+                                    float* scales, cudaStream_t stream) {
+  const long long blocks = batches * (rows / 128) * (cols / 128);
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  quantize_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(w),
+                                                                            rows, cols, codes, scales);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

@@ -1,0 +1,773 @@
+// Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, sm_100a).
+//
+// GEMM1 (gate/up):  h[r, :] = a1[r, :] . w13[e(r)]^T, followed in the epilogue
+//   by a2 = bf16(bf16(silu(gate)) * up) and, on the FP8 path, the per-(row,128)
+//   power-of-two E4M3 re-quantisation (vLLM PR #64760 analysis, §1.2: the
+//   fused SiLU-mul-quant kernel, here fused into the GEMM epilogue so the bf16
+//   intermediate never reaches HBM).
+// GEMM2 (down):     y[flat(r), :] = topk_weight(flat(r)) * a2[r, :] . w2[e(r)]^T,
+//   reading a2 in expert-sorted order with plain TMA tiles (§1.1, sorted-A)
+//   and scattering rows to their flat assignment index.
+//
+// Rows are the expert-sorted, block-padded assignments produced by align; a
+// block of block_m rows belongs to one expert.  Two tile orientations:
+//   normal : MMA M = 128 token rows, N = 256 weight rows (GEMM1: 128 gate +
+//            128 up rows of one 128-column intermediate group);
+//   swap-AB: MMA M = 128 weight rows, N = block_m token rows -- the
+//            orientation the AWS/kinachrichten page ("Swap-AB") describes for
+//            decode batches, where the token count cannot fill the MMA M.
+//
+// Kernel structure (one CTA per SM, persistent over tiles, 10 warps):
+//   warp 0     : TMA producer (one lane), multi-stage smem ring;
+//   warp 1     : TMEM allocator and MMA issuer (one lane);
+//   warps 2..9 : epilogue, two groups of four warps (each group covers the
+//                128 TMEM lanes; the groups split the accumulator columns).
+// bf16: the whole K reduction accumulates in TMEM (double-buffered across
+// tiles).  FP8: weights carry one fp32 scale per 128x128 block and activations
+// one power-of-two scale per (row, 128); every 128-deep K block accumulates
+// into its own TMEM buffer (double-buffered) and the epilogue promotes it into
+// fp32 registers with the product of the two scales.
+#include <cudaTypedefs.h>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+namespace {
+
+constexpr int kThreads = 320;
+constexpr int kEpiWarps = 8;
+constexpr int kSmemLimit = 232448;  // max dynamic shared memory per block on sm_100
+constexpr int kSmemReserve = 4096;  // barriers, TMEM slot, exchange buffers
+constexpr int kXchgOffset = 512;    // exchange buffers start here inside the reserve
+
+// wait-site codes reported in the status word (low byte)
+constexpr int kWhereProducer = 1, kWhereMma = 2, kWhereEpiAcc = 3, kWhereEpiXchg = 4, kWhereDrain = 5;
+
+constexpr int ceil_pow2(int v) {
+  int p = 1;
+  while (p < v) p <<= 1;
+  return p;
+}
+
+template <bool kDown, bool kFP8, bool kSwap, int kBM>
+struct Cfg {
+  static constexpr int kKElems = kFP8 ? 128 : 64;  // K elements per stage (128 bytes per row)
+  static constexpr int kTokRows = kSwap ? kBM : 128;
+  static constexpr int kWRows = (kSwap && kDown) ? 128 : 256;
+  static constexpr int kTokBytes = kTokRows * 128;
+  static constexpr int kWBytes = kWRows * 128;
+  static constexpr int kStageBytes = kTokBytes + kWBytes;
+  static constexpr int kStagesFit = (kSmemLimit - kSmemReserve - 1024) / kStageBytes;
+  static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
+  static constexpr int kMmaN = kSwap ? kBM : 256;
+  static constexpr int kAccCols = kSwap ? (kDown ? kBM : 2 * kBM) : 256;
+  static constexpr int kTmemCols = ceil_pow2((2 * kAccCols) < 32 ? 32 : 2 * kAccCols);
+  // output columns per tile: GEMM1 -> 128 intermediate columns; GEMM2 -> H columns
+  static constexpr int kTileN = kDown ? (kSwap ? 128 : 256) : 128;
+  static constexpr int kHalfTok = kBM / 2;  // swap: token columns per epilogue group
+  static constexpr size_t kSmemBytes = static_cast<size_t>(kStages) * kStageBytes + kSmemReserve + 1024;
+  static_assert(kStages >= 2, "pipeline needs at least two stages");
+  static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
+  static_assert(!kSwap || kBM == 16 || kBM == 32 || kBM == 64, "swap-AB block_m");
+};
+
+struct Args {
+  int E, H, I, nflat, capacity;
+  const int32_t* ntpp;
+  const int32_t* expert_ids;
+  const int32_t* sorted_ids;
+  const float* topk_weights;
+  const float* a_scale_t;  // [K/128, capacity]
+  const float* w_scale;    // [E, Nw/128, K/128]
+  void* out;               // GEMM1: a2 [capacity, I]; GEMM2: y [nflat, H]
+  float* out_scale_t;      // GEMM1 FP8: a2 scale [I/128, capacity]
+  int* status;
+};
+
+__device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
+                                          int where) {
+  const bool ok = mbar_wait(bar, parity, abort, status, MOE_STATUS_WAIT_TIMEOUT | where);
+  return __all_sync(0xffffffffu, ok);
+}
+
+__device__ __forceinline__ void store_bf16x16(__nv_bfloat16* dst, const float (&v)[16]) {
+  uint4 u[2];
+  __nv_bfloat162* h = reinterpret_cast<__nv_bfloat162*>(u);
+#pragma unroll
+  for (int i = 0; i < 8; ++i) h[i] = __floats2bfloat162_rn(v[2 * i], v[2 * i + 1]);
+  reinterpret_cast<uint4*>(dst)[0] = u[0];
+  reinterpret_cast<uint4*>(dst)[1] = u[1];
+}
+
+template <bool kDown, bool kFP8, bool kSwap, int kBM>
+__global__ void __launch_bounds__(kThreads, 1)
+    moe_gemm_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant__ CUtensorMap tm_w,
+                    const Args args) {
+  using C = Cfg<kDown, kFP8, kSwap, kBM>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* reserve = smem + static_cast<size_t>(C::kStages) * C::kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(reserve);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* acc_full = empty + C::kStages;
+  uint64_t* acc_empty = acc_full + 2;
+  uint64_t* xchg_bar = acc_empty + 2;
+  uint64_t* drain = xchg_bar + 2;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+  float* xchg = reinterpret_cast<float*>(reserve + kXchgOffset);  // [2][2 * 128] floats
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    for (int b = 0; b < 2; ++b) {
+      mbar_init(&acc_full[b], 1);
+      mbar_init(&acc_empty[b], kEpiWarps);
+      mbar_init(&xchg_bar[b], kEpiWarps * 32);
+    }
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_tok);
+    tma_prefetch_desc(&tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+
+  const int H = args.H, I = args.I;
+  const int K = kDown ? I : H;                           // reduction length
+  const int rows_per_block = C::kTokRows;                // == block_m of the alignment
+  const int n_tiles = (kDown ? H : I) / C::kTileN;
+  const int num_mblocks = __ldg(args.ntpp) / rows_per_block;
+  const int num_tiles = num_mblocks * n_tiles;
+  const int k_stages = K / C::kKElems;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_a = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      long long fills = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
+        const int e = __ldg(args.expert_ids + mb);
+        const int tok_row = mb * rows_per_block;
+        int w_row0, w_row1;
+        if constexpr (kDown) {
+          w_row0 = e * H + nt * C::kTileN;
+          w_row1 = w_row0;
+        } else {
+          w_row0 = e * 2 * I + nt * 128;      // gate rows
+          w_row1 = w_row0 + I;                // up rows
+        }
+        for (int ks = 0; ks < k_stages; ++ks) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status,
+                         MOE_STATUS_WAIT_TIMEOUT | kWhereProducer)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + static_cast<size_t>(stage) * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          const int kx = ks * C::kKElems;
+          tma_load_2d(st, &tm_tok, &full[stage], kx, tok_row, pol_a);
+          if constexpr (kDown) {
+            tma_load_2d(st + C::kTokBytes, &tm_w, &full[stage], kx, w_row0, pol_w);
+          } else {
+            tma_load_2d(st + C::kTokBytes, &tm_w, &full[stage], kx, w_row0, pol_w);
+            tma_load_2d(st + C::kTokBytes + 16384, &tm_w, &full[stage], kx, w_row1, pol_w);
+          }
+          ++fills;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let every copy already issued land before the CTA tears down
+        for (int s = 0; s < C::kStages; ++s) {
+          const long long n_s = fills / C::kStages + (s < fills % C::kStages ? 1 : 0);
+          if (n_s > 0) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[s], static_cast<uint32_t>((n_s - 1) & 1)) &&
+                   globaltimer_ns() - t0 < kWaitTimeoutNs) {
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      constexpr uint32_t idesc = make_idesc(128, C::kMmaN, kFP8);
+      int stage = 0, abuf = 0;
+      uint32_t phase = 0, aphase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if constexpr (!kFP8) {
+          if (!mbar_wait(&acc_empty[abuf], aphase ^ 1u, abort_flag, args.status,
+                         MOE_STATUS_WAIT_TIMEOUT | kWhereMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+        }
+        for (int ks = 0; ks < k_stages; ++ks) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, args.status, MOE_STATUS_WAIT_TIMEOUT | kWhereMma)) {
+            ok = false;
+            break;
+          }
+          if constexpr (kFP8) {
+            if (!mbar_wait(&acc_empty[abuf], aphase ^ 1u, abort_flag, args.status,
+                           MOE_STATUS_WAIT_TIMEOUT | kWhereMma)) {
+              ok = false;
+              break;
+            }
+          }
+          tc_fence_after();
+          const uint32_t d = tmem_base + static_cast<uint32_t>(abuf * C::kAccCols);
+          const uint32_t tok = smem_u32(smem + static_cast<size_t>(stage) * C::kStageBytes);
+          const uint32_t w = tok + C::kTokBytes;
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t koff = k * 32;  // 16 bf16 or 32 e4m3 elements
+            const uint32_t acc = kFP8 ? (k > 0 ? 1u : 0u) : ((ks > 0 || k > 0) ? 1u : 0u);
+            if constexpr (!kSwap) {
+              const uint64_t ad = smem_desc_sw128(tok + koff), bd = smem_desc_sw128(w + koff);
+              if constexpr (kFP8) mma_fp8(d, ad, bd, idesc, acc); else mma_bf16(d, ad, bd, idesc, acc);
+            } else if constexpr (!kDown) {
+              const uint64_t bd = smem_desc_sw128(tok + koff);
+              const uint64_t ag = smem_desc_sw128(w + koff), au = smem_desc_sw128(w + 16384 + koff);
+              if constexpr (kFP8) {
+                mma_fp8(d, ag, bd, idesc, acc);
+                mma_fp8(d + kBM, au, bd, idesc, acc);
+              } else {
+                mma_bf16(d, ag, bd, idesc, acc);
+                mma_bf16(d + kBM, au, bd, idesc, acc);
+              }
+            } else {
+              const uint64_t ad = smem_desc_sw128(w + koff), bd = smem_desc_sw128(tok + koff);
+              if constexpr (kFP8) mma_fp8(d, ad, bd, idesc, acc); else mma_bf16(d, ad, bd, idesc, acc);
+            }
+          }
+          mma_commit(&empty[stage]);
+          if constexpr (kFP8) {
+            mma_commit(&acc_full[abuf]);
+            abuf ^= 1;
+            if (abuf == 0) aphase ^= 1u;
+          }
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        if constexpr (!kFP8) {
+          mma_commit(&acc_full[abuf]);
+          abuf ^= 1;
+          if (abuf == 0) aphase ^= 1u;
+        }
+      }
+      // every MMA this thread issued has completed once `drain` flips
+      // (waited on even after an abort: TMEM must not be freed under a running MMA)
+      mma_commit(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0)) {
+        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+          report_status(args.status, MOE_STATUS_WAIT_TIMEOUT | kWhereDrain);
+          break;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp & 3;                 // TMEM lane quarter this warp may access
+    const int g = (warp - 2) >> 2;          // epilogue group
+    const int row = 32 * q + lane;          // accumulator row (TMEM lane)
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+    int abuf = 0;
+    uint32_t aphase = 0;
+    int xbuf = 0;
+    uint32_t xphase = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
+      const int e = __ldg(args.expert_ids + mb);
+
+      if constexpr (!kSwap) {
+        // ---------------- normal: row = token row of the tile
+        const int grow = mb * 128 + row;  // sorted row
+        constexpr int kCols = kDown ? 128 : 64;  // accumulator columns per group (per gate/up half for GEMM1)
+        float acc_a[kFP8 ? kCols : 1];
+        float acc_b[(kFP8 && !kDown) ? kCols : 1];
+        if constexpr (kFP8) {
+#pragma unroll
+          for (int i = 0; i < kCols; ++i) acc_a[i] = 0.f;
+          if constexpr (!kDown) {
+#pragma unroll
+            for (int i = 0; i < kCols; ++i) acc_b[i] = 0.f;
+          }
+          const int kb_n = K / 128;
+          const float* sa_p = args.a_scale_t + grow;
+          const float* sw_a;
+          const float* sw_b;
+          if constexpr (kDown) {
+            sw_a = args.w_scale + (static_cast<size_t>(e) * (H / 128) + nt * 2 + g) * kb_n;
+            sw_b = sw_a;
+          } else {
+            sw_a = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + nt) * kb_n;
+            sw_b = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + I / 128 + nt) * kb_n;
+          }
+          float sa_next = __ldg(sa_p);
+          for (int kb = 0; kb < kb_n; ++kb) {
+            const float sa = sa_next;
+            if (kb + 1 < kb_n) sa_next = __ldg(sa_p + static_cast<size_t>(kb + 1) * args.capacity);
+            const float fa = sa * __ldg(sw_a + kb);
+            const float fb = sa * __ldg(sw_b + kb);
+            if (!warp_wait(&acc_full[abuf], aphase, abort_flag, args.status, kWhereEpiAcc)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t t0 = tmem_base + lane_addr + static_cast<uint32_t>(abuf * C::kAccCols);
+            if constexpr (kDown) {
+#pragma unroll
+              for (int c = 0; c < kCols / 16; ++c) {
+                float d[16];
+                tmem_ld16(t0 + g * 128 + 16 * c, d);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) acc_a[16 * c + i] = fmaf(d[i], fa, acc_a[16 * c + i]);
+              }
+            } else {
+#pragma unroll
+              for (int c = 0; c < kCols / 16; ++c) {
+                float dg[16], du[16];
+                tmem_ld16(t0 + g * 64 + 16 * c, dg);
+                tmem_ld16(t0 + 128 + g * 64 + 16 * c, du);
+                tmem_wait_ld();
+#pragma unroll
+                for (int i = 0; i < 16; ++i) {
+                  acc_a[16 * c + i] = fmaf(dg[i], fa, acc_a[16 * c + i]);
+                  acc_b[16 * c + i] = fmaf(du[i], fb, acc_b[16 * c + i]);
+                }
+              }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[abuf]);
+            abuf ^= 1;
+            if (abuf == 0) aphase ^= 1u;
+          }
+          if (!ok) break;
+        }
+
+        if constexpr (!kDown) {
+          // ---- GEMM1 epilogue: SiLU(gate) * up, bf16 store or FP8 requant
+          __nv_bfloat16* a2 = static_cast<__nv_bfloat16*>(args.out);
+          const int col0 = nt * 128 + g * 64;  // intermediate column of this group's first value
+          if constexpr (!kFP8) {
+            if (!warp_wait(&acc_full[abuf], aphase, abort_flag, args.status, kWhereEpiAcc)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t t0 = tmem_base + lane_addr + static_cast<uint32_t>(abuf * C::kAccCols);
+            uint32_t packed[32];
+#pragma unroll
+            for (int c = 0; c < 4; ++c) {
+              float dg[16], du[16];
+              tmem_ld16(t0 + g * 64 + 16 * c, dg);
+              tmem_ld16(t0 + 128 + g * 64 + 16 * c, du);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const float p0 = silu_mul_bf16(bf16_round(dg[2 * i]), bf16_round(du[2 * i]));
+                const float p1 = silu_mul_bf16(bf16_round(dg[2 * i + 1]), bf16_round(du[2 * i + 1]));
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
+                packed[8 * c + i] = *reinterpret_cast<const uint32_t*>(&h2);
+              }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[abuf]);
+            abuf ^= 1;
+            if (abuf == 0) aphase ^= 1u;
+            uint4* dst = reinterpret_cast<uint4*>(a2 + static_cast<size_t>(grow) * I + col0);
+#pragma unroll
+            for (int i = 0; i < 8; ++i)
+              dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+          } else {
+            float amax = 0.f;
+#pragma unroll
+            for (int i = 0; i < 64; ++i) {
+              const float p = silu_mul_bf16(bf16_round(acc_a[i]), bf16_round(acc_b[i]));
+              acc_a[i] = p;
+              amax = fmaxf(amax, fabsf(p));
+            }
+            // the 128-column group spans both epilogue groups: exchange the row maxima
+            float* xb = xchg + xbuf * 256;
+            xb[g * 128 + row] = amax;
+            mbar_arrive(&xchg_bar[xbuf]);
+            if (!warp_wait(&xchg_bar[xbuf], xphase, abort_flag, args.status, kWhereEpiXchg)) {
+              ok = false;
+              break;
+            }
+            amax = fmaxf(xb[row], xb[128 + row]);
+            xbuf ^= 1;
+            if (xbuf == 0) xphase ^= 1u;
+            const float scale = act_scale_from_amax(amax);
+            const float inv = pow2_recip(scale);
+            uint32_t words[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) {
+              words[i] = static_cast<uint32_t>(f32x2_to_e4m3x2(acc_a[4 * i] * inv, acc_a[4 * i + 1] * inv)) |
+                         (static_cast<uint32_t>(f32x2_to_e4m3x2(acc_a[4 * i + 2] * inv, acc_a[4 * i + 3] * inv))
+                          << 16);
+            }
+            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) + static_cast<size_t>(grow) * I +
+                                                  col0);
+#pragma unroll
+            for (int i = 0; i < 4; ++i)
+              dst[i] = make_uint4(words[4 * i], words[4 * i + 1], words[4 * i + 2], words[4 * i + 3]);
+            if (g == 0) args.out_scale_t[static_cast<size_t>(nt) * args.capacity + grow] = scale;
+          }
+        } else {
+          // ---- GEMM2 epilogue: routed weight, scatter the row to y[flat]
+          const int flat = __ldg(args.sorted_ids + grow);
+          const bool real = flat < args.nflat;
+          const float wt = real ? __ldg(args.topk_weights + flat) : 0.f;
+          __nv_bfloat16* yrow =
+              static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(real ? flat : 0) * H + nt * 256 + g * 128;
+          if constexpr (kFP8) {
+            if (real) {
+#pragma unroll
+              for (int c = 0; c < 8; ++c) {
+                float v[16];
+#pragma unroll
+                for (int i = 0; i < 16; ++i) v[i] = acc_a[16 * c + i] * wt;
+                store_bf16x16(yrow + 16 * c, v);
+              }
+            }
+          } else {
+            if (!warp_wait(&acc_full[abuf], aphase, abort_flag, args.status, kWhereEpiAcc)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t t0 = tmem_base + lane_addr + static_cast<uint32_t>(abuf * C::kAccCols);
+            uint32_t packed[64];
+#pragma unroll
+            for (int c = 0; c < 8; ++c) {
+              float d[16];
+              tmem_ld16(t0 + g * 128 + 16 * c, d);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                const __nv_bfloat162 h2 = __floats2bfloat162_rn(d[2 * i] * wt, d[2 * i + 1] * wt);
+                packed[8 * c + i] = *reinterpret_cast<const uint32_t*>(&h2);
+              }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[abuf]);
+            abuf ^= 1;
+            if (abuf == 0) aphase ^= 1u;
+            if (real) {
+              uint4* dst = reinterpret_cast<uint4*>(yrow);
+#pragma unroll
+              for (int i = 0; i < 16; ++i)
+                dst[i] = make_uint4(packed[4 * i], packed[4 * i + 1], packed[4 * i + 2], packed[4 * i + 3]);
+            }
+          }
+        }
+      } else {
+        // ---------------- swap-AB: row = weight row of the tile, columns = token rows
+        constexpr int kHT = C::kHalfTok;           // token columns of this group
+        const int tok0 = mb * kBM + g * kHT;       // first sorted row of this group
+        float acc_a[kHT];                          // gate (GEMM1) or down (GEMM2)
+        float acc_b[kDown ? 1 : kHT];              // up (GEMM1)
+        // column offsets of this group's values inside one accumulator buffer
+        const uint32_t col_a = static_cast<uint32_t>(g * kHT);
+        const uint32_t col_b = static_cast<uint32_t>(kBM + g * kHT);
+        if constexpr (kFP8) {
+#pragma unroll
+          for (int j = 0; j < kHT; ++j) acc_a[j] = 0.f;
+          if constexpr (!kDown) {
+#pragma unroll
+            for (int j = 0; j < kHT; ++j) acc_b[j] = 0.f;
+          }
+          const int kb_n = K / 128;
+          const float* sw_a;
+          const float* sw_b;
+          if constexpr (kDown) {
+            sw_a = args.w_scale + (static_cast<size_t>(e) * (H / 128) + nt) * kb_n;
+            sw_b = sw_a;
+          } else {
+            sw_a = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + nt) * kb_n;
+            sw_b = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + I / 128 + nt) * kb_n;
+          }
+          for (int kb = 0; kb < kb_n; ++kb) {
+            const float swa = __ldg(sw_a + kb);
+            const float swb = __ldg(sw_b + kb);
+            const float* sa_p = args.a_scale_t + static_cast<size_t>(kb) * args.capacity + tok0;
+            float fa[kHT];
+#pragma unroll
+            for (int j = 0; j < kHT; ++j) fa[j] = __ldg(sa_p + j);
+            if (!warp_wait(&acc_full[abuf], aphase, abort_flag, args.status, kWhereEpiAcc)) {
+              ok = false;
+              break;
+            }
+            tc_fence_after();
+            const uint32_t t0 = tmem_base + lane_addr + static_cast<uint32_t>(abuf * C::kAccCols);
+#pragma unroll
+            for (int c = 0; c < kHT / 8; ++c) {
+              float da[8], db[8];
+              tmem_ld8(t0 + col_a + 8 * c, da);
+              if constexpr (!kDown) tmem_ld8(t0 + col_b + 8 * c, db);
+              tmem_wait_ld();
+#pragma unroll
+              for (int i = 0; i < 8; ++i) {
+                acc_a[8 * c + i] = fmaf(da[i], fa[8 * c + i] * swa, acc_a[8 * c + i]);
+                if constexpr (!kDown) acc_b[8 * c + i] = fmaf(db[i], fa[8 * c + i] * swb, acc_b[8 * c + i]);
+              }
+            }
+            tc_fence_before();
+            __syncwarp();
+            if (lane == 0) mbar_arrive(&acc_empty[abuf]);
+            abuf ^= 1;
+            if (abuf == 0) aphase ^= 1u;
+          }
+          if (!ok) break;
+        } else {
+          if (!warp_wait(&acc_full[abuf], aphase, abort_flag, args.status, kWhereEpiAcc)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t t0 = tmem_base + lane_addr + static_cast<uint32_t>(abuf * C::kAccCols);
+#pragma unroll
+          for (int c = 0; c < kHT / 8; ++c) {
+            float da[8], db[8];
+            tmem_ld8(t0 + col_a + 8 * c, da);
+            if constexpr (!kDown) tmem_ld8(t0 + col_b + 8 * c, db);
+            tmem_wait_ld();
+#pragma unroll
+            for (int i = 0; i < 8; ++i) {
+              acc_a[8 * c + i] = da[i];
+              if constexpr (!kDown) acc_b[8 * c + i] = db[i];
+            }
+          }
+          tc_fence_before();
+          __syncwarp();
+          if (lane == 0) mbar_arrive(&acc_empty[abuf]);
+          abuf ^= 1;
+          if (abuf == 0) aphase ^= 1u;
+        }
+
+        if constexpr (!kDown) {
+          // ---- GEMM1: this thread owns intermediate column nt*128 + row for kHT tokens
+          const int icol = nt * 128 + row;
+#pragma unroll
+          for (int j = 0; j < kHT; ++j) acc_a[j] = silu_mul_bf16(bf16_round(acc_a[j]), bf16_round(acc_b[j]));
+          if constexpr (!kFP8) {
+            __nv_bfloat16* a2 = static_cast<__nv_bfloat16*>(args.out);
+#pragma unroll
+            for (int j = 0; j < kHT; ++j) a2[static_cast<size_t>(tok0 + j) * I + icol] = __float2bfloat16_rn(acc_a[j]);
+          } else {
+            // amax of each token over the 128 columns: warp butterfly, then the 4 warps of the group
+            float* xb = xchg + xbuf * 256;  // [group][quarter][kHT]
+#pragma unroll
+            for (int j = 0; j < kHT; ++j) {
+              float m = fabsf(acc_a[j]);
+#pragma unroll
+              for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+              if (lane == 0) xb[(g * 4 + q) * kHT + j] = m;
+            }
+            mbar_arrive(&xchg_bar[xbuf]);
+            if (!warp_wait(&xchg_bar[xbuf], xphase, abort_flag, args.status, kWhereEpiXchg)) {
+              ok = false;
+              break;
+            }
+            uint8_t* a2 = static_cast<uint8_t*>(args.out);
+#pragma unroll
+            for (int j = 0; j < kHT; ++j) {
+              float m = xb[(g * 4 + 0) * kHT + j];
+              m = fmaxf(m, xb[(g * 4 + 1) * kHT + j]);
+              m = fmaxf(m, xb[(g * 4 + 2) * kHT + j]);
+              m = fmaxf(m, xb[(g * 4 + 3) * kHT + j]);
+              const float scale = act_scale_from_amax(m);
+              const float v = acc_a[j] * pow2_recip(scale);
+              a2[static_cast<size_t>(tok0 + j) * I + icol] =
+                  static_cast<uint8_t>(f32x2_to_e4m3x2(v, 0.f) & 0xFFu);
+              if (row == 0) args.out_scale_t[static_cast<size_t>(nt) * args.capacity + tok0 + j] = scale;
+            }
+            xbuf ^= 1;
+            if (xbuf == 0) xphase ^= 1u;
+          }
+        } else {
+          // ---- GEMM2: this thread owns H column nt*128 + row for kHT tokens
+          __nv_bfloat16* y = static_cast<__nv_bfloat16*>(args.out);
+          const int hcol = nt * 128 + row;
+#pragma unroll
+          for (int j = 0; j < kHT; ++j) {
+            const int flat = __ldg(args.sorted_ids + tok0 + j);
+            if (flat < args.nflat) {
+              const float wt = __ldg(args.topk_weights + flat);
+              y[static_cast<size_t>(flat) * H + hcol] = __float2bfloat16_rn(acc_a[j] * wt);
+            }
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// host side
+// ----------------------------------------------------------------------------
+PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
+  static PFN_cuTensorMapEncodeTiled_v12000 fn = nullptr;
+  if (fn == nullptr) {
+    void* p = nullptr;
+    cudaDriverEntryPointQueryResult q;
+    if (cudaGetDriverEntryPoint("cuTensorMapEncodeTiled", &p, cudaEnableDefault, &q) == cudaSuccess &&
+        q == cudaDriverEntryPointSuccess)
+      fn = reinterpret_cast<PFN_cuTensorMapEncodeTiled_v12000>(p);
+  }
+  return fn;
+}
+
+// 2-D K-major tensor map: [rows, cols] elements of `elem_bytes`, box = 128 bytes x box_rows, 128-byte swizzle
+bool make_map(CUtensorMap* map, const void* base, long long rows, long long cols, int elem_bytes, int box_rows) {
+  auto fn = encode_fn();
+  if (fn == nullptr) return false;
+  const CUtensorMapDataType dt =
+      elem_bytes == 2 ? CU_TENSOR_MAP_DATA_TYPE_BFLOAT16 : CU_TENSOR_MAP_DATA_TYPE_UINT8;
+  cuuint64_t dims[2] = {static_cast<cuuint64_t>(cols), static_cast<cuuint64_t>(rows)};
+  cuuint64_t strides[1] = {static_cast<cuuint64_t>(cols) * elem_bytes};
+  cuuint32_t box[2] = {static_cast<cuuint32_t>(128 / elem_bytes), static_cast<cuuint32_t>(box_rows)};
+  cuuint32_t estr[2] = {1, 1};
+  const CUresult r = fn(map, dt, 2, const_cast<void*>(base), dims, strides, box, estr, CU_TENSOR_MAP_INTERLEAVE_NONE,
+                        CU_TENSOR_MAP_SWIZZLE_128B, CU_TENSOR_MAP_L2_PROMOTION_L2_256B,
+                        CU_TENSOR_MAP_FLOAT_OOB_FILL_NONE);
+  return r == CUDA_SUCCESS;
+}
+
+template <bool kDown, bool kFP8, bool kSwap, int kBM>
+cudaError_t launch_on(const GemmProblem& p, const void* tok, const void* w, const Args& args, cudaStream_t s) {
+  using C = Cfg<kDown, kFP8, kSwap, kBM>;
+  auto kern = moe_gemm_kernel<kDown, kFP8, kSwap, kBM>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(C::kSmemBytes));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const int elem = kFP8 ? 1 : 2;
+  const long long K = kDown ? p.I : p.H;
+  const long long wrows = kDown ? static_cast<long long>(p.E) * p.H : static_cast<long long>(p.E) * 2 * p.I;
+  CUtensorMap tm_tok, tm_w;
+  if (!make_map(&tm_tok, tok, p.capacity, K, elem, C::kTokRows)) return cudaErrorInvalidValue;
+  if (!make_map(&tm_w, w, wrows, K, elem, kDown ? C::kWRows : 128)) return cudaErrorInvalidValue;
+  const int n_tiles = (kDown ? p.H : p.I) / C::kTileN;
+  const long long max_tiles = static_cast<long long>(p.capacity / C::kTokRows) * n_tiles;
+  int grid = p.num_sms;
+  if (max_tiles < grid) grid = static_cast<int>(max_tiles);
+  if (grid <= 0) return cudaSuccess;
+  kern<<<grid, kThreads, C::kSmemBytes, s>>>(tm_tok, tm_w, args);
+  return cudaGetLastError();
+}
+
+template <bool kDown, bool kFP8>
+cudaError_t dispatch(const GemmProblem& p, const void* tok, const void* w, const Args& args, cudaStream_t s) {
+  if (!p.swap) return launch_on<kDown, kFP8, false, 128>(p, tok, w, args, s);
+  switch (p.block_m) {
+    case 16: return launch_on<kDown, kFP8, true, 16>(p, tok, w, args, s);
+    case 32: return launch_on<kDown, kFP8, true, 32>(p, tok, w, args, s);
+    case 64: return launch_on<kDown, kFP8, true, 64>(p, tok, w, args, s);
+    default: return cudaErrorInvalidValue;
+  }
+}
+
+template <bool kDown, bool kFP8, bool kSwap, int kBM>
+size_t smem_of() {
+  return Cfg<kDown, kFP8, kSwap, kBM>::kSmemBytes;
+}
+
+}  // namespace
+
+cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const float* a1_scale_t, const void* w13,
+                         const float* w13_scale, void* a2, float* a2_scale_t, cudaStream_t stream) {
+  Args args{};
+  args.E = p.E;
+  args.H = p.H;
+  args.I = p.I;
+  args.nflat = p.nflat;
+  args.capacity = p.capacity;
+  args.ntpp = p.ntpp;
+  args.expert_ids = p.expert_ids;
+  args.sorted_ids = p.sorted_ids;
+  args.topk_weights = p.topk_weights;
+  args.a_scale_t = a1_scale_t;
+  args.w_scale = w13_scale;
+  args.out = a2;
+  args.out_scale_t = a2_scale_t;
+  args.status = p.status;
+  return p.fp8 ? dispatch<false, true>(p, a1, w13, args, stream) : dispatch<false, false>(p, a1, w13, args, stream);
+}
+
+cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const float* a2_scale_t, const void* w2,
+                         const float* w2_scale, void* y, cudaStream_t stream) {
+  Args args{};
+  args.E = p.E;
+  args.H = p.H;
+  args.I = p.I;
+  args.nflat = p.nflat;
+  args.capacity = p.capacity;
+  args.ntpp = p.ntpp;
+  args.expert_ids = p.expert_ids;
+  args.sorted_ids = p.sorted_ids;
+  args.topk_weights = p.topk_weights;
+  args.a_scale_t = a2_scale_t;
+  args.w_scale = w2_scale;
+  args.out = y;
+  args.out_scale_t = nullptr;
+  args.status = p.status;
+  return p.fp8 ? dispatch<true, true>(p, a2, w2, args, stream) : dispatch<true, false>(p, a2, w2, args, stream);
+}
+
+size_t gemm_smem_bytes(bool gemm2, bool fp8, bool swap, int block_m) {
+  if (!swap) {
+    if (gemm2) return fp8 ? smem_of<true, true, false, 128>() : smem_of<true, false, false, 128>();
+    return fp8 ? smem_of<false, true, false, 128>() : smem_of<false, false, false, 128>();
+  }
+  return 0;
+}
+
+}  // namespace moe

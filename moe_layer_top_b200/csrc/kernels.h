@@ -1,0 +1,58 @@
+// Host-side launchers of the MoE kernels (internal to the library).
+#pragma once
+
+#include <cuda_runtime.h>
+#include <stdint.h>
+#include <stddef.h>
+
+namespace moe {
+
+// router ---------------------------------------------------------------------
+cudaError_t launch_route(const float* logits, int T, int E, int topk, int renormalize, int32_t* ids,
+                         float* weights, cudaStream_t stream);
+
+// align ----------------------------------------------------------------------
+constexpr int kAlignChunk = 256;  // assignments per warp-chunk
+inline int align_chunks(long long n) { return static_cast<int>((n + kAlignChunk - 1) / kAlignChunk); }
+
+cudaError_t launch_align(const int32_t* topk_ids, int n, int E, int block_m, int capacity,
+                         int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp, int32_t* counts_ws,
+                         int32_t* offsets_ws, int32_t* chunk_scratch, int32_t* user_counts,
+                         int32_t* user_offsets, int* status, cudaStream_t stream);
+
+// gather x rows into sorted order (bf16 copy, or FP8 per-(row,128) quantisation)
+cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32_t* sorted_ids,
+                          const int32_t* ntpp, int capacity, bool fp8, void* a1, float* a1_scale_t,
+                          cudaStream_t stream);
+
+// out[t] = sum_j y[t*topk + j]
+cudaError_t launch_combine(const void* y, int T, int topk, int H, void* out, cudaStream_t stream);
+
+// FP8 128x128 block weight quantisation
+cudaError_t launch_quantize_weights(const void* w, long long batches, int rows, int cols, uint8_t* codes,
+                                    float* scales, cudaStream_t stream);
+
+// grouped GEMMs ----------------------------------------------------------------
+struct GemmProblem {
+  int E, H, I, topk, nflat, block_m, capacity;
+  bool fp8, swap;
+  const int32_t* ntpp;
+  const int32_t* expert_ids;
+  const int32_t* sorted_ids;
+  const float* topk_weights;  // [nflat]
+  int* status;
+  int num_sms;
+};
+
+// GEMM1 + fused SiLU*up (+ FP8 requant): a1 [cap, H] -> a2 [cap, I] (+ a2_scale_t [I/128, cap])
+cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const float* a1_scale_t, const void* w13,
+                         const float* w13_scale, void* a2, float* a2_scale_t, cudaStream_t stream);
+
+// GEMM2 + routed weight: a2 [cap, I] -> y [nflat, H] bf16 (rows scattered by sorted_ids)
+cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const float* a2_scale_t, const void* w2,
+                         const float* w2_scale, void* y, cudaStream_t stream);
+
+// shared-memory bytes the GEMM variant needs (for validation / occupancy)
+size_t gemm_smem_bytes(bool gemm2, bool fp8, bool swap, int block_m);
+
+}  // namespace moe

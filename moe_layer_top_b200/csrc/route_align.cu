@@ -1,0 +1,324 @@
+// Router and expert alignment kernels.
+//
+// Router ("Warum MoE-Kernel so wichtig sind", AWS/kinachrichten page: token
+// routing): one warp per token, the E logits spread over the lanes; k rounds
+// of a warp-wide argmax pick the experts (descending logit, lower index on
+// ties); softmax statistics come from butterfly reductions, so the result is
+// bitwise reproducible.
+//
+// Alignment (vLLM PR #64760 analysis, §1.1: sorted_token_ids,
+// num_tokens_post_padded, BLOCK_SIZE_M-padded expert runs): a counting sort
+// of the flat assignments t*topk + j by expert in three passes --
+//   1. per warp-chunk of 256 assignments, an expert histogram (shared-memory
+//      atomics; counts are order independent);
+//   2. per expert, an exclusive scan of its chunk counts (chunk order);
+//   3. per warp-chunk, a stable scatter: the rank of an assignment among the
+//      earlier ones of its expert inside the chunk comes from __match_any_sync
+//      over 32 lanes plus a per-warp running counter, so the sorted order is
+//      ascending flat order inside every expert, whatever the scheduling.
+// Padding slots, the tail past num_tokens_post_padded and the per-block
+// expert ids are filled by the same third pass.
+#include <climits>
+
+#include "common.cuh"
+#include "kernels.h"
+
+namespace moe {
+
+// ----------------------------------------------------------------------------
+// router
+// ----------------------------------------------------------------------------
+template <int VPL>  // logits per lane (E <= 32 * VPL)
+__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int topk,
+                                                    int renormalize, int32_t* __restrict__ ids,
+                                                    float* __restrict__ weights) {
+  const int lane = threadIdx.x & 31;
+  const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (tok >= T) return;
+  const float* row = logits + static_cast<size_t>(tok) * E;
+
+  float v[VPL];
+  uint32_t taken = 0;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) {
+    const int e = lane + 32 * i;
+    v[i] = (e < E) ? __ldg(row + e) : -INFINITY;
+    if (e >= E) taken |= 1u << i;
+  }
+  // softmax statistics over all experts
+  float m = -INFINITY;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i)
+    if (!((taken >> i) & 1u)) m = fmaxf(m, v[i]);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  float z = 0.f;
+#pragma unroll
+  for (int i = 0; i < VPL; ++i)
+    if (!((taken >> i) & 1u)) z += expf(v[i] - m);
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
+
+  // k rounds of warp argmax; lane r keeps the r-th choice
+  float my_logit = 0.f;
+  int my_id = -1;
+  for (int r = 0; r < topk; ++r) {
+    float best = -INFINITY;
+    int bi = INT_MAX;
+#pragma unroll
+    for (int i = 0; i < VPL; ++i) {
+      if ((taken >> i) & 1u) continue;
+      if (bi == INT_MAX || v[i] > best) {  // ascending index inside a lane: strict > keeps the lower one
+        best = v[i];
+        bi = lane + 32 * i;
+      }
+    }
+#pragma unroll
+    for (int off = 16; off > 0; off >>= 1) {
+      const float ob = __shfl_xor_sync(0xffffffffu, best, off);
+      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
+      if (oi != INT_MAX && (bi == INT_MAX || ob > best || (ob == best && oi < bi))) {
+        best = ob;
+        bi = oi;
+      }
+    }
+    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
+    if (lane == r) {
+      my_logit = best;
+      my_id = bi;
+    }
+  }
+  const float ex = (lane < topk) ? expf(my_logit - m) : 0.f;
+  float s = ex;
+#pragma unroll
+  for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  if (lane < topk) {
+    const size_t o = static_cast<size_t>(tok) * topk + lane;
+    ids[o] = my_id;
+    weights[o] = renormalize ? __fdiv_rn(ex, s) : __fdiv_rn(ex, z);
+  }
+}
+
+cudaError_t launch_route(const float* logits, int T, int E, int topk, int renormalize, int32_t* ids,
+                         float* weights, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const int threads = 256;
+  const int blocks = static_cast<int>((static_cast<long long>(T) * 32 + threads - 1) / threads);
+  if (E <= 128)
+    route_kernel<4><<<blocks, threads, 0, stream>>>(logits, T, E, topk, renormalize, ids, weights);
+  else if (E <= 256)
+    route_kernel<8><<<blocks, threads, 0, stream>>>(logits, T, E, topk, renormalize, ids, weights);
+  else if (E <= 512)
+    route_kernel<16><<<blocks, threads, 0, stream>>>(logits, T, E, topk, renormalize, ids, weights);
+  else
+    route_kernel<32><<<blocks, threads, 0, stream>>>(logits, T, E, topk, renormalize, ids, weights);
+  return cudaGetLastError();
+}
+
+// ----------------------------------------------------------------------------
+// align pass 1: per-chunk expert histograms
+// ----------------------------------------------------------------------------
+constexpr int kAlignWarps = 8;
+
+__global__ void __launch_bounds__(kAlignWarps * 32) align_count_kernel(const int32_t* __restrict__ ids, int n,
+                                                                       int E, int nchunks,
+                                                                       int32_t* __restrict__ chunk_counts,
+                                                                       int* status) {
+  extern __shared__ int32_t hist_all[];
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  const int chunk = blockIdx.x * kAlignWarps + warp;
+  if (chunk >= nchunks) return;
+  int32_t* hist = hist_all + warp * E;
+  for (int e = lane; e < E; e += 32) hist[e] = 0;
+  __syncwarp();
+  const int base = chunk * kAlignChunk;
+  for (int i = lane; i < kAlignChunk; i += 32) {
+    const int f = base + i;
+    if (f < n) {
+      const int e = __ldg(ids + f);
+      if (e >= 0 && e < E)
+        atomicAdd(&hist[e], 1);
+      else
+        report_status(status, MOE_STATUS_BAD_EXPERT_ID);
+    }
+  }
+  __syncwarp();
+  int32_t* out = chunk_counts + static_cast<size_t>(chunk) * E;
+  for (int e = lane; e < E; e += 32) out[e] = hist[e];
+}
+
+// ----------------------------------------------------------------------------
+// align pass 2: per expert, exclusive scan over chunks (in place) and total
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) align_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
+                                                         int32_t* __restrict__ counts_ws,
+                                                         int32_t* __restrict__ user_counts) {
+  __shared__ int32_t warp_sums[8];
+  const int e = blockIdx.x;
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+  int32_t carry = 0;
+  for (int c0 = 0; c0 < nchunks; c0 += 256) {
+    const int c = c0 + threadIdx.x;
+    const int32_t v = (c < nchunks) ? chunk_counts[static_cast<size_t>(c) * E + e] : 0;
+    int32_t incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int32_t before = 0, tile_total = 0;
+#pragma unroll
+    for (int w = 0; w < 8; ++w) {
+      const int32_t s = warp_sums[w];
+      if (w < warp) before += s;
+      tile_total += s;
+    }
+    if (c < nchunks) chunk_counts[static_cast<size_t>(c) * E + e] = carry + before + incl - v;
+    carry += tile_total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) {
+    counts_ws[e] = carry;
+    if (user_counts) user_counts[e] = carry;
+  }
+}
+
+// ----------------------------------------------------------------------------
+// align pass 3: stable scatter, padding, block expert ids
+// ----------------------------------------------------------------------------
+__device__ __forceinline__ int owner_expert(const int32_t* offs, int E, int p) {
+  // largest e with offs[e] <= p (offs non-decreasing, offs[0] = 0)
+  int lo = 0, hi = E;  // invariant: offs[lo] <= p, answer in [lo, hi)
+  while (hi - lo > 1) {
+    const int mid = (lo + hi) >> 1;
+    if (offs[mid] <= p)
+      lo = mid;
+    else
+      hi = mid;
+  }
+  return lo;
+}
+
+__global__ void __launch_bounds__(kAlignWarps * 32) align_scatter_kernel(
+    const int32_t* __restrict__ ids, int n, int E, int block_m, int capacity, int nchunks,
+    const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ counts_ws, int32_t* __restrict__ sorted_ids,
+    int32_t* __restrict__ expert_ids, int32_t* __restrict__ ntpp_out, int32_t* __restrict__ offsets_ws,
+    int32_t* __restrict__ user_offsets) {
+  extern __shared__ int32_t smem_i32[];
+  int32_t* offs = smem_i32;                    // [E + 1]
+  int32_t* cnt = offs + (E + 1);               // [E]
+  int32_t* running = cnt + E;                  // [kAlignWarps][E]
+  __shared__ int32_t warp_sums[kAlignWarps];
+  const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
+
+  // padded offsets: exclusive scan of round_up(count, block_m) over experts
+  int32_t carry = 0;
+  for (int e0 = 0; e0 < E; e0 += blockDim.x) {
+    const int e = e0 + threadIdx.x;
+    const int32_t c = (e < E) ? counts_ws[e] : 0;
+    if (e < E) cnt[e] = c;
+    const int32_t v = (c + block_m - 1) / block_m * block_m;
+    int32_t incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int32_t before = 0, tile_total = 0;
+    for (int w = 0; w < kAlignWarps; ++w) {
+      const int32_t s = warp_sums[w];
+      if (w < warp) before += s;
+      tile_total += s;
+    }
+    if (e < E) offs[e] = carry + before + incl - v;
+    carry += tile_total;
+    __syncthreads();
+  }
+  if (threadIdx.x == 0) offs[E] = carry;
+  __syncthreads();
+  const int ntpp = offs[E];
+  if (blockIdx.x == 0) {
+    for (int e = threadIdx.x; e <= E; e += blockDim.x) {
+      offsets_ws[e] = offs[e];
+      if (user_offsets) user_offsets[e] = offs[e];
+    }
+    if (threadIdx.x == 0) *ntpp_out = ntpp;
+  }
+
+  // stable scatter of this block's warp-chunks
+  const int chunk = blockIdx.x * kAlignWarps + warp;
+  if (chunk < nchunks) {
+    int32_t* run = running + warp * E;
+    for (int e = lane; e < E; e += 32) run[e] = 0;
+    __syncwarp();
+    const int32_t* cb = chunk_base + static_cast<size_t>(chunk) * E;
+    const int base = chunk * kAlignChunk;
+    for (int i0 = 0; i0 < kAlignChunk; i0 += 32) {
+      const int f = base + i0 + lane;
+      int e = -1;
+      if (f < n) {
+        e = __ldg(ids + f);
+        if (e < 0 || e >= E) e = -1;  // reported by pass 1; never indexed
+      }
+      const uint32_t same = __match_any_sync(0xffffffffu, e);
+      const uint32_t lower = same & ((1u << lane) - 1u);
+      const int rank = __popc(lower);
+      int dest = -1;
+      if (e >= 0) dest = offs[e] + cb[e] + run[e] + rank;
+      __syncwarp();
+      if (e >= 0) {
+        sorted_ids[dest] = f;
+        if (lower == 0) run[e] += __popc(same);  // one lane per expert group updates the counter
+      }
+      __syncwarp();
+    }
+  }
+
+  // sentinel in padding and tail; expert of every block
+  const int stride = gridDim.x * blockDim.x;
+  for (int p = blockIdx.x * blockDim.x + threadIdx.x; p < capacity; p += stride) {
+    bool pad = true;
+    if (p < ntpp) {
+      const int e = owner_expert(offs, E, p);
+      pad = p >= offs[e] + cnt[e];
+    }
+    if (pad) sorted_ids[p] = n;
+  }
+  const int nblocks = capacity / block_m;
+  for (int b = blockIdx.x * blockDim.x + threadIdx.x; b < nblocks; b += stride) {
+    const int p = b * block_m;
+    expert_ids[b] = (p < ntpp) ? owner_expert(offs, E, p) : -1;
+  }
+}
+
+cudaError_t launch_align(const int32_t* topk_ids, int n, int E, int block_m, int capacity, int32_t* sorted_ids,
+                         int32_t* expert_ids, int32_t* ntpp, int32_t* counts_ws, int32_t* offsets_ws,
+                         int32_t* chunk_scratch, int32_t* user_counts, int32_t* user_offsets, int* status,
+                         cudaStream_t stream) {
+  const int nchunks = align_chunks(n);
+  if (nchunks == 0) return cudaSuccess;
+  const int threads = kAlignWarps * 32;
+  const int blocks = (nchunks + kAlignWarps - 1) / kAlignWarps;
+  const size_t smem1 = static_cast<size_t>(kAlignWarps) * E * sizeof(int32_t);
+  align_count_kernel<<<blocks, threads, smem1, stream>>>(topk_ids, n, E, nchunks, chunk_scratch, status);
+  cudaError_t err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  align_scan_kernel<<<E, 256, 0, stream>>>(chunk_scratch, nchunks, E, counts_ws, user_counts);
+  err = cudaGetLastError();
+  if (err != cudaSuccess) return err;
+  const size_t smem3 = (static_cast<size_t>(E + 1) + E + static_cast<size_t>(kAlignWarps) * E) * sizeof(int32_t);
+  int blocks3 = blocks;
+  const int fill_blocks = (capacity + threads * 4 - 1) / (threads * 4);
+  if (fill_blocks > blocks3) blocks3 = fill_blocks < 296 ? fill_blocks : 296;
+  if (blocks3 < blocks) blocks3 = blocks;
+  align_scatter_kernel<<<blocks3, threads, smem3, stream>>>(topk_ids, n, E, block_m, capacity, nchunks,
+                                                            chunk_scratch, counts_ws, sorted_ids, expert_ids, ntpp,
+                                                            offsets_ws, user_offsets);
+  return cudaGetLastError();
+}
+
+}  // namespace moe

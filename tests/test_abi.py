@@ -1,0 +1,141 @@
+"""The C-ABI library loads, exports every symbol the header declares, and
+rejects bad arguments on the host before touching the device (no GPU needed)."""
+
+import ctypes
+import os
+import re
+
+import pytest
+
+from moe_layer_top_b200 import ops
+
+ROOT = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+HEADER = os.path.join(ROOT, "include", "moe_b200.h")
+
+
+def _declared():
+    with open(HEADER) as f:
+        text = f.read()
+    return sorted(set(re.findall(r"^MOE_API\s+[\w\s\*]+?\b(moe_\w+)\(", text, flags=re.M)))
+
+
+@pytest.fixture(scope="module")
+def L():
+    if not os.path.exists(ops.library_path()):
+        from moe_layer_top_b200 import build
+        build.build()
+    return ops.lib()
+
+
+def test_header_declares_the_boundary():
+    names = _declared()
+    for required in ("moe_route", "moe_align_capacity", "moe_align", "moe_workspace_size", "moe_fused_forward"):
+        assert required in names
+    assert set(names) == set(ops.EXPORTED)
+
+
+def test_library_exports_every_declared_symbol(L):
+    for name in _declared():
+        assert hasattr(L, name), name
+    assert L.moe_version() == 100
+
+
+def test_struct_sizes_match_header():
+    assert ctypes.sizeof(ops.MoeProblem) == 16 * 4
+    assert ctypes.sizeof(ops.MoeWorkspaceLayout) == 15 * 8 + 4 * 4
+
+
+def test_align_capacity_formula(L):
+    assert ops.align_capacity(1, 8, 128, 16) == 128
+    assert ops.align_capacity(0, 8, 128, 16) == 0
+    assert ops.align_capacity(16, 2, 8, 128) == 128 * ((32 + 8 * 127 + 127) // 128)
+    assert L.moe_align_capacity(-1, 8, 128, 16) == -1
+    from oracle import moe_oracle as O
+    for args in [(1, 8, 128, 16), (64, 8, 128, 16), (256, 8, 128, 32), (16384, 8, 128, 128), (37, 3, 5, 64)]:
+        assert ops.align_capacity(*args) == O.align_capacity(*args)
+
+
+def test_resolve_problem_auto_modes(L):
+    q = ops.resolve_problem(ops.problem(1, 128, 8, 4096, 1536))
+    assert q.mode == ops.MODE_SWAP_AB and q.block_m == 16
+    q = ops.resolve_problem(ops.problem(16384, 128, 8, 4096, 1536, fp8=True))
+    assert q.mode == ops.MODE_NORMAL and q.block_m == 128
+    q = ops.resolve_problem(ops.problem(64, 128, 8, 4096, 1536, mode=ops.MODE_NORMAL))
+    assert q.block_m == 128
+    q = ops.resolve_problem(ops.problem(64, 128, 8, 4096, 1536, block_m=32))
+    assert q.mode == ops.MODE_SWAP_AB and q.block_m == 32
+
+
+@pytest.mark.parametrize("bad", [
+    dict(T=-1), dict(E=0), dict(E=2000), dict(topk=0), dict(topk=9, E=8), dict(H=100), dict(I=0), dict(I=200),
+    dict(mode=7), dict(mode=ops.MODE_NORMAL, block_m=16), dict(mode=ops.MODE_SWAP_AB, block_m=128),
+    dict(block_m=48),
+])
+def test_invalid_problems_are_rejected(L, bad):
+    kw = dict(T=16, E=8, topk=2, H=256, I=128)
+    kw.update(bad)
+    p = ops.problem(kw["T"], kw["E"], kw["topk"], kw["H"], kw["I"], mode=kw.get("mode", 0),
+                    block_m=kw.get("block_m", 0))
+    assert L.moe_workspace_size(ctypes.byref(p)) == 0
+    with pytest.raises(ops.MoeError) as ei:
+        ops.resolve_problem(p)
+    assert ei.value.code == ops.MOE_ERR_INVALID
+
+
+def test_workspace_layout_is_aligned_and_ordered(L):
+    for fp8 in (False, True):
+        p = ops.problem(64, 128, 8, 4096, 1536, fp8=fp8)
+        lay = ops.workspace_layout(p)
+        offs = [lay.status, lay.topk_ids, lay.topk_weights, lay.sorted_token_ids, lay.expert_ids,
+                lay.num_tokens_post_padded, lay.expert_counts, lay.expert_offsets, lay.align_scratch, lay.a1,
+                lay.a2, lay.y]
+        assert all(o % 256 == 0 for o in offs)
+        assert offs == sorted(offs)
+        assert (lay.a1_scale >= 0) == fp8 and (lay.a2_scale >= 0) == fp8
+        assert lay.total_bytes == ops.workspace_size(p)
+        assert lay.y + 64 * 8 * 4096 * 2 <= lay.total_bytes
+
+
+def _fake(addr):
+    return ctypes.c_void_p(addr)
+
+
+def test_forward_argument_errors_before_any_launch(L):
+    p = ops.problem(16, 8, 2, 256, 128)
+    need = ops.workspace_size(p)
+    good = _fake(1 << 20)
+    args = lambda **o: [ctypes.byref(p), o.get("x", good), o.get("logits", good), None, None,
+                        o.get("w13", good), o.get("w2", good), None, None, o.get("out", good), o.get("ws", good),
+                        o.get("nbytes", need), None]
+    assert L.moe_fused_forward(*args(x=None)) == ops.MOE_ERR_INVALID
+    assert L.moe_fused_forward(*args(logits=None)) == ops.MOE_ERR_INVALID        # no routing input at all
+    assert L.moe_fused_forward(*args(x=_fake((1 << 20) + 8))) == ops.MOE_ERR_INVALID   # misaligned
+    assert L.moe_fused_forward(*args(ws=_fake((1 << 20) + 16))) == ops.MOE_ERR_INVALID  # ws not 256-aligned
+    assert L.moe_fused_forward(*args(nbytes=need - 1)) == ops.MOE_ERR_WORKSPACE
+    assert b"workspace" in L.moe_last_error_string()
+    pf = ops.problem(16, 8, 2, 256, 128, fp8=True)
+    assert L.moe_fused_forward(ctypes.byref(pf), good, good, None, None, good, good, None, None, good, good,
+                               ops.workspace_size(pf), None) == ops.MOE_ERR_INVALID   # FP8 without scales
+    bad_stage = L.moe_forward_stages(*args()[:-1], 4, 2, None)
+    assert bad_stage == ops.MOE_ERR_INVALID
+
+
+def test_route_align_quantize_argument_errors(L):
+    g = _fake(1 << 20)
+    assert L.moe_route(g, 4, 8, 9, 1, g, g, None) == ops.MOE_ERR_INVALID      # topk > E
+    assert L.moe_route(g, 4, 8, 2, 3, g, g, None) == ops.MOE_ERR_INVALID      # renormalize not 0/1
+    assert L.moe_route(None, 4, 8, 2, 1, g, g, None) == ops.MOE_ERR_INVALID
+    ws = int(L.moe_align_workspace_size(4, 2, 8))
+    assert ws > 0
+    assert L.moe_align(g, 4, 2, 8, 16, g, g, g, None, None, g, ws - 1, None) == ops.MOE_ERR_WORKSPACE
+    assert L.moe_align(g, 4, 2, 8, 0, g, g, g, None, None, g, ws, None) == ops.MOE_ERR_INVALID
+    assert L.moe_quantize_weights_fp8(g, 1, 100, 128, g, g, None) == ops.MOE_ERR_INVALID
+    assert L.moe_quantize_weights_fp8(g, 1, 128, 128, None, g, None) == ops.MOE_ERR_INVALID
+
+
+def test_product_path_has_no_fallback(tmp_path, monkeypatch):
+    """With the library missing, the binding raises instead of computing anything."""
+    monkeypatch.setattr(ops, "_LIB_PATH", str(tmp_path / "missing.so"))
+    monkeypatch.setattr(ops, "_lib", None)
+    with pytest.raises(RuntimeError):
+        ops.lib()

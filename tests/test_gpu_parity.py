@@ -1,0 +1,253 @@
+"""CUDA path vs the CPU oracle, through the C ABI.
+
+Bit-exact: routing ids, the alignment (permutation, padding, block experts,
+counts, offsets), FP8 weight codes/scales and the FP8 GEMM1 input.  Within
+tolerance (normwise 5e-3 bf16 / 2e-2 FP8, max |diff| <= 0.05 max |ref|): the
+layer output, on every tile orientation, at small sizes in full and at the
+benchmark sizes on sampled tokens."""
+
+import numpy as np
+import pytest
+import torch
+
+from moe_layer_top_b200 import inputs, ops
+from oracle import moe_oracle as O
+from tests.gpu_helpers import Case, assert_close, errors
+
+pytestmark = pytest.mark.gpu
+
+MID_BF16 = inputs.make_custom_config("mid_bf16", E=16, topk=4, H=1024, I=512, fp8=False, routing="logits")
+MID_FP8 = inputs.make_custom_config("mid_fp8", E=16, topk=4, H=1024, I=512, fp8=True, routing="uniform_ids")
+MODES = [(ops.MODE_NORMAL, 128), (ops.MODE_SWAP_AB, 16), (ops.MODE_SWAP_AB, 32), (ops.MODE_SWAP_AB, 64)]
+
+
+@pytest.fixture(autouse=True, scope="module")
+def _built():
+    if not torch.cuda.is_available():
+        pytest.skip("no CUDA device")
+    from moe_layer_top_b200 import build
+    build.build()
+
+
+# ----------------------------------------------------------------------------- routing
+@pytest.mark.parametrize("T,E,k,bias", [(16, 8, 2, 0.0), (64, 128, 8, 0.0), (16384, 128, 8, 0.5), (3, 256, 8, 0.0),
+                                        (50, 1000, 32, 0.0)])
+def test_route_matches_oracle(T, E, k, bias):
+    g = torch.Generator(device="cuda").manual_seed(T * 7 + E)
+    logits = torch.randn((T, E), generator=g, device="cuda") + bias * torch.randn((E,), generator=g, device="cuda")
+    ids, w = ops.route(logits, k)
+    torch.cuda.synchronize()
+    ref_ids, ref_w = O.route(logits.cpu().numpy(), k)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ref_ids)
+    np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=1e-5, atol=1e-7)
+
+
+def test_route_ties_take_lower_index():
+    logits = torch.zeros((4, 64), device="cuda")
+    logits[1, 10:20] = 1.0
+    logits[2] = torch.round(torch.randn(64, device="cuda") * 2) / 2   # many exact ties
+    ids, w = ops.route(logits, 8)
+    ref_ids, ref_w = O.route(logits.cpu().numpy(), 8)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ref_ids)
+    np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=1e-5)
+
+
+def test_route_without_renormalisation():
+    logits = torch.randn((33, 128), device="cuda")
+    ids, w = ops.route(logits, 8, renormalize=False)
+    ref_ids, ref_w = O.route(logits.cpu().numpy(), 8, renormalize=False)
+    np.testing.assert_array_equal(ids.cpu().numpy(), ref_ids)
+    np.testing.assert_allclose(w.cpu().numpy(), ref_w, rtol=1e-5, atol=1e-8)
+
+
+# ----------------------------------------------------------------------------- alignment
+def _ids(T, E, k, dist, seed):
+    rng = np.random.default_rng(seed)
+    if dist == "uniform":
+        return np.stack([rng.permutation(E)[:k] for _ in range(T)]).astype(np.int32)
+    if dist == "dup":
+        return rng.integers(0, E, (T, k)).astype(np.int32)
+    if dist == "one":
+        return np.full((T, k), 3 % E, dtype=np.int32)
+    return np.minimum(rng.zipf(1.3, (T, k)) - 1, E - 1).astype(np.int32)
+
+
+@pytest.mark.parametrize("T,E,k,bm,dist", [
+    (1, 128, 8, 16, "uniform"), (4, 128, 8, 16, "uniform"), (64, 128, 8, 16, "uniform"),
+    (256, 128, 8, 32, "dup"), (1024, 128, 8, 64, "dup"), (16384, 128, 8, 128, "uniform"),
+    (8192, 256, 8, 128, "skew"), (33, 256, 8, 16, "skew"), (100, 16, 4, 128, "one"), (7, 1, 1, 16, "uniform"),
+    (1000, 1024, 32, 32, "dup"), (3, 8, 8, 64, "uniform"),
+])
+def test_align_matches_oracle_bit_exact(T, E, k, bm, dist):
+    ids = _ids(T, E, k, dist, T + E + bm)
+    res = ops.align(torch.from_numpy(ids).cuda(), E, bm)
+    torch.cuda.synchronize()
+    ref = O.align(ids, E, bm)
+    assert res["capacity"] == ref["capacity"]
+    np.testing.assert_array_equal(res["sorted_token_ids"].cpu().numpy(), ref["sorted_token_ids"])
+    np.testing.assert_array_equal(res["expert_ids"].cpu().numpy(), ref["expert_ids"])
+    assert int(res["num_tokens_post_padded"].item()) == ref["num_tokens_post_padded"]
+    np.testing.assert_array_equal(res["expert_counts"].cpu().numpy(), ref["expert_counts"])
+    np.testing.assert_array_equal(res["expert_offsets"].cpu().numpy(), ref["expert_offsets"])
+
+
+def test_align_reports_bad_expert_id():
+    ids = torch.tensor([[0, 1], [2, 9]], dtype=torch.int32, device="cuda")   # 9 >= E
+    res = ops.align(ids, 8, 16)
+    torch.cuda.synchronize()
+    status = int(res["workspace"][:4].view(torch.int32).item())
+    assert status == ops.MOE_STATUS_BAD_EXPERT_ID
+    # the three good assignments are still placed, in order
+    s = res["sorted_token_ids"].cpu().numpy()
+    assert sorted(s[s != 4].tolist()) == [0, 1, 2]
+
+
+# ----------------------------------------------------------------------------- FP8 preparation
+def test_weight_quantisation_bit_exact():
+    cfg = inputs.CONFIGS["decode_bf16"]
+    w13, w2 = inputs.make_expert_weights(cfg, 5, 0, device="cuda")
+    for w in (w13, w2):
+        codes, scales = ops.quantize_weights_fp8(w[None])
+        torch.cuda.synchronize()
+        rc, rs = O.quantize_weight_block128(w.float().cpu().double().numpy())
+        np.testing.assert_array_equal(codes[0].cpu().numpy(), rc)
+        np.testing.assert_array_equal(scales[0].cpu().numpy(), rs)
+
+
+def test_weight_quantisation_zero_block_and_extremes():
+    w = torch.zeros((1, 256, 256), dtype=torch.bfloat16, device="cuda")
+    w[0, 0, 0] = 3.0
+    w[0, 200, 130] = -1e-30
+    w[0, 130:140, 0:128] = torch.randn((10, 128), device="cuda").to(torch.bfloat16) * 1e4
+    codes, scales = ops.quantize_weights_fp8(w)
+    rc, rs = O.quantize_weight_block128(w[0].float().cpu().double().numpy())
+    np.testing.assert_array_equal(codes[0].cpu().numpy(), rc)
+    np.testing.assert_array_equal(scales[0].cpu().numpy(), rs)
+
+
+def test_gather_quantises_x_bit_exact():
+    c = Case(MID_FP8, 37, seed=3, mode=ops.MODE_NORMAL)
+    c.run()
+    v = c.views()
+    ntpp = int(v["num_tokens_post_padded"].item())
+    sorted_ids = v["sorted_token_ids"][:ntpp].cpu().numpy()
+    nflat = 37 * MID_FP8.topk
+    rows = np.nonzero(sorted_ids < nflat)[0]
+    x = c.x.float().cpu().double().numpy()[sorted_ids[rows] // MID_FP8.topk]
+    rc, rs = O.quantize_act_group128(x)
+    np.testing.assert_array_equal(v["a1"][:ntpp].cpu().numpy()[rows], rc)
+    np.testing.assert_array_equal(v["a1_scale_t"][:, :ntpp].cpu().numpy().T[rows], rs)
+    pad = np.nonzero(sorted_ids >= nflat)[0]
+    assert np.all(v["a1"][:ntpp].cpu().numpy()[pad] == 0)
+
+
+# ----------------------------------------------------------------------------- layer output
+@pytest.mark.parametrize("mode,bm", [(ops.MODE_AUTO, 0)] + MODES)
+def test_tiny_layer_all_modes(mode, bm):
+    c = Case(inputs.CONFIGS["tiny"], 16, seed=0, mode=mode, block_m=bm)
+    out = c.run()
+    assert c.status() == ops.MOE_STATUS_OK
+    ref = c.oracle()
+    v = c.views()
+    np.testing.assert_array_equal(v["topk_ids"].cpu().numpy(), ref["topk_ids"])
+    assert_close(out.float().cpu().numpy(), ref["out"], fp8=False)
+
+
+@pytest.mark.parametrize("cfg", [MID_BF16, MID_FP8], ids=["bf16", "fp8"])
+@pytest.mark.parametrize("T", [1, 37, 700])
+@pytest.mark.parametrize("mode,bm", MODES)
+def test_mid_layer(cfg, T, mode, bm):
+    c = Case(cfg, T, seed=T, mode=mode, block_m=bm)
+    out = c.run()
+    assert c.status() == ops.MOE_STATUS_OK
+    ref = c.oracle()
+    assert_close(out.float().cpu().numpy(), ref["out"], fp8=cfg.fp8)
+
+
+@pytest.mark.parametrize("T", [1, 4, 16, 64])
+def test_decode_bf16_full_size(T):
+    c = Case(inputs.CONFIGS["decode_bf16"], T, seed=0)
+    out = c.run()
+    assert c.status() == ops.MOE_STATUS_OK
+    ref = c.oracle()
+    assert_close(out.float().cpu().numpy(), ref["out"], fp8=False)
+
+
+def _sample(T, n, seed):
+    rng = np.random.default_rng(seed)
+    return np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(n, T), replace=False)]))
+
+
+@pytest.mark.parametrize("name,T,n", [("fp8_uniform", 256, 6), ("fp8_uniform", 1024, 4), ("prefill_fp8", 16384, 4),
+                                      ("skewed_fp8", 1, 1), ("skewed_fp8", 32, 4), ("skewed_fp8", 512, 3)])
+def test_fp8_full_size_sampled(name, T, n):
+    cfg = inputs.CONFIGS[name]
+    c = Case(cfg, T, seed=0)
+    out = c.run()
+    assert c.status() == ops.MOE_STATUS_OK
+    tok = _sample(T, n, T)
+    ref = c.oracle(tokens=tok)
+    assert_close(out[torch.from_numpy(tok).cuda()].float().cpu().numpy(), ref["out"], fp8=True)
+    if "logits" in c.routing:   # the routing of every token is checked in full
+        ids, _ = O.route(c.routing["logits"].cpu().numpy(), cfg.topk)
+        np.testing.assert_array_equal(c.views()["topk_ids"].cpu().numpy(), ids)
+
+
+# ----------------------------------------------------------------------------- properties
+@pytest.mark.parametrize("cfg", [MID_BF16, MID_FP8], ids=["bf16", "fp8"])
+def test_run_to_run_bitwise_deterministic(cfg):
+    c = Case(cfg, 300, seed=1)
+    a = c.run().clone()
+    b = c.run().clone()
+    assert torch.equal(a, b)
+
+
+@pytest.mark.parametrize("cfg", [MID_BF16, MID_FP8], ids=["bf16", "fp8"])
+def test_block_size_invariance(cfg):
+    """Swap-AB with block_m 16/32/64 keeps every element's K order: bitwise equal.
+    The normal orientation is within the stated tolerance of it."""
+    outs = {}
+    w = inputs.make_weights(cfg, 2, device="cuda")
+    for mode, bm in MODES:
+        c = Case(cfg, 45, seed=2, mode=mode, block_m=bm, weights=w)
+        outs[(mode, bm)] = c.run().clone()
+    base = outs[(ops.MODE_SWAP_AB, 16)]
+    assert torch.equal(base, outs[(ops.MODE_SWAP_AB, 32)])
+    assert torch.equal(base, outs[(ops.MODE_SWAP_AB, 64)])
+    nr, mr = errors(outs[(ops.MODE_NORMAL, 128)].float().cpu().numpy(), base.float().cpu().numpy())
+    assert nr <= (2e-2 if cfg.fp8 else 5e-3) and mr <= 0.05
+
+
+def test_output_canaries_untouched():
+    cfg = MID_BF16
+    c = Case(cfg, 29, seed=4)
+    guard = torch.full((3 * 29 * cfg.H,), 1234.0, dtype=torch.bfloat16, device="cuda")
+    out = guard[29 * cfg.H:2 * 29 * cfg.H].view(29, cfg.H)
+    c.out = out
+    c.run()
+    assert torch.all(guard[:29 * cfg.H] == 1234.0) and torch.all(guard[2 * 29 * cfg.H:] == 1234.0)
+    assert not torch.any(out == 1234.0)
+
+
+def test_zero_tokens_is_a_no_op():
+    cfg = MID_BF16
+    c = Case(cfg, 1, seed=0)
+    p = ops.problem(0, cfg.E, cfg.topk, cfg.H, cfg.I)
+    out = torch.empty((0, cfg.H), dtype=torch.bfloat16, device="cuda")
+    ops.fused_forward(p, c.x[:0], c.w13, c.w2, logits=c.routing["logits"][:0], out=out,
+                      ws=torch.empty(256, dtype=torch.uint8, device="cuda"))
+    torch.cuda.synchronize()
+
+
+def test_all_tokens_on_one_expert_and_topk_equals_E():
+    cfg = inputs.make_custom_config("hot", E=8, topk=8, H=512, I=256, fp8=True, routing="uniform_ids")
+    c = Case(cfg, 200, seed=5)
+    c.routing["topk_ids"] = torch.arange(8, dtype=torch.int32, device="cuda").repeat(200, 1)
+    c.run()
+    ref = c.oracle()
+    assert_close(c.out.float().cpu().numpy(), ref["out"], fp8=True)
+    cfg1 = inputs.make_custom_config("one", E=4, topk=2, H=256, I=128, fp8=False, routing="uniform_ids")
+    c1 = Case(cfg1, 300, seed=6)
+    c1.routing["topk_ids"] = torch.full((300, 2), 1, dtype=torch.int32, device="cuda")   # duplicates in each row
+    c1.run()
+    assert_close(c1.out.float().cpu().numpy(), c1.oracle()["out"], fp8=False)
