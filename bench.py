@@ -1,0 +1,505 @@
+"""Benchmark of the fused top-k MoE layer on B200.
+
+    python bench.py [--gpus N] [--steps K] [--warmup W] [--workload NAME] [--impl ours|reference]
+
+One step = one pass of the whole layer (route -> align -> gather -> GEMM1
+(+SiLU*up) -> GEMM2 (+routed weight) -> combine) over one batch of seeded
+synthetic input resident in HBM.  The default workload is the bf16
+Qwen3-235B-shaped decode layer (H=4096, E=128, top-8, I=1536); the headline
+batch is its largest sweep point (T=64) and every sweep point is reported.
+L2 is flushed (a 256 MiB write) before every timed step; the flush is outside
+the CUDA-event brackets.  Multi-GPU runs are independent replicas (the layer
+has no exchange step on one node): each rank runs the same workload and the
+time is the max over ranks.
+
+The ``--impl reference`` arm times the CPU oracle (the plain float64 numpy
+restatement of the layer) on the host cores, on bounded token samples of the
+same workload.
+"""
+
+from __future__ import annotations
+
+import argparse
+import hashlib
+import json
+import os
+import statistics
+import subprocess
+import sys
+import tempfile
+import time
+
+ROOT = os.path.dirname(os.path.abspath(__file__))
+sys.path.insert(0, ROOT)
+
+import numpy as np  # noqa: E402
+import torch  # noqa: E402
+
+from moe_layer_top_b200 import inputs  # noqa: E402
+
+L2_FLUSH_BYTES = 256 << 20
+
+
+def parse_args():
+    ap = argparse.ArgumentParser()
+    ap.add_argument("--gpus", type=int, default=1)
+    ap.add_argument("--steps", type=int, default=20)
+    ap.add_argument("--warmup", type=int, default=5)
+    ap.add_argument("--workload", default="decode_bf16", choices=sorted(inputs.CONFIGS))
+    ap.add_argument("--tokens", type=int, default=0,
+                    help="run only this batch size (default: the workload's sweep, headline = its largest)")
+    ap.add_argument("--experts", type=int, default=0,
+                    help="override the expert count (small profiling cases of the same kernels)")
+    ap.add_argument("--impl", default="ours", choices=["ours", "reference"])
+    ap.add_argument("--no-cpu-baseline", action="store_true")
+    ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for the CPU baseline")
+    ap.add_argument("--seed", type=int, default=0)
+    return ap.parse_args()
+
+
+# ----------------------------------------------------------------------------- distributed plumbing
+def dist_setup(args):
+    world = int(os.environ.get("WORLD_SIZE", "1"))
+    rank = int(os.environ.get("RANK", "0"))
+    local = int(os.environ.get("LOCAL_RANK", "0"))
+    if world > 1:
+        import datetime
+        import torch.distributed as dist
+        backend = "nccl" if (torch.cuda.is_available() and args.impl == "ours") else "gloo"
+        if backend == "nccl":
+            torch.cuda.set_device(local)
+        dist.init_process_group(backend, timeout=datetime.timedelta(seconds=120))
+    elif torch.cuda.is_available() and args.impl == "ours":
+        torch.cuda.set_device(0)
+    return rank, world, local
+
+
+def barrier(world):
+    if world > 1:
+        import torch.distributed as dist
+        dist.barrier()
+
+
+def max_over_ranks(v: float, world: int) -> float:
+    if world == 1:
+        return v
+    import torch.distributed as dist
+    dev = "cuda" if dist.get_backend() == "nccl" else "cpu"
+    t = torch.tensor([v], dtype=torch.float64, device=dev)
+    dist.all_reduce(t, op=dist.ReduceOp.MAX)
+    return float(t.item())
+
+
+# ----------------------------------------------------------------------------- clocks
+class ClockSampler:
+    """nvidia-smi sampled every 200 ms while the timed region runs."""
+
+    FIELDS = ("clocks.sm,clocks.max.sm,power.draw,clocks_event_reasons.active,clocks_event_reasons.hw_slowdown,"
+              "clocks_event_reasons.hw_thermal_slowdown,clocks_event_reasons.sw_thermal_slowdown,"
+              "clocks_event_reasons.sw_power_cap")
+
+    def __init__(self, index: int):
+        self.index = index
+        self.proc = None
+        self.path = None
+
+    def __enter__(self):
+        fd, self.path = tempfile.mkstemp(suffix=".csv")
+        os.close(fd)
+        try:
+            self.proc = subprocess.Popen(
+                ["nvidia-smi", "-i", str(self.index), f"--query-gpu={self.FIELDS}", "--format=csv,noheader,nounits",
+                 "-lms", "200"], stdout=open(self.path, "w"), stderr=subprocess.DEVNULL)
+        except OSError:
+            self.proc = None
+        time.sleep(0.3)
+        return self
+
+    def __exit__(self, *exc):
+        if self.proc is not None:
+            self.proc.terminate()
+            try:
+                self.proc.wait(timeout=5)
+            except subprocess.TimeoutExpired:
+                self.proc.kill()
+
+    def summary(self):
+        if self.proc is None or self.path is None:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["nvidia-smi unavailable"]}
+        rows = []
+        with open(self.path) as f:
+            for line in f:
+                parts = [p.strip() for p in line.split(",")]
+                if len(parts) >= 8:
+                    rows.append(parts)
+        os.unlink(self.path)
+        if not rows:
+            return {"sm_mhz": None, "sm_max_mhz": None, "reasons": ["no samples"]}
+        sm = [float(r[0]) for r in rows if r[0].replace(".", "").isdigit()]
+        smax = [float(r[1]) for r in rows if r[1].replace(".", "").isdigit()]
+        names = ["hw_slowdown", "hw_thermal_slowdown", "sw_thermal_slowdown", "sw_power_cap"]
+        reasons = sorted({n for r in rows for n, v in zip(names, r[4:8]) if v.lower() == "active"})
+        return {"sm_mhz": statistics.median(sm) if sm else None, "sm_max_mhz": max(smax) if smax else None,
+                "reasons": reasons, "samples": len(rows)}
+
+
+# ----------------------------------------------------------------------------- peaks
+def measured_peaks():
+    path = os.path.join(ROOT, "MEASURED_PEAKS.json")
+    try:
+        with open(path) as f:
+            d = json.load(f)
+        return {"hbm_gbs": float(d["hbm_gbs"]), "bf16_tflops": float(d["bf16_tflops"]),
+                "bf16_tflops_sustained": float(d.get("bf16_tflops_sustained", d["bf16_tflops"])),
+                "source": "measured"}
+    except (OSError, KeyError, ValueError):
+        return {"hbm_gbs": 6650.0, "bf16_tflops": 1590.0, "bf16_tflops_sustained": 1400.0, "source": "fallback"}
+
+
+KERNEL_SOURCES = {
+    "gemm1": ("common.cuh", "gemm.cu", "kernels.h"),
+    "gemm2": ("common.cuh", "gemm.cu", "kernels.h"),
+}
+
+
+def kernel_source_sha(kernel: str) -> str:
+    """Hash of the sources that define a kernel (a stored ncu figure is only
+    valid while it matches)."""
+    src = os.path.join(ROOT, "moe_layer_top_b200", "csrc")
+    h = hashlib.sha256()
+    for name in KERNEL_SOURCES.get(kernel, tuple(sorted(os.listdir(src)))):
+        with open(os.path.join(src, name), "rb") as f:
+            h.update(f.read())
+    return h.hexdigest()[:16]
+
+
+def traffic_record(kernel: str, workload: str, T: int):
+    """DRAM bytes per launch from a committed ncu summary, if the kernel
+    source is unchanged since it was captured."""
+    path = os.path.join(ROOT, "profiles", "ncu_traffic.json")
+    try:
+        with open(path) as f:
+            recs = json.load(f)
+    except (OSError, ValueError):
+        return None
+    digest = kernel_source_sha(kernel)
+    for r in recs:
+        if r.get("kernel") == kernel and r.get("workload") == workload and int(r.get("T", -1)) == T \
+                and r.get("source_sha") == digest:
+            return float(r["dram_bytes_per_launch"])
+    return None
+
+
+# ----------------------------------------------------------------------------- our arm
+def workload_config(args):
+    import dataclasses
+    cfg = inputs.CONFIGS[args.workload]
+    if args.experts:
+        cfg = dataclasses.replace(cfg, name=f"{cfg.name}[E={args.experts}]", E=args.experts)
+    return cfg
+
+
+class Workload:
+    def __init__(self, cfg, T, seed, weights):
+        from moe_layer_top_b200 import ops
+        self.ops = ops
+        self.cfg, self.T = cfg, T
+        dev = torch.device("cuda")
+        self.w13, self.w2, self.s13, self.s2 = weights
+        self.x = inputs.make_tokens(cfg, T, seed, device=dev)
+        self.routing = inputs.make_routing(cfg, T, seed, device=dev)
+        self.p = ops.problem(T, cfg.E, cfg.topk, cfg.H, cfg.I, fp8=cfg.fp8)
+        self.q = ops.resolve_problem(self.p)
+        self.ws = ops.alloc_workspace(self.p)
+        self.out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
+
+    def kw(self):
+        return dict(logits=self.routing.get("logits"), topk_ids=self.routing.get("topk_ids"),
+                    topk_weights=self.routing.get("topk_weights"), w13_scale=self.s13, w2_scale=self.s2,
+                    out=self.out, ws=self.ws)
+
+    def stage(self, s):
+        self.ops.forward_stages(self.p, self.x, self.w13, self.w2, s, s + 1, **self.kw())
+
+    def forward(self):
+        self.ops.fused_forward(self.p, self.x, self.w13, self.w2, **self.kw())
+
+    def algorithmic(self):
+        """Algorithmic bytes / FLOPs of the layer and of each GEMM for this routing."""
+        v = self.ops.workspace_views(self.p, self.ws)
+        counts = v["expert_counts"].cpu().numpy()
+        ntpp = int(v["num_tokens_post_padded"].item())
+        hit = int((counts > 0).sum())
+        cfg = self.cfg
+        elem = 1 if cfg.fp8 else 2
+        w13_e = 2 * cfg.I * cfg.H * elem + (2 * cfg.I // 128) * (cfg.H // 128) * 4 * cfg.fp8
+        w2_e = cfg.H * cfg.I * elem + (cfg.H // 128) * (cfg.I // 128) * 4 * cfg.fp8
+        nflat = self.T * cfg.topk
+        route_io = self.T * cfg.E * 4 if "logits" in self.routing else nflat * 8
+        rows = ntpp
+        gemm1 = hit * w13_e + rows * cfg.H * elem + rows * cfg.I * elem
+        gemm2 = hit * w2_e + rows * cfg.I * elem + nflat * cfg.H * 2
+        layer = hit * (w13_e + w2_e) + self.T * cfg.H * 2 * 2 + route_io
+        flops = 2.0 * nflat * 3 * cfg.H * cfg.I
+        return {"hit_experts": hit, "padded_rows": ntpp, "layer_bytes": layer, "gemm1_bytes": gemm1,
+                "gemm2_bytes": gemm2, "flops": flops, "w13_bytes_per_expert": w13_e, "w2_bytes_per_expert": w2_e}
+
+
+def make_weights(cfg, seed):
+    from moe_layer_top_b200 import ops
+    w13, w2 = inputs.make_weights(cfg, seed, device="cuda")
+    if cfg.fp8:
+        q13, s13 = ops.quantize_weights_fp8(w13)
+        q2, s2 = ops.quantize_weights_fp8(w2)
+        del w13, w2
+        torch.cuda.empty_cache()
+        return q13, q2, s13, s2
+    return w13, w2, None, None
+
+
+def time_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor, world: int):
+    """Per-stage CUDA-event times (ms) of `steps` timed passes, L2 flushed before each."""
+    ops = wl.ops
+    stream = torch.cuda.current_stream()
+    for _ in range(warmup):
+        flush.zero_()
+        wl.forward()
+    torch.cuda.synchronize()
+    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(ops.NUM_STAGES + 1)] for _ in range(steps)]
+    barrier(world)
+    torch.cuda.synchronize()
+    wall0 = time.perf_counter()
+    for i in range(steps):
+        flush.zero_()
+        ev[i][0].record(stream)
+        for s in range(ops.NUM_STAGES):
+            wl.stage(s)
+            ev[i][s + 1].record(stream)
+    torch.cuda.synchronize()
+    barrier(world)
+    wall = time.perf_counter() - wall0
+    per_stage = np.array([[ev[i][s].elapsed_time(ev[i][s + 1]) for s in range(ops.NUM_STAGES)]
+                          for i in range(steps)])
+    return per_stage, wall
+
+
+def e2e_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor):
+    """Same metric with host buffers: pinned H2D of x (+ routing input), the
+    layer, D2H of the output, all inside the CUDA-event brackets."""
+    x_h = wl.x.cpu().pin_memory()
+    r_h = {k: v.cpu().pin_memory() for k, v in wl.routing.items()}
+    out_h = torch.empty(wl.out.shape, dtype=wl.out.dtype).pin_memory()
+    x_d = torch.empty_like(wl.x)
+    r_d = {k: torch.empty_like(v) for k, v in wl.routing.items()}
+    stream = torch.cuda.current_stream()
+    ops = wl.ops
+
+    def one():
+        x_d.copy_(x_h, non_blocking=True)
+        for k in r_d:
+            r_d[k].copy_(r_h[k], non_blocking=True)
+        ops.fused_forward(wl.p, x_d, wl.w13, wl.w2, logits=r_d.get("logits"), topk_ids=r_d.get("topk_ids"),
+                          topk_weights=r_d.get("topk_weights"), w13_scale=wl.s13, w2_scale=wl.s2, out=wl.out,
+                          ws=wl.ws)
+        out_h.copy_(wl.out, non_blocking=True)
+
+    for _ in range(warmup):
+        flush.zero_()
+        one()
+    torch.cuda.synchronize()
+    times = []
+    for _ in range(steps):
+        flush.zero_()
+        a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
+        a.record(stream)
+        one()
+        b.record(stream)
+        b.synchronize()
+        times.append(a.elapsed_time(b))
+    h2d = x_h.numel() * x_h.element_size() + sum(v.numel() * v.element_size() for v in r_h.values())
+    d2h = out_h.numel() * out_h.element_size()
+    return float(np.sum(times)), h2d, d2h
+
+
+def cpu_baseline(cfg, T, seed, budget_s):
+    """The oracle, as it stands, timed on a bounded token sample of the workload.
+
+    The generator's inputs for the sampled tokens (and the oracle's own FP8
+    block quantisation of the weights they touch) are prepared untimed; the
+    timed region is the oracle's forward on those tokens."""
+    from oracle import moe_oracle as O
+    dev = "cuda" if torch.cuda.is_available() else "cpu"
+    x = inputs.make_tokens(cfg, T, seed, device=dev).float().cpu().double().numpy()
+    routing = {k: v.cpu().numpy() for k, v in inputs.make_routing(cfg, T, seed, device=dev).items()}
+    if "logits" in routing:
+        ids_all, _ = O.route(routing["logits"], cfg.topk)
+        rkw = {"logits": routing["logits"]}
+    else:
+        ids_all = routing["topk_ids"]
+        rkw = {"topk_ids": routing["topk_ids"], "topk_weights": routing["topk_weights"]}
+    host = {}
+
+    def prepare(tokens):
+        for e in np.unique(ids_all[tokens]):
+            e = int(e)
+            if e not in host:
+                a, b = inputs.make_expert_weights(cfg, e, seed, device=dev)
+                a = a.float().cpu().double().numpy()
+                b = b.float().cpu().double().numpy()
+                host[e] = (*O.quantize_weight_block128(a), *O.quantize_weight_block128(b)) if cfg.fp8 \
+                    else (a, None, b, None)
+
+    class View:
+        def __init__(self, i):
+            self.i = i
+
+        def __getitem__(self, e):
+            return host[int(e)][self.i]
+
+    order = np.random.default_rng(seed).permutation(T)
+    done, t_spent, n = 0, 0.0, 1
+    while done < T and (done == 0 or t_spent < budget_s):
+        tok = order[done:done + n]
+        prepare(tok)
+        t0 = time.perf_counter()
+        if cfg.fp8:
+            O.moe_forward(x, View(0), View(2), cfg.topk, w13_scale=View(1), w2_scale=View(3), tokens=tok, **rkw)
+        else:
+            O.moe_forward(x, View(0), View(2), cfg.topk, tokens=tok, **rkw)
+        t_spent += time.perf_counter() - t0
+        done += len(tok)
+        n = min(2 * n, T - done) if done < T else n
+    try:
+        from threadpoolctl import threadpool_info
+        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
+    except Exception:  # noqa: BLE001
+        cores = 1
+    return {"value": done / t_spent, "unit": "tokens/s", "cores": cores, "kind": "oracle",
+            "sample": f"{done} of {T} tokens of {cfg.name} (T={T}); float64 numpy oracle forward, inputs "
+                      f"prepared untimed; {t_spent:.2f} s timed"}
+
+
+def run_ours(args, rank, world, local):
+    from moe_layer_top_b200 import build, ops
+    build.build()
+    ops.lib()
+    cfg = workload_config(args)
+    T_head = args.tokens or max(cfg.tokens)
+    sweep_T = [T_head] if args.tokens else sorted(cfg.tokens)
+    peaks = measured_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    weights = make_weights(cfg, args.seed)
+    results = {}
+    with ClockSampler(local) as clocks:
+        for T in sweep_T:
+            wl = Workload(cfg, T, args.seed, weights)
+            steps = args.steps if T == T_head else max(3, args.steps // 2)
+            per_stage, wall = time_steps(wl, steps, args.warmup, flush, world)
+            step_ms = per_stage.sum(axis=1)
+            total_ms = max_over_ranks(float(step_ms.sum()), world)
+            results[T] = {"wl": wl, "per_stage": per_stage, "total_ms": total_ms, "steps": steps, "wall_s": wall}
+    clk = clocks.summary()
+    head = results[T_head]
+    wl = head["wl"]
+    alg = wl.algorithmic()
+    K = head["steps"]
+    value = world * T_head * K / (head["total_ms"] / 1e3)
+    ms_per_step = head["total_ms"] / K
+    stage_ms = head["per_stage"].mean(axis=0)
+    # dominant kernel: the stage with the largest share of the step
+    dom = int(np.argmax(stage_ms))
+    dom_name = ops.STAGE_NAMES[dom]
+    dom_bytes = {"gemm1": alg["gemm1_bytes"], "gemm2": alg["gemm2_bytes"]}.get(dom_name)
+    if dom_bytes is None:
+        dom_bytes = alg["layer_bytes"]
+    achieved = dom_bytes / (stage_ms[dom] / 1e3) / 1e9
+    traffic = traffic_record(dom_name, args.workload, T_head)
+    roofline = {"bound": "hbm", "kernel": dom_name, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                "peak_source": peaks["source"], "algorithmic_bytes": dom_bytes}
+    sweep = []
+    for T in sweep_T:
+        r = results[T]
+        a = r["wl"].algorithmic()
+        ms = r["total_ms"] / r["steps"]
+        sm = r["per_stage"].mean(axis=0)
+        sweep.append({"T": T, "tokens_per_s": round(world * T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+                      "layer_hbm_frac": round(a["layer_bytes"] / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+                      "tflops": round(a["flops"] / (ms / 1e3) / 1e12, 2), "hit_experts": a["hit_experts"],
+                      "stage_us": {ops.STAGE_NAMES[s]: round(float(sm[s]) * 1e3, 1) for s in range(ops.NUM_STAGES)},
+                      "mode": "swap_ab" if r["wl"].q.mode == ops.MODE_SWAP_AB else "normal",
+                      "block_m": r["wl"].q.block_m})
+    e2e_ms, h2d, d2h = e2e_steps(wl, K, args.warmup, flush)
+    e2e_ms = max_over_ranks(e2e_ms, world)
+    e2e = {"value": round(world * T_head * K / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
+           "d2h_bytes_per_step": d2h}
+    line = {
+        "metric": "fused-MoE tokens/s; % HBM roofline (decode), % FP8/BF16 TC peak (prefill)",
+        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
+        "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "fp8_e4m3" if cfg.fp8 else "bf16", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: H={cfg.H} E={cfg.E} topk={cfg.topk} I={cfg.I} T={T_head}",
+                   "global_batch": world * T_head, "tokens_per_gpu": T_head, "parallelism": f"replicas{world}",
+                   "weights": "fp8 e4m3 + 128x128 fp32 scales" if cfg.fp8 else "bf16",
+                   "routing": cfg.routing, "l2": "flushed (256 MiB write) before every step, outside the timing",
+                   "layer_bytes_per_step": alg["layer_bytes"], "hit_experts": alg["hit_experts"]},
+        "roofline": roofline,
+        "layer_hbm_frac": round(alg["layer_bytes"] / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+        "stage_us": {ops.STAGE_NAMES[s]: round(float(stage_ms[s]) * 1e3, 1) for s in range(ops.NUM_STAGES)},
+        "sweep": sweep,
+        "e2e": e2e,
+        "gpu_launches": K * 8,
+        "clocks": clk,
+    }
+    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+        line["cpu_baseline"] = cpu_baseline(cfg, T_head, args.seed, args.cpu_budget)
+    return line
+
+
+# ----------------------------------------------------------------------------- reference arm (the oracle)
+def run_reference(args, rank, world):
+    cfg = workload_config(args)
+    T = args.tokens or max(cfg.tokens)
+    if rank != 0:
+        return None
+    for _ in range(args.warmup):
+        cpu_baseline(cfg, T, args.seed, budget_s=0.0)
+    vals = []
+    base = None
+    per_step_budget = max(1.0, args.cpu_budget / max(1, args.steps))
+    for _ in range(args.steps):
+        base = cpu_baseline(cfg, T, args.seed, budget_s=per_step_budget)
+        vals.append(base["value"])
+    value = float(np.mean(vals))
+    base["value"] = round(value, 3)
+    return {
+        "impl": "reference",
+        "metric": "fused-MoE tokens/s; % HBM roofline (decode), % FP8/BF16 TC peak (prefill)",
+        "value": round(value, 3), "unit": "tokens/s", "n_gpus": world, "steps": args.steps, "warmup": args.warmup,
+        "ms_per_step": round(1e3 * T / value, 3), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "dtype": "f64", "data": "synthetic",
+        "config": {"workload": f"{cfg.name}: H={cfg.H} E={cfg.E} topk={cfg.topk} I={cfg.I} T={T}",
+                   "global_batch": T, "parallelism": "cpu"},
+        "cpu_baseline": base,
+        "e2e": {"value": round(value, 3), "unit": "tokens/s", "h2d_bytes_per_step": 0, "d2h_bytes_per_step": 0},
+    }
+
+
+def main():
+    args = parse_args()
+    rank, world, local = dist_setup(args)
+    try:
+        if args.impl == "reference":
+            line = run_reference(args, rank, world)
+        else:
+            line = run_ours(args, rank, world, local)
+        if rank == 0 and line is not None:
+            print(json.dumps(line), flush=True)
+    finally:
+        if world > 1:
+            import torch.distributed as dist
+            dist.destroy_process_group()
+
+
+if __name__ == "__main__":
+    main()
