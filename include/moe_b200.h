@@ -175,6 +175,36 @@ MOE_API int moe_align(const int32_t* topk_ids, int32_t T, int32_t topk, int32_t 
               int32_t* expert_counts, int32_t* expert_offsets, void* ws, size_t ws_bytes, void* stream);
 
 /*
+ * moe_align without a workspace, for callers that cannot allocate device
+ * memory when they align (a framework that owns every allocation and lends
+ * none, code running inside a CUDA-graph capture with a fixed memory plan,
+ * a serving loop that bans allocator calls after start-up).  The pages have
+ * no counterpart of this entry point; it is a deployment convenience.
+ *
+ * Same arguments, results and determinism as moe_align, minus ws/ws_bytes:
+ * the scratch moe_align would take from the workspace lives instead in one
+ * static device array of MOE_ALIGN_NOALLOC_SCRATCH_BYTES, which every GPU
+ * that loads this library holds until the process exits.
+ *  - Limit: moe_align_workspace_size(T, topk, E) must not exceed
+ *    MOE_ALIGN_NOALLOC_SCRATCH_BYTES (1 MiB: about 520 000 assignments at
+ *    E = 128, 260 000 at E = 256); larger problems return MOE_ERR_INVALID
+ *    before anything is enqueued.
+ *  - The first call on each device looks up the array's device address
+ *    (cudaGetSymbolAddress, with that device current); make that first call
+ *    before any stream capture.
+ *  - All calls on a device share the array, and it keeps the previous
+ *    call's contents; each call clears or rewrites every entry it reads.
+ *    Calls whose executions overlap on the GPU (unordered streams) race.
+ *  - An expert id outside [0, E) is not reported (the status word lives in
+ *    the shared array); the outputs of that call are then undefined.
+ *  - Calls no allocator (no cudaMalloc, cudaFree or allocating library call).
+ */
+#define MOE_ALIGN_NOALLOC_SCRATCH_BYTES (1 << 20)
+MOE_API int moe_align_noalloc(const int32_t* topk_ids, int32_t T, int32_t topk, int32_t E, int32_t block_m,
+                              int32_t* sorted_token_ids, int32_t* expert_ids, int32_t* num_tokens_post_padded,
+                              int32_t* expert_counts, int32_t* expert_offsets, void* stream);
+
+/*
  * FP8 weight preparation: w [batches, rows, cols] bf16 -> codes [batches,
  * rows, cols] E4M3 and scales [batches, rows/128, cols/128] fp32 with, per
  * 128 x 128 block, scale = max(blockmax, 1e-10) / 448 (fp32) and

@@ -276,6 +276,10 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
 
 }  // namespace
 
+namespace moe {
+int record_error(int code, const char* msg) { return fail(code, "%s", msg); }
+}  // namespace moe
+
 extern "C" {
 
 const char* moe_last_error_string(void) { return g_last_error.c_str(); }

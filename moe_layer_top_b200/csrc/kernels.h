@@ -52,6 +52,9 @@ cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const float* a1_s
 cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const float* a2_scale_t, const void* w2,
                          const float* w2_scale, void* y, cudaStream_t stream);
 
+// set the per-thread error message returned by moe_last_error_string(); returns code
+int record_error(int code, const char* msg);
+
 // shared-memory bytes the GEMM variant needs (for validation / occupancy)
 size_t gemm_smem_bytes(bool gemm2, bool fp8, bool swap, int block_m);
 

@@ -42,7 +42,7 @@ STAGE_NAMES = ("route", "align", "gather", "gemm1", "gemm2", "combine")
 EXPORTED = (
     "moe_last_error_string", "moe_route", "moe_align_capacity", "moe_align_workspace_size", "moe_align",
     "moe_quantize_weights_fp8", "moe_resolve_problem", "moe_workspace_size", "moe_get_workspace_layout",
-    "moe_fused_forward", "moe_forward_stages", "moe_read_status", "moe_version",
+    "moe_fused_forward", "moe_forward_stages", "moe_read_status", "moe_version", "moe_align_noalloc",
 )
 
 
@@ -90,6 +90,7 @@ def lib():
             "moe_align_capacity": (i64, [i32, i32, i32, i32]),
             "moe_align_workspace_size": (sz, [i32, i32, i32]),
             "moe_align": (ctypes.c_int, [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
+            "moe_align_noalloc": (ctypes.c_int, [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
             "moe_quantize_weights_fp8": (ctypes.c_int, [vp, i64, i32, i32, vp, vp, vp]),
             "moe_resolve_problem": (ctypes.c_int, [P]),
             "moe_workspace_size": (sz, [P]),
