@@ -4,7 +4,9 @@
 
 One step = one pass of the whole layer (route -> align -> gather -> GEMM1
 (+SiLU*up) -> GEMM2 (+routed weight) -> combine) over one batch of seeded
-synthetic input resident in HBM.  The default workload is the bf16
+synthetic input resident in HBM, replayed from a CUDA graph of one
+moe_fused_forward call (the way a decode loop runs it).  Per-kernel times come
+from a second graph of the same stages with event nodes between them.  The default workload is the bf16
 Qwen3-235B-shaped decode layer (H=4096, E=128, top-8, I=1536); the headline
 batch is its largest sweep point (T=64) and every sweep point is reported.
 L2 is flushed (a 256 MiB write) before every timed step; the flush is outside
@@ -245,6 +247,15 @@ class Workload:
                 "gemm2_bytes": gemm2, "flops": flops, "w13_bytes_per_expert": w13_e, "w2_bytes_per_expert": w2_e}
 
 
+def kernels_per_forward(cfg, T, has_logits):
+    """Kernels of this library one moe_fused_forward launches: a single-CTA
+    route+align for T*topk <= 8192 and E <= 256, else route + 3 align passes;
+    then gather, GEMM1, GEMM2, combine."""
+    small = T * cfg.topk <= 8192 and cfg.E <= 256
+    head = 1 if small else (1 if has_logits else 0) + 3
+    return head + 4
+
+
 def make_weights(cfg, seed):
     from moe_layer_top_b200 import ops
     w13, w2 = inputs.make_weights(cfg, seed, device="cuda")
@@ -257,30 +268,102 @@ def make_weights(cfg, seed):
     return w13, w2, None, None
 
 
+class StageEvents:
+    """CUDA events recorded as nodes of a captured graph.
+
+    Inside stream capture a plain event record only expresses a dependency;
+    cudaEventRecordWithFlags(..., cudaEventRecordExternal) makes it a timing
+    node of the graph, so every replay stamps the events again."""
+
+    def __init__(self, n):
+        import ctypes
+        import glob
+        self.ctypes = ctypes
+        self.ev = [torch.cuda.Event(enable_timing=True) for _ in range(n)]
+        for e in self.ev:
+            e.record()
+        torch.cuda.synchronize()
+        libs = glob.glob(os.path.join(os.path.dirname(torch.__file__), "..", "nvidia", "cuda_runtime", "lib",
+                                      "libcudart.so*")) + ["libcudart.so.12", "libcudart.so"]
+        self.rt = None
+        for lib in libs:
+            try:
+                self.rt = ctypes.CDLL(lib)
+                break
+            except OSError:
+                continue
+        if self.rt is None:
+            raise RuntimeError("libcudart not found")
+        self.rt.cudaEventRecordWithFlags.argtypes = [ctypes.c_void_p, ctypes.c_void_p, ctypes.c_uint]
+        self.rt.cudaEventRecordWithFlags.restype = ctypes.c_int
+
+    def record(self, i):
+        if not torch.cuda.is_current_stream_capturing():
+            self.ev[i].record()
+            return
+        stream = torch.cuda.current_stream().cuda_stream
+        rc = self.rt.cudaEventRecordWithFlags(self.ctypes.c_void_p(self.ev[i].cuda_event),
+                                              self.ctypes.c_void_p(stream), 1)
+        if rc != 0:
+            raise RuntimeError(f"cudaEventRecordWithFlags failed ({rc})")
+
+    def elapsed(self):
+        return [self.ev[i].elapsed_time(self.ev[i + 1]) for i in range(len(self.ev) - 1)]
+
+
+def capture(fn):
+    """Capture fn() into a CUDA graph (after it has run once eagerly)."""
+    fn()
+    torch.cuda.synchronize()
+    g = torch.cuda.CUDAGraph()
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
+    return g
+
+
 def time_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor, world: int):
-    """Per-stage CUDA-event times (ms) of `steps` timed passes, L2 flushed before each."""
+    """Two timed passes, L2 flushed before every step (outside the events):
+    A) a CUDA graph of moe_fused_forward, one event pair per replay -> step times;
+    B) a CUDA graph of the same stages with event nodes between them -> per-stage times."""
     ops = wl.ops
     stream = torch.cuda.current_stream()
+    g_fwd = capture(wl.forward)
+    se = StageEvents(ops.NUM_STAGES + 1)
+
+    def staged():
+        se.record(0)
+        for s in range(ops.NUM_STAGES):
+            wl.stage(s)
+            se.record(s + 1)
+
+    g_stg = capture(staged)
     for _ in range(warmup):
         flush.zero_()
-        wl.forward()
+        g_fwd.replay()
+        flush.zero_()
+        g_stg.replay()
     torch.cuda.synchronize()
-    ev = [[torch.cuda.Event(enable_timing=True) for _ in range(ops.NUM_STAGES + 1)] for _ in range(steps)]
+    ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
     barrier(world)
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     for i in range(steps):
         flush.zero_()
         ev[i][0].record(stream)
-        for s in range(ops.NUM_STAGES):
-            wl.stage(s)
-            ev[i][s + 1].record(stream)
+        g_fwd.replay()
+        ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
     wall = time.perf_counter() - wall0
-    per_stage = np.array([[ev[i][s].elapsed_time(ev[i][s + 1]) for s in range(ops.NUM_STAGES)]
-                          for i in range(steps)])
-    return per_stage, wall
+    step_ms = np.array([a.elapsed_time(b) for a, b in ev])
+    per_stage = []
+    for i in range(steps):
+        flush.zero_()
+        g_stg.replay()
+        torch.cuda.synchronize()
+        per_stage.append(se.elapsed())
+    return step_ms, np.array(per_stage), wall
 
 
 def e2e_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor):
@@ -394,8 +477,7 @@ def run_ours(args, rank, world, local):
         for T in sweep_T:
             wl = Workload(cfg, T, args.seed, weights)
             steps = args.steps if T == T_head else max(3, args.steps // 2)
-            per_stage, wall = time_steps(wl, steps, args.warmup, flush, world)
-            step_ms = per_stage.sum(axis=1)
+            step_ms, per_stage, wall = time_steps(wl, steps, args.warmup, flush, world)
             total_ms = max_over_ranks(float(step_ms.sum()), world)
             results[T] = {"wl": wl, "per_stage": per_stage, "total_ms": total_ms, "steps": steps, "wall_s": wall}
     clk = clocks.summary()
@@ -442,13 +524,14 @@ def run_ours(args, rank, world, local):
                    "global_batch": world * T_head, "tokens_per_gpu": T_head, "parallelism": f"replicas{world}",
                    "weights": "fp8 e4m3 + 128x128 fp32 scales" if cfg.fp8 else "bf16",
                    "routing": cfg.routing, "l2": "flushed (256 MiB write) before every step, outside the timing",
+                   "launch": "CUDA graph of moe_fused_forward (PDL between kernels)",
                    "layer_bytes_per_step": alg["layer_bytes"], "hit_experts": alg["hit_experts"]},
         "roofline": roofline,
         "layer_hbm_frac": round(alg["layer_bytes"] / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
         "stage_us": {ops.STAGE_NAMES[s]: round(float(stage_ms[s]) * 1e3, 1) for s in range(ops.NUM_STAGES)},
         "sweep": sweep,
         "e2e": e2e,
-        "gpu_launches": K * 8,
+        "gpu_launches": K * kernels_per_forward(cfg, T_head, "logits" in wl.routing),
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

@@ -77,8 +77,8 @@ extern "C" {
 #define MOE_MODE_SWAP_AB 2 /* MMA M = 128 weight rows, N = block_m token rows */
 
 /* stages of moe_forward_stages, in pipeline order */
-#define MOE_STAGE_ROUTE 0   /* skipped when no router logits are given */
-#define MOE_STAGE_ALIGN 1   /* histogram, scan, stable scatter */
+#define MOE_STAGE_ROUTE 0   /* router (skipped without logits); for T*topk <= 8192 and E <= 256 it also aligns */
+#define MOE_STAGE_ALIGN 1   /* histogram, scan, stable scatter (no work when the route stage aligned) */
 #define MOE_STAGE_GATHER 2  /* x rows into expert-sorted order (+ FP8 quantisation) */
 #define MOE_STAGE_GEMM1 3   /* gate/up grouped GEMM + fused SiLU*up (+ FP8 requant) */
 #define MOE_STAGE_GEMM2 4   /* down grouped GEMM + routed-weight scatter */
@@ -102,7 +102,8 @@ typedef struct moe_problem {
   int32_t mode;         /* MOE_MODE_* */
   int32_t block_m;      /* rows per expert block: 16, 32 or 64 (swap-AB), 128 (normal); 0 = auto */
   int32_t renormalize;  /* router: 1 = renormalise the chosen softmax weights (default), 0 = keep them */
-  int32_t reserved[7];  /* must be zero */
+  int32_t split_k;      /* swap-AB GEMMs: 0 = split K when few tiles are in flight (default), 1 = never */
+  int32_t reserved[6];  /* must be zero */
 } moe_problem;
 
 /*
@@ -120,11 +121,13 @@ typedef struct moe_workspace_layout {
   int64_t expert_counts;    /* int32 [E] */
   int64_t expert_offsets;   /* int32 [E + 1] */
   int64_t align_scratch;    /* int32 [chunks * E] */
-  int64_t a1;               /* bf16 or E4M3 [capacity, H] x rows in sorted order */
+  int64_t a1;               /* bf16 or E4M3 [capacity, H] x rows in sorted order (padding rows unspecified) */
   int64_t a1_scale;         /* fp32 [H/128, capacity] (FP8 only; K-block major) */
-  int64_t a2;               /* bf16 or E4M3 [capacity, I] activation in sorted order */
+  int64_t a2;               /* bf16 or E4M3 [capacity, I] activation in sorted order (padding rows unspecified) */
   int64_t a2_scale;         /* fp32 [I/128, capacity] (FP8 only; K-block major) */
   int64_t y;                /* bf16 [T*topk, H] weighted expert outputs */
+  int64_t partials;         /* fp32 split-K partial sums of the swap-AB GEMMs (swap-AB only) */
+  int64_t tile_counters;    /* int32 per-tile split-K arrival counters (swap-AB only) */
   int64_t total_bytes;
   int32_t capacity;         /* rows of sorted_token_ids */
   int32_t block_m;

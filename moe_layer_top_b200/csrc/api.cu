@@ -76,7 +76,8 @@ int validate_problem(const moe_problem* p) {
     return fail(MOE_ERR_UNSUPPORTED, "weight_dtype %d", p->weight_dtype);
   if (p->mode < MOE_MODE_AUTO || p->mode > MOE_MODE_SWAP_AB) return fail(MOE_ERR_INVALID, "mode %d", p->mode);
   if (p->renormalize != 0 && p->renormalize != 1) return fail(MOE_ERR_INVALID, "renormalize must be 0 or 1");
-  for (int i = 0; i < 7; ++i)
+  if (p->split_k != 0 && p->split_k != 1) return fail(MOE_ERR_INVALID, "split_k must be 0 or 1");
+  for (int i = 0; i < 6; ++i)
     if (p->reserved[i] != 0) return fail(MOE_ERR_INVALID, "reserved fields must be zero");
   if (p->mode == MOE_MODE_NORMAL && p->block_m != 0 && p->block_m != 128)
     return fail(MOE_ERR_INVALID, "normal mode uses block_m = 128 (got %d)", p->block_m);
@@ -158,6 +159,16 @@ int make_plan(const moe_problem* in, Plan* plan) {
   L.a2 = take(cap * p.I * elem);
   L.a2_scale = plan->fp8 ? take(cap * (p.I / 128) * 4) : -1;
   L.y = take(plan->nflat * p.H * 2);
+  if (p.mode == MOE_MODE_SWAP_AB) {
+    // one buffer serves both GEMMs (they run one after the other); GEMM1's
+    // units hold 2*block_m accumulator columns, GEMM2's block_m
+    L.partials = take(static_cast<int64_t>(moe::kMaxSplitUnits) * 128 * 2 * p.block_m * 4);
+    const int64_t blocks = cap / p.block_m;
+    L.tile_counters = take((blocks * (p.I / 128) + blocks * (p.H / 128)) * 4);
+  } else {
+    L.partials = -1;
+    L.tile_counters = -1;
+  }
   L.total_bytes = off;
   L.capacity = static_cast<int32_t>(cap);
   L.block_m = p.block_m;
@@ -207,6 +218,10 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
   const float* wts = logits ? at<float>(ws, L.topk_weights) : topk_weights;
   const int nflat = static_cast<int>(plan.nflat);
   const int cap = L.capacity;
+  const bool small = moe::route_align_small_fits(plan.nflat, p.E);
+  const bool swap = p.mode == MOE_MODE_SWAP_AB;
+  const int n_counters = swap ? (cap / p.block_m) * (p.I / 128 + p.H / 128) : 0;
+  bool aligned_already = false;
   cudaError_t e;
 
   for (int s = stage_begin; s < stage_end; ++s) {
@@ -214,13 +229,33 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
       case MOE_STAGE_ROUTE:
         if ((e = cudaMemsetAsync(status, 0, sizeof(int), stream)) != cudaSuccess)
           return cuda_fail(e, "clear status");
-        if (logits) {
+        if (small && stage_end > MOE_STAGE_ALIGN) {
+          // small batch: routing and the alignment in one single-CTA kernel
+          e = moe::launch_route_align_small(logits, logits ? nullptr : topk_ids, p.T, p.E, p.topk, p.renormalize,
+                                            at<int32_t>(ws, L.topk_ids), at<float>(ws, L.topk_weights), p.block_m,
+                                            cap, at<int32_t>(ws, L.sorted_token_ids), at<int32_t>(ws, L.expert_ids),
+                                            at<int32_t>(ws, L.num_tokens_post_padded),
+                                            at<int32_t>(ws, L.expert_counts), at<int32_t>(ws, L.expert_offsets),
+                                            status, stream);
+          if (e != cudaSuccess) return cuda_fail(e, "route+align");
+          aligned_already = true;
+        } else if (logits) {
           e = moe::launch_route(logits, p.T, p.E, p.topk, p.renormalize, at<int32_t>(ws, L.topk_ids),
                                 at<float>(ws, L.topk_weights), stream);
           if (e != cudaSuccess) return cuda_fail(e, "route");
         }
         break;
       case MOE_STAGE_ALIGN:
+        if (aligned_already) break;
+        if (small) {
+          e = moe::launch_route_align_small(nullptr, ids, p.T, p.E, p.topk, p.renormalize, nullptr, nullptr,
+                                            p.block_m, cap, at<int32_t>(ws, L.sorted_token_ids),
+                                            at<int32_t>(ws, L.expert_ids), at<int32_t>(ws, L.num_tokens_post_padded),
+                                            at<int32_t>(ws, L.expert_counts), at<int32_t>(ws, L.expert_offsets),
+                                            status, stream);
+          if (e != cudaSuccess) return cuda_fail(e, "align");
+          break;
+        }
         e = moe::launch_align(ids, nflat, p.E, p.block_m, cap, at<int32_t>(ws, L.sorted_token_ids),
                               at<int32_t>(ws, L.expert_ids), at<int32_t>(ws, L.num_tokens_post_padded),
                               at<int32_t>(ws, L.expert_counts), at<int32_t>(ws, L.expert_offsets),
@@ -230,7 +265,8 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
       case MOE_STAGE_GATHER:
         e = moe::launch_gather(x, p.H, p.topk, nflat, at<int32_t>(ws, L.sorted_token_ids),
                                at<int32_t>(ws, L.num_tokens_post_padded), cap, plan.fp8, at<void>(ws, L.a1),
-                               plan.fp8 ? at<float>(ws, L.a1_scale) : nullptr, stream);
+                               plan.fp8 ? at<float>(ws, L.a1_scale) : nullptr,
+                               swap ? at<int>(ws, L.tile_counters) : nullptr, swap ? n_counters : 0, stream);
         if (e != cudaSuccess) return cuda_fail(e, "gather");
         break;
       case MOE_STAGE_GEMM1:
@@ -251,6 +287,11 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
         gp.topk_weights = wts;
         gp.status = status;
         gp.num_sms = sms;
+        gp.split_mode = p.split_k;
+        gp.partials1 = swap ? at<float>(ws, L.partials) : nullptr;
+        gp.partials2 = gp.partials1;
+        gp.counters1 = swap ? at<int>(ws, L.tile_counters) : nullptr;
+        gp.counters2 = swap ? at<int>(ws, L.tile_counters) + (cap / p.block_m) * (p.I / 128) : nullptr;
         if (s == MOE_STAGE_GEMM1) {
           e = moe::launch_gemm1(gp, at<void>(ws, L.a1), plan.fp8 ? at<float>(ws, L.a1_scale) : nullptr, w13,
                                 w13_scale, at<void>(ws, L.a2), plan.fp8 ? at<float>(ws, L.a2_scale) : nullptr,
@@ -343,6 +384,13 @@ int moe_align(const int32_t* topk_ids, int32_t T, int32_t topk, int32_t E, int32
     e = cudaMemsetAsync(num_tokens_post_padded, 0, sizeof(int32_t), s);
     if (e == cudaSuccess && expert_counts) e = cudaMemsetAsync(expert_counts, 0, E * sizeof(int32_t), s);
     if (e == cudaSuccess && expert_offsets) e = cudaMemsetAsync(expert_offsets, 0, (E + 1) * sizeof(int32_t), s);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "align");
+  }
+  if (moe::route_align_small_fits(n, E)) {
+    e = moe::launch_route_align_small(nullptr, topk_ids, T, E, topk, 1, nullptr, nullptr, block_m,
+                                      static_cast<int>(cap), sorted_token_ids, expert_ids, num_tokens_post_padded,
+                                      expert_counts ? expert_counts : counts, expert_offsets ? expert_offsets : offs,
+                                      status, s);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "align");
   }
   e = moe::launch_align(topk_ids, static_cast<int>(n), E, block_m, static_cast<int>(cap), sorted_token_ids,

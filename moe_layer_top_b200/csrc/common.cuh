@@ -90,6 +90,22 @@ __device__ __forceinline__ bool mbar_wait(uint64_t* bar, uint32_t parity, volati
 }
 
 // --------------------------------------------------------------------------
+// programmatic dependent launch: every kernel of the pipeline lets the next
+// one launch once all of its CTAs are resident, and waits for the previous
+// one to complete (and its memory to be visible) before reading its outputs.
+// Both are no-ops when the kernel was launched without the attribute.
+// Kernels that wait use plain global loads only -- no __ldg and no
+// const __restrict__ pointers: those compile to invariant non-coherent loads
+// that the compiler may hoist above the wait, reading data the previous
+// kernel has not written yet.
+// --------------------------------------------------------------------------
+__device__ __forceinline__ void pdl_launch_dependents() {
+  asm volatile("griddepcontrol.launch_dependents;" ::: "memory");
+}
+
+__device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
+
+// --------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast
 // --------------------------------------------------------------------------
 __device__ __forceinline__ void tma_prefetch_desc(const void* map) {
@@ -194,6 +210,56 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
       : "r"(taddr));
 #pragma unroll
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
+}
+
+// 32 lanes x 32 consecutive 32-bit columns (raw bits)
+__device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x32.b32 "
+      "{%0, %1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, "
+      "%16, %17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31}, [%32];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7]),
+        "=r"(r[8]), "=r"(r[9]), "=r"(r[10]), "=r"(r[11]), "=r"(r[12]), "=r"(r[13]), "=r"(r[14]), "=r"(r[15]),
+        "=r"(r[16]), "=r"(r[17]), "=r"(r[18]), "=r"(r[19]), "=r"(r[20]), "=r"(r[21]), "=r"(r[22]), "=r"(r[23]),
+        "=r"(r[24]), "=r"(r[25]), "=r"(r[26]), "=r"(r[27]), "=r"(r[28]), "=r"(r[29]), "=r"(r[30]), "=r"(r[31])
+      : "r"(taddr));
+}
+
+__device__ __forceinline__ void tmem_st32(uint32_t taddr, const uint32_t (&r)[32]) {
+  asm volatile(
+      "tcgen05.st.sync.aligned.32x32b.x32.b32 [%0], "
+      "{%1, %2, %3, %4, %5, %6, %7, %8, %9, %10, %11, %12, %13, %14, %15, %16, "
+      "%17, %18, %19, %20, %21, %22, %23, %24, %25, %26, %27, %28, %29, %30, %31, %32};" ::"r"(taddr),
+      "r"(r[0]), "r"(r[1]), "r"(r[2]), "r"(r[3]), "r"(r[4]), "r"(r[5]), "r"(r[6]), "r"(r[7]), "r"(r[8]),
+      "r"(r[9]), "r"(r[10]), "r"(r[11]), "r"(r[12]), "r"(r[13]), "r"(r[14]), "r"(r[15]), "r"(r[16]),
+      "r"(r[17]), "r"(r[18]), "r"(r[19]), "r"(r[20]), "r"(r[21]), "r"(r[22]), "r"(r[23]), "r"(r[24]),
+      "r"(r[25]), "r"(r[26]), "r"(r[27]), "r"(r[28]), "r"(r[29]), "r"(r[30]), "r"(r[31])
+      : "memory");
+}
+
+__device__ __forceinline__ void tmem_wait_st() { asm volatile("tcgen05.wait::st.sync.aligned;" ::: "memory"); }
+
+// two fp32 lanes at once: (a0, a1) <- (d0, d1) * (f, f) + (a0, a1), each correctly rounded
+__device__ __forceinline__ void ffma2(uint32_t& a0, uint32_t& a1, uint32_t d0, uint32_t d1, float f) {
+  asm("{\n\t.reg .b64 ra, rd, rf;\n\t"
+      "mov.b64 ra, {%0, %1};\n\t"
+      "mov.b64 rd, {%2, %3};\n\t"
+      "mov.b64 rf, {%4, %4};\n\t"
+      "fma.rn.f32x2 ra, rd, rf, ra;\n\t"
+      "mov.b64 {%0, %1}, ra;\n\t}"
+      : "+r"(a0), "+r"(a1)
+      : "r"(d0), "r"(d1), "r"(__float_as_uint(f)));
+}
+
+// (a0, a1) <- (d0, d1) * (f, f)
+__device__ __forceinline__ void fmul2(uint32_t& a0, uint32_t& a1, uint32_t d0, uint32_t d1, float f) {
+  asm("{\n\t.reg .b64 ra, rd, rf;\n\t"
+      "mov.b64 rd, {%2, %3};\n\t"
+      "mov.b64 rf, {%4, %4};\n\t"
+      "mul.rn.f32x2 ra, rd, rf;\n\t"
+      "mov.b64 {%0, %1}, ra;\n\t}"
+      : "=r"(a0), "=r"(a1)
+      : "r"(d0), "r"(d1), "r"(__float_as_uint(f)));
 }
 
 // Shared-memory matrix descriptor of a K-major tile written by TMA with the

@@ -33,30 +33,35 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
 }  // namespace
 
 // ----------------------------------------------------------------------------
-// gather: a1[r] = x[sorted_ids[r] / topk] for r < num_tokens_post_padded
-// (zeros for padding rows).  FP8: per (row, 128 columns) the power-of-two
+// gather: a1[r] = x[sorted_ids[r] / topk] for the real rows r <
+// num_tokens_post_padded; padding rows are not written.  FP8: per (row, 128 columns) the power-of-two
 // scale of the vLLM PR #64760 analysis §1.2 rule, codes into a1 [cap, H],
 // scales into a1_scale_t [H/128, cap] (K-block major for the GEMM epilogue).
 // A block walks rows; a thread owns 8 consecutive columns, 16 threads one
 // 128-column group.
 // ----------------------------------------------------------------------------
 template <bool FP8>
-__global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* __restrict__ x, int H, int topk,
-                                                     int nflat, const int32_t* __restrict__ sorted_ids,
-                                                     const int32_t* __restrict__ ntpp_ptr, int capacity,
-                                                     void* __restrict__ a1, float* __restrict__ a1_scale_t) {
+__global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* x, int H, int topk,
+                                                     int nflat, const int32_t* sorted_ids,
+                                                     const int32_t* ntpp_ptr, int capacity,
+                                                     void* a1, float* a1_scale_t, int* zero, int zero_n) {
+  pdl_launch_dependents();
+  pdl_wait();
+  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < zero_n; i += gridDim.x * blockDim.x) zero[i] = 0;
   const int ntpp = *ntpp_ptr;
   const int vecs = H / 8;
   const int iters = (vecs + blockDim.x - 1) / blockDim.x;
   for (int row = blockIdx.x; row < ntpp; row += gridDim.x) {
-    const int flat = __ldg(sorted_ids + row);
-    const bool real = flat < nflat;
-    const __nv_bfloat16* src = x + static_cast<size_t>(real ? flat / topk : 0) * H;
+    const int flat = (*(sorted_ids + row));
+    // padding rows are left as they are: every GEMM output row and column
+    // depends only on its own input row, and padding outputs are never stored
+    if (flat >= nflat) continue;
+    const __nv_bfloat16* src = x + static_cast<size_t>(flat / topk) * H;
     for (int it = 0; it < iters; ++it) {
       const int v = it * blockDim.x + threadIdx.x;  // uniform trip count: shuffles below see full warps
       const bool in = v < vecs;
       uint4 u = make_uint4(0, 0, 0, 0);
-      if (in && real) u = __ldg(reinterpret_cast<const uint4*>(src) + v);
+      if (in) u = (*(reinterpret_cast<const uint4*>(src) + v));
       if constexpr (!FP8) {
         if (in) reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a1) + static_cast<size_t>(row) * H)[v] = u;
       } else {
@@ -84,17 +89,16 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* __rest
 }
 
 cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32_t* sorted_ids,
-                          const int32_t* ntpp, int capacity, bool fp8, void* a1, float* a1_scale_t,
-                          cudaStream_t stream) {
+                          const int32_t* ntpp, int capacity, bool fp8, void* a1, float* a1_scale_t, int* zero,
+                          int zero_n, cudaStream_t stream) {
   if (capacity == 0) return cudaSuccess;
   int blocks = capacity < 148 * 8 ? capacity : 148 * 8;
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (fp8)
-    gather_kernel<true><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), H, topk, nflat, sorted_ids,
-                                                    ntpp, capacity, a1, a1_scale_t);
-  else
-    gather_kernel<false><<<blocks, 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(x), H, topk, nflat,
-                                                     sorted_ids, ntpp, capacity, a1, a1_scale_t);
-  return cudaGetLastError();
+    return launch_pdl(gather_kernel<true>, blocks, 256, 0, stream, xb, H, topk, nflat, sorted_ids, ntpp, capacity, a1,
+                      a1_scale_t, zero, zero_n);
+  return launch_pdl(gather_kernel<false>, blocks, 256, 0, stream, xb, H, topk, nflat, sorted_ids, ntpp, capacity, a1,
+                    a1_scale_t, zero, zero_n);
 }
 
 // ----------------------------------------------------------------------------
@@ -102,8 +106,10 @@ cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32
 // weighted accumulation; the weights were applied in the GEMM2 epilogue):
 // out[t, :] = bf16(sum_j y[t*topk + j, :]) in fp32, j ascending.
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __restrict__ y, int T, int topk, int H,
-                                                      __nv_bfloat16* __restrict__ out) {
+__global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* y, int T, int topk, int H,
+                                                      __nv_bfloat16* out) {
+  pdl_launch_dependents();
+  pdl_wait();
   const int vecs = H / 8;
   const long long total = static_cast<long long>(T) * vecs;
   for (long long i = blockIdx.x * static_cast<long long>(blockDim.x) + threadIdx.x; i < total;
@@ -114,7 +120,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* __res
     const uint4* src = reinterpret_cast<const uint4*>(y + static_cast<size_t>(t) * topk * H) + v;
     for (int j = 0; j < topk; ++j) {
       float f[8];
-      unpack8(__ldg(src + static_cast<size_t>(j) * vecs), f);
+      unpack8((*(src + static_cast<size_t>(j) * vecs)), f);
 #pragma unroll
       for (int k = 0; k < 8; ++k) acc[k] += f[k];
     }
@@ -127,9 +133,8 @@ cudaError_t launch_combine(const void* y, int T, int topk, int H, void* out, cud
   const long long total = static_cast<long long>(T) * (H / 8);
   long long blocks = (total + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  combine_kernel<<<static_cast<int>(blocks), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(y), T, topk, H,
-                                                               static_cast<__nv_bfloat16*>(out));
-  return cudaGetLastError();
+  return launch_pdl(combine_kernel, static_cast<int>(blocks), 256, 0, stream, static_cast<const __nv_bfloat16*>(y), T,
+                    topk, H, static_cast<__nv_bfloat16*>(out));
 }
 
 // ----------------------------------------------------------------------------
@@ -137,10 +142,12 @@ cudaError_t launch_combine(const void* y, int T, int topk, int H, void* out, cud
 // elements).  scale = max(blockmax, 1e-10) / 448 and code = e4m3(w / scale),
 // both divisions correctly rounded in fp32.
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) quantize_weights_kernel(const __nv_bfloat16* __restrict__ w, int rows,
-                                                               int cols, uint8_t* __restrict__ codes,
-                                                               float* __restrict__ scales) {
+__global__ void __launch_bounds__(256) quantize_weights_kernel(const __nv_bfloat16* w, int rows,
+                                                               int cols, uint8_t* codes,
+                                                               float* scales) {
   __shared__ float warp_max[8];
+  pdl_launch_dependents();
+  pdl_wait();
   const int nbc = cols / 128, nbr = rows / 128;
   const long long blk = blockIdx.x;
   const long long b = blk / (static_cast<long long>(nbr) * nbc);
@@ -155,7 +162,7 @@ __global__ void __launch_bounds__(256) quantize_weights_kernel(const __nv_bfloat
 #pragma unroll
   for (int i = 0; i < 8; ++i) {
     float t[8];
-    unpack8(__ldg(src + i), t);
+    unpack8((*(src + i)), t);
 #pragma unroll
     for (int k = 0; k < 8; ++k) {
       f[8 * i + k] = t[k];
@@ -191,9 +198,8 @@ cudaError_t launch_quantize_weights(const void* w, long long batches, int rows, 
   const long long blocks = batches * (rows / 128) * (cols / 128);
   if (blocks == 0) return cudaSuccess;
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
-  quantize_weights_kernel<<<static_cast<unsigned>(blocks), 256, 0, stream>>>(static_cast<const __nv_bfloat16*>(w),
-                                                                            rows, cols, codes, scales);
-  return cudaGetLastError();
+  return launch_pdl(quantize_weights_kernel, static_cast<unsigned>(blocks), 256, 0, stream,
+                    static_cast<const __nv_bfloat16*>(w), rows, cols, codes, scales);
 }
 
 }  // namespace moe

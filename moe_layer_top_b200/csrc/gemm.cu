@@ -40,7 +40,7 @@ constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
 constexpr int kSmemLimit = 232448;  // max dynamic shared memory per block on sm_100
 constexpr int kSmemReserve = 4096;  // barriers, TMEM slot, exchange buffers
-constexpr int kXchgOffset = 512;    // exchange buffers start here inside the reserve
+constexpr int kXchgOffset = 512;    // exchange buffers (2 x 256 floats) and the split-K ticket start here
 
 // wait-site codes reported in the status word (low byte)
 constexpr int kWhereProducer = 1, kWhereMma = 2, kWhereEpiAcc = 3, kWhereEpiXchg = 4, kWhereDrain = 5;
@@ -84,7 +84,37 @@ struct Args {
   void* out;               // GEMM1: a2 [capacity, I]; GEMM2: y [nflat, H]
   float* out_scale_t;      // GEMM1 FP8: a2 scale [I/128, capacity]
   int* status;
+  float* partials;         // swap-AB split-K: [unit][acc column][128] fp32 partial sums
+  int* tile_counters;      // swap-AB split-K: arrivals per tile (zero between launches)
+  int split_mode;          // 0: chosen from the tile count, 1: no split
 };
+
+// Split-K for the swap-AB tiles: when so few tiles are in flight that most
+// SMs would idle, the K range of every tile is cut in S pieces.  The splits
+// publish fp32 partial sums and the last one to arrive adds them in split
+// order (fence, barrier, atomic ticket, barrier, fence, reload): under full
+// HBM load that hand-off costs several microseconds per tile, more than the
+// balance it buys once at least half of the SMs have a tile, so it is used
+// only below that.  S is a pure function of (tiles, CTAs, K stages), so every
+// role and CTA agree on it and the result is deterministic.  A split needs
+// >= 4 stages and the launch at most kMaxSplitUnits units (the buffer).
+constexpr int kMaxSplits = 4;
+
+__device__ __forceinline__ int choose_splits(int tiles, int ctas, int k_stages, int mode) {
+  if (mode == 1 || tiles <= 0 || 2 * tiles > ctas) return 1;
+  int best = 1;
+  long long best_u = tiles, best_w = (tiles + ctas - 1) / ctas;  // efficiency = u / (ctas * w)
+  for (int sp = 2; sp <= kMaxSplits; ++sp) {
+    if (k_stages / sp < 4 || static_cast<long long>(tiles) * sp > kMaxSplitUnits) break;
+    const long long u = static_cast<long long>(tiles) * sp, w = (u + ctas - 1) / ctas;
+    if (u * best_w * 100 > best_u * w * 105) {  // at least 5 % better
+      best = sp;
+      best_u = u;
+      best_w = w;
+    }
+  }
+  return best;
+}
 
 __device__ __forceinline__ bool warp_wait(uint64_t* bar, uint32_t parity, volatile int* abort, int* status,
                                           int where) {
@@ -120,6 +150,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* xchg = reinterpret_cast<float*>(reserve + kXchgOffset);  // [2][2 * 128] floats
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -146,14 +177,17 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();  // everything above overlapped the previous kernel's tail
 
   const int H = args.H, I = args.I;
   const int K = kDown ? I : H;                           // reduction length
   const int rows_per_block = C::kTokRows;                // == block_m of the alignment
   const int n_tiles = (kDown ? H : I) / C::kTileN;
-  const int num_mblocks = __ldg(args.ntpp) / rows_per_block;
+  const int num_mblocks = (*(args.ntpp)) / rows_per_block;
   const int num_tiles = num_mblocks * n_tiles;
   const int k_stages = K / C::kKElems;
+  const int splits = kSwap ? choose_splits(num_tiles, gridDim.x, k_stages, args.split_mode) : 1;
+  const int num_units = num_tiles * splits;
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
@@ -164,9 +198,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       uint32_t phase = 0;
       long long fills = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x) {
+        const int tile = unit / splits, split = unit - tile * splits;
+        const int ks0 = split * k_stages / splits, ks1 = (split + 1) * k_stages / splits;
         const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
-        const int e = __ldg(args.expert_ids + mb);
+        const int e = (*(args.expert_ids + mb));
         const int tok_row = mb * rows_per_block;
         int w_row0, w_row1;
         if constexpr (kDown) {
@@ -176,7 +212,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           w_row0 = e * 2 * I + nt * 128;      // gate rows
           w_row1 = w_row0 + I;                // up rows
         }
-        for (int ks = 0; ks < k_stages; ++ks) {
+        for (int ks = ks0; ks < ks1; ++ks) {
           if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status,
                          MOE_STATUS_WAIT_TIMEOUT | kWhereProducer)) {
             ok = false;
@@ -219,7 +255,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       int stage = 0, abuf = 0;
       uint32_t phase = 0, aphase = 0;
       bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x) {
+        const int split = unit % splits;
+        const int ks0 = split * k_stages / splits, ks1 = (split + 1) * k_stages / splits;
         if constexpr (!kFP8) {
           if (!mbar_wait(&acc_empty[abuf], aphase ^ 1u, abort_flag, args.status,
                          MOE_STATUS_WAIT_TIMEOUT | kWhereMma)) {
@@ -228,7 +266,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
           tc_fence_after();
         }
-        for (int ks = 0; ks < k_stages; ++ks) {
+        for (int ks = ks0; ks < ks1; ++ks) {
           if (!mbar_wait(&full[stage], phase, abort_flag, args.status, MOE_STATUS_WAIT_TIMEOUT | kWhereMma)) {
             ok = false;
             break;
@@ -247,7 +285,7 @@ __global__ void __launch_bounds__(kThreads, 1)
 #pragma unroll
           for (int k = 0; k < 4; ++k) {
             const uint32_t koff = k * 32;  // 16 bf16 or 32 e4m3 elements
-            const uint32_t acc = kFP8 ? (k > 0 ? 1u : 0u) : ((ks > 0 || k > 0) ? 1u : 0u);
+            const uint32_t acc = kFP8 ? (k > 0 ? 1u : 0u) : ((ks > ks0 || k > 0) ? 1u : 0u);
             if constexpr (!kSwap) {
               const uint64_t ad = smem_desc_sw128(tok + koff), bd = smem_desc_sw128(w + koff);
               if constexpr (kFP8) mma_fp8(d, ad, bd, idesc, acc); else mma_bf16(d, ad, bd, idesc, acc);
@@ -306,9 +344,11 @@ __global__ void __launch_bounds__(kThreads, 1)
     int xbuf = 0;
     uint32_t xphase = 0;
     bool ok = true;
-    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+    for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x) {
+      const int tile = unit / splits, split = unit - tile * splits;
+      const int ks0 = split * k_stages / splits, ks1 = (split + 1) * k_stages / splits;
       const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
-      const int e = __ldg(args.expert_ids + mb);
+      const int e = (*(args.expert_ids + mb));
 
       if constexpr (!kSwap) {
         // ---------------- normal: row = token row of the tile
@@ -334,12 +374,12 @@ __global__ void __launch_bounds__(kThreads, 1)
             sw_a = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + nt) * kb_n;
             sw_b = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + I / 128 + nt) * kb_n;
           }
-          float sa_next = __ldg(sa_p);
+          float sa_next = (*(sa_p));
           for (int kb = 0; kb < kb_n; ++kb) {
             const float sa = sa_next;
-            if (kb + 1 < kb_n) sa_next = __ldg(sa_p + static_cast<size_t>(kb + 1) * args.capacity);
-            const float fa = sa * __ldg(sw_a + kb);
-            const float fb = sa * __ldg(sw_b + kb);
+            if (kb + 1 < kb_n) sa_next = (*(sa_p + static_cast<size_t>(kb + 1) * args.capacity));
+            const float fa = sa * (*(sw_a + kb));
+            const float fb = sa * (*(sw_b + kb));
             if (!warp_wait(&acc_full[abuf], aphase, abort_flag, args.status, kWhereEpiAcc)) {
               ok = false;
               break;
@@ -450,9 +490,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           // ---- GEMM2 epilogue: routed weight, scatter the row to y[flat]
-          const int flat = __ldg(args.sorted_ids + grow);
+          const int flat = (*(args.sorted_ids + grow));
           const bool real = flat < args.nflat;
-          const float wt = real ? __ldg(args.topk_weights + flat) : 0.f;
+          const float wt = real ? (*(args.topk_weights + flat)) : 0.f;
           __nv_bfloat16* yrow =
               static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(real ? flat : 0) * H + nt * 256 + g * 128;
           if constexpr (kFP8) {
@@ -523,13 +563,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             sw_a = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + nt) * kb_n;
             sw_b = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + I / 128 + nt) * kb_n;
           }
-          for (int kb = 0; kb < kb_n; ++kb) {
-            const float swa = __ldg(sw_a + kb);
-            const float swb = __ldg(sw_b + kb);
+          for (int kb = ks0; kb < ks1; ++kb) {
+            const float swa = (*(sw_a + kb));
+            const float swb = (*(sw_b + kb));
             const float* sa_p = args.a_scale_t + static_cast<size_t>(kb) * args.capacity + tok0;
             float fa[kHT];
 #pragma unroll
-            for (int j = 0; j < kHT; ++j) fa[j] = __ldg(sa_p + j);
+            for (int j = 0; j < kHT; ++j) fa[j] = (*(sa_p + j));
             if (!warp_wait(&acc_full[abuf], aphase, abort_flag, args.status, kWhereEpiAcc)) {
               ok = false;
               break;
@@ -581,6 +621,53 @@ __global__ void __launch_bounds__(kThreads, 1)
           if (abuf == 0) aphase ^= 1u;
         }
 
+        if (splits > 1) {
+          // ---- split-K: publish this split's partial sums; the last split of
+          // the tile to arrive adds all of them in split order and goes on.
+          constexpr int kAccW = kDown ? kBM : 2 * kBM;
+          float* part = args.partials + static_cast<size_t>(unit) * (kAccW * 128);
+#pragma unroll
+          for (int j = 0; j < kHT; ++j) {
+            part[(col_a + j) * 128 + row] = acc_a[j];
+            if constexpr (!kDown) part[(col_b + j) * 128 + row] = acc_b[j];
+          }
+          __threadfence();
+          mbar_arrive(&xchg_bar[xbuf]);
+          if (!warp_wait(&xchg_bar[xbuf], xphase, abort_flag, args.status, kWhereEpiXchg)) {
+            ok = false;
+            break;
+          }
+          // the ticket gets a slot of its own: the exchange buffers are reused by the
+          // FP8 amax exchange right after, possibly before every warp has read it
+          volatile int* ticket_slot = reinterpret_cast<volatile int*>(xchg + 512);
+          if (warp == 2 && lane == 0) *ticket_slot = atomicAdd(args.tile_counters + tile, 1);
+          xbuf ^= 1;
+          if (xbuf == 0) xphase ^= 1u;
+          mbar_arrive(&xchg_bar[xbuf]);
+          if (!warp_wait(&xchg_bar[xbuf], xphase, abort_flag, args.status, kWhereEpiXchg)) {
+            ok = false;
+            break;
+          }
+          const int ticket = *ticket_slot;
+          xbuf ^= 1;
+          if (xbuf == 0) xphase ^= 1u;
+          if (ticket != splits - 1) continue;
+          __threadfence();
+          if (warp == 2 && lane == 0) args.tile_counters[tile] = 0;  // ready for the next launch
+          const float* tile_part = args.partials + static_cast<size_t>(tile) * splits * (kAccW * 128);
+#pragma unroll
+          for (int j = 0; j < kHT; ++j) {
+            float sa = 0.f, sb = 0.f;
+            for (int sp = 0; sp < splits; ++sp) {
+              const float* ps = tile_part + static_cast<size_t>(sp) * (kAccW * 128);
+              sa += (sp == split) ? acc_a[j] : __ldcg(ps + (col_a + j) * 128 + row);
+              if constexpr (!kDown) sb += (sp == split) ? acc_b[j] : __ldcg(ps + (col_b + j) * 128 + row);
+            }
+            acc_a[j] = sa;
+            if constexpr (!kDown) acc_b[j] = sb;
+          }
+        }
+
         if constexpr (!kDown) {
           // ---- GEMM1: this thread owns intermediate column nt*128 + row for kHT tokens
           const int icol = nt * 128 + row;
@@ -627,9 +714,9 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int hcol = nt * 128 + row;
 #pragma unroll
           for (int j = 0; j < kHT; ++j) {
-            const int flat = __ldg(args.sorted_ids + tok0 + j);
+            const int flat = (*(args.sorted_ids + tok0 + j));
             if (flat < args.nflat) {
-              const float wt = __ldg(args.topk_weights + flat);
+              const float wt = (*(args.topk_weights + flat));
               y[static_cast<size_t>(flat) * H + hcol] = __float2bfloat16_rn(acc_a[j] * wt);
             }
           }
@@ -696,12 +783,11 @@ cudaError_t launch_on(const GemmProblem& p, const void* tok, const void* w, cons
   if (!make_map(&tm_tok, tok, p.capacity, K, elem, C::kTokRows)) return cudaErrorInvalidValue;
   if (!make_map(&tm_w, w, wrows, K, elem, kDown ? C::kWRows : 128)) return cudaErrorInvalidValue;
   const int n_tiles = (kDown ? p.H : p.I) / C::kTileN;
-  const long long max_tiles = static_cast<long long>(p.capacity / C::kTokRows) * n_tiles;
+  const long long max_units = static_cast<long long>(p.capacity / C::kTokRows) * n_tiles * (kSwap ? kMaxSplits : 1);
   int grid = p.num_sms;
-  if (max_tiles < grid) grid = static_cast<int>(max_tiles);
+  if (max_units < grid) grid = static_cast<int>(max_units);
   if (grid <= 0) return cudaSuccess;
-  kern<<<grid, kThreads, C::kSmemBytes, s>>>(tm_tok, tm_w, args);
-  return cudaGetLastError();
+  return launch_pdl(kern, grid, kThreads, C::kSmemBytes, s, tm_tok, tm_w, args);
 }
 
 template <bool kDown, bool kFP8>
@@ -739,6 +825,9 @@ cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const float* a1_s
   args.out = a2;
   args.out_scale_t = a2_scale_t;
   args.status = p.status;
+  args.partials = p.partials1;
+  args.tile_counters = p.counters1;
+  args.split_mode = p.split_mode;
   return p.fp8 ? dispatch<false, true>(p, a1, w13, args, stream) : dispatch<false, false>(p, a1, w13, args, stream);
 }
 
@@ -759,6 +848,9 @@ cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const float* a2_s
   args.out = y;
   args.out_scale_t = nullptr;
   args.status = p.status;
+  args.partials = p.partials2;
+  args.tile_counters = p.counters2;
+  args.split_mode = p.split_mode;
   return p.fp8 ? dispatch<true, true>(p, a2, w2, args, stream) : dispatch<true, false>(p, a2, w2, args, stream);
 }
 

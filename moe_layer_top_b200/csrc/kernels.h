@@ -7,6 +7,25 @@
 
 namespace moe {
 
+// Launch `kern` on `stream` with programmatic stream serialisation, so that
+// it may start while the previous kernel of the stream finishes (each kernel
+// calls griddepcontrol.wait before it reads what its predecessors wrote).
+template <typename... KArgs, typename... Args>
+cudaError_t launch_pdl(void (*kern)(KArgs...), dim3 grid, dim3 block, size_t smem, cudaStream_t stream,
+                       Args&&... args) {
+  cudaLaunchConfig_t cfg = {};
+  cfg.gridDim = grid;
+  cfg.blockDim = block;
+  cfg.dynamicSmemBytes = smem;
+  cfg.stream = stream;
+  cudaLaunchAttribute attr[1];
+  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
+  attr[0].val.programmaticStreamSerializationAllowed = 1;
+  cfg.attrs = attr;
+  cfg.numAttrs = 1;
+  return cudaLaunchKernelEx(&cfg, kern, static_cast<KArgs>(args)...);
+}
+
 // router ---------------------------------------------------------------------
 cudaError_t launch_route(const float* logits, int T, int E, int topk, int renormalize, int32_t* ids,
                          float* weights, cudaStream_t stream);
@@ -20,10 +39,20 @@ cudaError_t launch_align(const int32_t* topk_ids, int n, int E, int block_m, int
                          int32_t* offsets_ws, int32_t* chunk_scratch, int32_t* user_counts,
                          int32_t* user_offsets, int* status, cudaStream_t stream);
 
-// gather x rows into sorted order (bf16 copy, or FP8 per-(row,128) quantisation)
+// single-CTA route (optional) + align for small batches
+constexpr int kSmallAlignMaxN = 8192;  // assignments (T * topk)
+constexpr int kSmallAlignMaxE = 256;
+bool route_align_small_fits(long long n, int E);
+cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in, int T, int E, int topk,
+                                     int renormalize, int32_t* ids_out, float* weights_out, int block_m, int capacity,
+                                     int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp, int32_t* counts,
+                                     int32_t* offsets, int* status, cudaStream_t stream);
+
+// gather x rows into sorted order (bf16 copy, or FP8 per-(row,128) quantisation);
+// also zeroes `zero_n` ints at `zero` (the split-K tile counters of the GEMMs)
 cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32_t* sorted_ids,
-                          const int32_t* ntpp, int capacity, bool fp8, void* a1, float* a1_scale_t,
-                          cudaStream_t stream);
+                          const int32_t* ntpp, int capacity, bool fp8, void* a1, float* a1_scale_t, int* zero,
+                          int zero_n, cudaStream_t stream);
 
 // out[t] = sum_j y[t*topk + j]
 cudaError_t launch_combine(const void* y, int T, int topk, int H, void* out, cudaStream_t stream);
@@ -42,7 +71,15 @@ struct GemmProblem {
   const float* topk_weights;  // [nflat]
   int* status;
   int num_sms;
+  int split_mode;      // 0 auto, 1 off (swap-AB split-K)
+  float* partials1;    // split-K partial sums of GEMM1 / GEMM2 (swap-AB)
+  float* partials2;
+  int* counters1;      // per-tile arrival counters, zero before the launch
+  int* counters2;
 };
+
+// swap-AB split-K: at most this many (tile, split) units per launch
+constexpr int kMaxSplitUnits = 1024;
 
 // GEMM1 + fused SiLU*up (+ FP8 requant): a1 [cap, H] -> a2 [cap, I] (+ a2_scale_t [I/128, cap])
 cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const float* a1_scale_t, const void* w13,

@@ -28,21 +28,18 @@ namespace moe {
 // ----------------------------------------------------------------------------
 // router
 // ----------------------------------------------------------------------------
+// One warp routes one token: lane r (< topk) returns the r-th chosen expert
+// and its weight.
 template <int VPL>  // logits per lane (E <= 32 * VPL)
-__global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ logits, int T, int E, int topk,
-                                                    int renormalize, int32_t* __restrict__ ids,
-                                                    float* __restrict__ weights) {
-  const int lane = threadIdx.x & 31;
-  const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
-  if (tok >= T) return;
-  const float* row = logits + static_cast<size_t>(tok) * E;
+__device__ __forceinline__ void route_token(const float* row, int E, int topk, int renormalize,
+                                            int lane, int& out_id, float& out_w) {
 
   float v[VPL];
   uint32_t taken = 0;
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = lane + 32 * i;
-    v[i] = (e < E) ? __ldg(row + e) : -INFINITY;
+    v[i] = (e < E) ? (*(row + e)) : -INFINITY;
     if (e >= E) taken |= 1u << i;
   }
   // softmax statistics over all experts
@@ -92,10 +89,26 @@ __global__ void __launch_bounds__(256) route_kernel(const float* __restrict__ lo
   float s = ex;
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
+  out_id = my_id;
+  out_w = renormalize ? __fdiv_rn(ex, s) : __fdiv_rn(ex, z);
+}
+
+template <int VPL>
+__global__ void __launch_bounds__(256) route_kernel(const float* logits, int T, int E, int topk,
+                                                    int renormalize, int32_t* ids,
+                                                    float* weights) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int lane = threadIdx.x & 31;
+  const int tok = (blockIdx.x * blockDim.x + threadIdx.x) >> 5;
+  if (tok >= T) return;
+  int id;
+  float w;
+  route_token<VPL>(logits + static_cast<size_t>(tok) * E, E, topk, renormalize, lane, id, w);
   if (lane < topk) {
     const size_t o = static_cast<size_t>(tok) * topk + lane;
-    ids[o] = my_id;
-    weights[o] = renormalize ? __fdiv_rn(ex, s) : __fdiv_rn(ex, z);
+    ids[o] = id;
+    weights[o] = w;
   }
 }
 
@@ -105,14 +118,12 @@ cudaError_t launch_route(const float* logits, int T, int E, int topk, int renorm
   const int threads = 256;
   const int blocks = static_cast<int>((static_cast<long long>(T) * 32 + threads - 1) / threads);
   if (E <= 128)
-    route_kernel<4><<<blocks, threads, 0, stream>>>(logits, T, E, topk, renormalize, ids, weights);
-  else if (E <= 256)
-    route_kernel<8><<<blocks, threads, 0, stream>>>(logits, T, E, topk, renormalize, ids, weights);
-  else if (E <= 512)
-    route_kernel<16><<<blocks, threads, 0, stream>>>(logits, T, E, topk, renormalize, ids, weights);
-  else
-    route_kernel<32><<<blocks, threads, 0, stream>>>(logits, T, E, topk, renormalize, ids, weights);
-  return cudaGetLastError();
+    return launch_pdl(route_kernel<4>, blocks, threads, 0, stream, logits, T, E, topk, renormalize, ids, weights);
+  if (E <= 256)
+    return launch_pdl(route_kernel<8>, blocks, threads, 0, stream, logits, T, E, topk, renormalize, ids, weights);
+  if (E <= 512)
+    return launch_pdl(route_kernel<16>, blocks, threads, 0, stream, logits, T, E, topk, renormalize, ids, weights);
+  return launch_pdl(route_kernel<32>, blocks, threads, 0, stream, logits, T, E, topk, renormalize, ids, weights);
 }
 
 // ----------------------------------------------------------------------------
@@ -120,11 +131,13 @@ cudaError_t launch_route(const float* logits, int T, int E, int topk, int renorm
 // ----------------------------------------------------------------------------
 constexpr int kAlignWarps = 8;
 
-__global__ void __launch_bounds__(kAlignWarps * 32) align_count_kernel(const int32_t* __restrict__ ids, int n,
+__global__ void __launch_bounds__(kAlignWarps * 32) align_count_kernel(const int32_t* ids, int n,
                                                                        int E, int nchunks,
-                                                                       int32_t* __restrict__ chunk_counts,
+                                                                       int32_t* chunk_counts,
                                                                        int* status) {
   extern __shared__ int32_t hist_all[];
+  pdl_launch_dependents();
+  pdl_wait();
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
   const int chunk = blockIdx.x * kAlignWarps + warp;
   if (chunk >= nchunks) return;
@@ -135,7 +148,7 @@ __global__ void __launch_bounds__(kAlignWarps * 32) align_count_kernel(const int
   for (int i = lane; i < kAlignChunk; i += 32) {
     const int f = base + i;
     if (f < n) {
-      const int e = __ldg(ids + f);
+      const int e = (*(ids + f));
       if (e >= 0 && e < E)
         atomicAdd(&hist[e], 1);
       else
@@ -150,10 +163,12 @@ __global__ void __launch_bounds__(kAlignWarps * 32) align_count_kernel(const int
 // ----------------------------------------------------------------------------
 // align pass 2: per expert, exclusive scan over chunks (in place) and total
 // ----------------------------------------------------------------------------
-__global__ void __launch_bounds__(256) align_scan_kernel(int32_t* __restrict__ chunk_counts, int nchunks, int E,
-                                                         int32_t* __restrict__ counts_ws,
-                                                         int32_t* __restrict__ user_counts) {
+__global__ void __launch_bounds__(256) align_scan_kernel(int32_t* chunk_counts, int nchunks, int E,
+                                                         int32_t* counts_ws,
+                                                         int32_t* user_counts) {
   __shared__ int32_t warp_sums[8];
+  pdl_launch_dependents();
+  pdl_wait();
   const int e = blockIdx.x;
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
   int32_t carry = 0;
@@ -202,15 +217,17 @@ __device__ __forceinline__ int owner_expert(const int32_t* offs, int E, int p) {
 }
 
 __global__ void __launch_bounds__(kAlignWarps * 32) align_scatter_kernel(
-    const int32_t* __restrict__ ids, int n, int E, int block_m, int capacity, int nchunks,
-    const int32_t* __restrict__ chunk_base, const int32_t* __restrict__ counts_ws, int32_t* __restrict__ sorted_ids,
-    int32_t* __restrict__ expert_ids, int32_t* __restrict__ ntpp_out, int32_t* __restrict__ offsets_ws,
-    int32_t* __restrict__ user_offsets) {
+    const int32_t* ids, int n, int E, int block_m, int capacity, int nchunks,
+    const int32_t* chunk_base, const int32_t* counts_ws, int32_t* sorted_ids,
+    int32_t* expert_ids, int32_t* ntpp_out, int32_t* offsets_ws,
+    int32_t* user_offsets) {
   extern __shared__ int32_t smem_i32[];
   int32_t* offs = smem_i32;                    // [E + 1]
   int32_t* cnt = offs + (E + 1);               // [E]
   int32_t* running = cnt + E;                  // [kAlignWarps][E]
   __shared__ int32_t warp_sums[kAlignWarps];
+  pdl_launch_dependents();
+  pdl_wait();
   const int lane = threadIdx.x & 31, warp = threadIdx.x >> 5;
 
   // padded offsets: exclusive scan of round_up(count, block_m) over experts
@@ -261,7 +278,7 @@ __global__ void __launch_bounds__(kAlignWarps * 32) align_scatter_kernel(
       const int f = base + i0 + lane;
       int e = -1;
       if (f < n) {
-        e = __ldg(ids + f);
+        e = (*(ids + f));
         if (e < 0 || e >= E) e = -1;  // reported by pass 1; never indexed
       }
       const uint32_t same = __match_any_sync(0xffffffffu, e);
@@ -304,21 +321,162 @@ cudaError_t launch_align(const int32_t* topk_ids, int n, int E, int block_m, int
   const int threads = kAlignWarps * 32;
   const int blocks = (nchunks + kAlignWarps - 1) / kAlignWarps;
   const size_t smem1 = static_cast<size_t>(kAlignWarps) * E * sizeof(int32_t);
-  align_count_kernel<<<blocks, threads, smem1, stream>>>(topk_ids, n, E, nchunks, chunk_scratch, status);
-  cudaError_t err = cudaGetLastError();
+  cudaError_t err = launch_pdl(align_count_kernel, blocks, threads, smem1, stream, topk_ids, n, E, nchunks,
+                               chunk_scratch, status);
   if (err != cudaSuccess) return err;
-  align_scan_kernel<<<E, 256, 0, stream>>>(chunk_scratch, nchunks, E, counts_ws, user_counts);
-  err = cudaGetLastError();
+  err = launch_pdl(align_scan_kernel, E, 256, 0, stream, chunk_scratch, nchunks, E, counts_ws, user_counts);
   if (err != cudaSuccess) return err;
   const size_t smem3 = (static_cast<size_t>(E + 1) + E + static_cast<size_t>(kAlignWarps) * E) * sizeof(int32_t);
   int blocks3 = blocks;
   const int fill_blocks = (capacity + threads * 4 - 1) / (threads * 4);
   if (fill_blocks > blocks3) blocks3 = fill_blocks < 296 ? fill_blocks : 296;
   if (blocks3 < blocks) blocks3 = blocks;
-  align_scatter_kernel<<<blocks3, threads, smem3, stream>>>(topk_ids, n, E, block_m, capacity, nchunks,
-                                                            chunk_scratch, counts_ws, sorted_ids, expert_ids, ntpp,
-                                                            offsets_ws, user_offsets);
-  return cudaGetLastError();
+  return launch_pdl(align_scatter_kernel, blocks3, threads, smem3, stream, topk_ids, n, E, block_m, capacity,
+                    nchunks, chunk_scratch, counts_ws, sorted_ids, expert_ids, ntpp, offsets_ws, user_offsets);
+}
+
+// ----------------------------------------------------------------------------
+// Small batches: routing and the whole alignment in one CTA of 1024 threads.
+// The assignments are split into 32 contiguous warp-chunks; per-warp expert
+// histograms, a per-expert scan over the warps, a block scan of the padded
+// counts, then each warp scatters its chunk in order (ranks from
+// __match_any_sync plus a running per-warp base), which is the same stable
+// order as the multi-CTA path.
+// ----------------------------------------------------------------------------
+template <int VPL>
+__global__ void __launch_bounds__(1024) route_align_small_kernel(
+    const float* logits, const int32_t* ids_in, int T, int E, int topk, int renormalize,
+    int32_t* ids_out, float* weights_out, int block_m, int capacity,
+    int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp_out,
+    int32_t* counts_out, int32_t* offsets_out, int* status) {
+  extern __shared__ int32_t sm_small[];
+  __shared__ int32_t warp_sums[32];
+  pdl_launch_dependents();
+  pdl_wait();
+  const int n = T * topk;
+  const int tid = threadIdx.x, lane = tid & 31, warp = tid >> 5;
+  int32_t* ids_s = sm_small;           // [n]
+  int32_t* hist = ids_s + n;           // [32][E]: counts, then running bases
+  int32_t* offs = hist + 32 * E;       // [E + 1]
+  int32_t* cnt = offs + E + 1;         // [E]
+
+  if (logits != nullptr) {
+    for (int t = warp; t < T; t += 32) {
+      int id;
+      float w;
+      route_token<VPL>(logits + static_cast<size_t>(t) * E, E, topk, renormalize, lane, id, w);
+      if (lane < topk) {
+        ids_out[t * topk + lane] = id;
+        weights_out[t * topk + lane] = w;
+        ids_s[t * topk + lane] = id;
+      }
+    }
+  } else {
+    for (int i = tid; i < n; i += 1024) ids_s[i] = (*(ids_in + i));
+  }
+  for (int i = tid; i < 32 * E; i += 1024) hist[i] = 0;
+  __syncthreads();
+
+  const int chunk = (n + 32 * 32 - 1) / (32 * 32) * 32;  // multiple of 32
+  const int begin = warp * chunk;
+  const int end = min(begin + chunk, n);
+  for (int i = begin + lane; i < end; i += 32) {
+    const int e = ids_s[i];
+    if (e >= 0 && e < E)
+      atomicAdd(&hist[warp * E + e], 1);
+    else
+      report_status(status, MOE_STATUS_BAD_EXPERT_ID);
+  }
+  __syncthreads();
+  for (int e = tid; e < E; e += 1024) {
+    int32_t run = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int32_t v = hist[w * E + e];
+      hist[w * E + e] = run;
+      run += v;
+    }
+    cnt[e] = run;
+  }
+  __syncthreads();
+  {
+    const int32_t v = tid < E ? (cnt[tid] + block_m - 1) / block_m * block_m : 0;
+    int32_t incl = v;
+#pragma unroll
+    for (int off = 1; off < 32; off <<= 1) {
+      const int32_t o = __shfl_up_sync(0xffffffffu, incl, off);
+      if (lane >= off) incl += o;
+    }
+    if (lane == 31) warp_sums[warp] = incl;
+    __syncthreads();
+    int32_t before = 0, total = 0;
+    for (int w = 0; w < 32; ++w) {
+      const int32_t s = warp_sums[w];
+      if (w < warp) before += s;
+      total += s;
+    }
+    if (tid < E) offs[tid] = before + incl - v;
+    if (tid == 0) offs[E] = total;
+  }
+  __syncthreads();
+  const int ntpp = offs[E];
+
+  for (int i0 = begin; i0 < end; i0 += 32) {
+    const int i = i0 + lane;
+    int e = -1;
+    if (i < end) {
+      e = ids_s[i];
+      if (e < 0 || e >= E) e = -1;
+    }
+    const uint32_t same = __match_any_sync(0xffffffffu, e);
+    const uint32_t lower = same & ((1u << lane) - 1u);
+    int dest = -1;
+    if (e >= 0) dest = offs[e] + hist[warp * E + e] + __popc(lower);
+    __syncwarp();
+    if (e >= 0) {
+      sorted_ids[dest] = i;
+      if (lower == 0) hist[warp * E + e] += __popc(same);
+    }
+    __syncwarp();
+  }
+  for (int p = tid; p < capacity; p += 1024) {
+    bool pad = true;
+    if (p < ntpp) {
+      const int e = owner_expert(offs, E, p);
+      pad = p >= offs[e] + cnt[e];
+    }
+    if (pad) sorted_ids[p] = n;
+  }
+  for (int b = tid; b < capacity / block_m; b += 1024) {
+    const int p = b * block_m;
+    expert_ids[b] = (p < ntpp) ? owner_expert(offs, E, p) : -1;
+  }
+  for (int e = tid; e <= E; e += 1024) {
+    offsets_out[e] = offs[e];
+    if (e < E) counts_out[e] = cnt[e];
+  }
+  if (tid == 0) *ntpp_out = ntpp;
+}
+
+bool route_align_small_fits(long long n, int E) { return n > 0 && n <= kSmallAlignMaxN && E <= kSmallAlignMaxE; }
+
+cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in, int T, int E, int topk,
+                                     int renormalize, int32_t* ids_out, float* weights_out, int block_m, int capacity,
+                                     int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp, int32_t* counts,
+                                     int32_t* offsets, int* status, cudaStream_t stream) {
+  const size_t smem = (static_cast<size_t>(T) * topk + 32 * static_cast<size_t>(E) + 2 * static_cast<size_t>(E) + 1) *
+                      sizeof(int32_t);
+  static bool attr_set[4] = {false, false, false, false};
+  auto pick = [&](auto kern, int idx) -> cudaError_t {
+    if (!attr_set[idx]) {
+      cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize, 96 * 1024);
+      if (e != cudaSuccess) return e;
+      attr_set[idx] = true;
+    }
+    return launch_pdl(kern, 1, 1024, smem, stream, logits, ids_in, T, E, topk, renormalize, ids_out, weights_out,
+                      block_m, capacity, sorted_ids, expert_ids, ntpp, counts, offsets, status);
+  };
+  if (E <= 128) return pick(route_align_small_kernel<4>, 0);
+  return pick(route_align_small_kernel<8>, 1);
 }
 
 }  // namespace moe

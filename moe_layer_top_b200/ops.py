@@ -50,7 +50,8 @@ class MoeProblem(ctypes.Structure):
     _fields_ = [
         ("T", ctypes.c_int32), ("E", ctypes.c_int32), ("topk", ctypes.c_int32), ("H", ctypes.c_int32),
         ("I", ctypes.c_int32), ("weight_dtype", ctypes.c_int32), ("mode", ctypes.c_int32),
-        ("block_m", ctypes.c_int32), ("renormalize", ctypes.c_int32), ("reserved", ctypes.c_int32 * 7),
+        ("block_m", ctypes.c_int32), ("renormalize", ctypes.c_int32), ("split_k", ctypes.c_int32),
+        ("reserved", ctypes.c_int32 * 6),
     ]
 
 
@@ -61,7 +62,7 @@ class MoeWorkspaceLayout(ctypes.Structure):
         ("num_tokens_post_padded", ctypes.c_int64), ("expert_counts", ctypes.c_int64),
         ("expert_offsets", ctypes.c_int64), ("align_scratch", ctypes.c_int64), ("a1", ctypes.c_int64),
         ("a1_scale", ctypes.c_int64), ("a2", ctypes.c_int64), ("a2_scale", ctypes.c_int64), ("y", ctypes.c_int64),
-        ("total_bytes", ctypes.c_int64), ("capacity", ctypes.c_int32), ("block_m", ctypes.c_int32),
+        ("partials", ctypes.c_int64), ("tile_counters", ctypes.c_int64), ("total_bytes", ctypes.c_int64), ("capacity", ctypes.c_int32), ("block_m", ctypes.c_int32),
         ("mode", ctypes.c_int32), ("align_chunks", ctypes.c_int32),
     ]
 
@@ -127,11 +128,12 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def problem(T, E, topk, H, I, fp8=False, mode=MODE_AUTO, block_m=0, renormalize=True) -> MoeProblem:
+def problem(T, E, topk, H, I, fp8=False, mode=MODE_AUTO, block_m=0, renormalize=True, split_k=True) -> MoeProblem:
     p = MoeProblem()
     p.T, p.E, p.topk, p.H, p.I = int(T), int(E), int(topk), int(H), int(I)
     p.weight_dtype = DTYPE_FP8_E4M3 if fp8 else DTYPE_BF16
     p.mode, p.block_m, p.renormalize = int(mode), int(block_m), 1 if renormalize else 0
+    p.split_k = 0 if split_k else 1
     return p
 
 

@@ -55,7 +55,7 @@ class Case:
     """One workload instance on the GPU plus its oracle evaluation."""
 
     def __init__(self, cfg: inputs.MoEConfig, T: int, seed: int = 0, mode=ops.MODE_AUTO, block_m=0,
-                 weights=None):
+                 weights=None, split_k=True):
         self.cfg, self.T, self.seed = cfg, T, seed
         dev = torch.device("cuda")
         if weights is None:
@@ -69,7 +69,8 @@ class Case:
         else:
             self.w13, self.w2 = self.w13_bf16, self.w2_bf16
             self.w13_scale = self.w2_scale = None
-        self.p = ops.problem(T, cfg.E, cfg.topk, cfg.H, cfg.I, fp8=cfg.fp8, mode=mode, block_m=block_m)
+        self.p = ops.problem(T, cfg.E, cfg.topk, cfg.H, cfg.I, fp8=cfg.fp8, mode=mode, block_m=block_m,
+                             split_k=split_k)
         self.q = ops.resolve_problem(self.p)
         self.ws = ops.alloc_workspace(self.p)
         self.out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
