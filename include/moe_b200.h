@@ -73,7 +73,7 @@ extern "C" {
 
 /* tile orientation of the two grouped GEMMs */
 #define MOE_MODE_AUTO 0    /* chosen from the expected tokens per expert */
-#define MOE_MODE_NORMAL 1  /* MMA M = 128 token rows, N = 256 weight rows */
+#define MOE_MODE_NORMAL 1  /* MMA M = 128 token rows (block_m 128), or 256 over two SMs (FP8, block_m 256), N = 256 */
 #define MOE_MODE_SWAP_AB 2 /* MMA M = 128 weight rows, N = block_m token rows */
 
 /* stages of moe_forward_stages, in pipeline order */
@@ -100,7 +100,7 @@ typedef struct moe_problem {
   int32_t I;            /* expert intermediate size */
   int32_t weight_dtype; /* MOE_DTYPE_* */
   int32_t mode;         /* MOE_MODE_* */
-  int32_t block_m;      /* rows per expert block: 16, 32 or 64 (swap-AB), 128 (normal); 0 = auto */
+  int32_t block_m;      /* rows per expert block: 16, 32, 64 (swap-AB); 128, or 256 for FP8 two-SM tiles (normal); 0 = auto */
   int32_t renormalize;  /* router: 1 = renormalise the chosen softmax weights (default), 0 = keep them */
   int32_t split_k;      /* swap-AB GEMMs: 0 = split K when few tiles are in flight (default), 1 = never */
   int32_t reserved[6];  /* must be zero */

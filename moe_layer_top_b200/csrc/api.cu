@@ -79,13 +79,16 @@ int validate_problem(const moe_problem* p) {
   if (p->split_k != 0 && p->split_k != 1) return fail(MOE_ERR_INVALID, "split_k must be 0 or 1");
   for (int i = 0; i < 6; ++i)
     if (p->reserved[i] != 0) return fail(MOE_ERR_INVALID, "reserved fields must be zero");
-  if (p->mode == MOE_MODE_NORMAL && p->block_m != 0 && p->block_m != 128)
-    return fail(MOE_ERR_INVALID, "normal mode uses block_m = 128 (got %d)", p->block_m);
+  const bool fp8 = p->weight_dtype == MOE_DTYPE_FP8_E4M3;
+  if (p->block_m == 256 && !fp8)
+    return fail(MOE_ERR_INVALID, "block_m = 256 (two-SM tiles) needs FP8 weights");
+  if (p->mode == MOE_MODE_NORMAL && p->block_m != 0 && p->block_m != 128 && p->block_m != 256)
+    return fail(MOE_ERR_INVALID, "normal mode uses block_m = 128 or 256 (got %d)", p->block_m);
   if (p->mode == MOE_MODE_SWAP_AB && p->block_m != 0 && p->block_m != 16 && p->block_m != 32 && p->block_m != 64)
     return fail(MOE_ERR_INVALID, "swap-AB mode uses block_m in {16, 32, 64} (got %d)", p->block_m);
   if (p->mode == MOE_MODE_AUTO && p->block_m != 0 && p->block_m != 16 && p->block_m != 32 && p->block_m != 64 &&
-      p->block_m != 128)
-    return fail(MOE_ERR_INVALID, "block_m %d not in {16, 32, 64, 128}", p->block_m);
+      p->block_m != 128 && p->block_m != 256)
+    return fail(MOE_ERR_INVALID, "block_m %d not in {16, 32, 64, 128, 256}", p->block_m);
   return MOE_OK;
 }
 
@@ -97,7 +100,7 @@ void resolve(moe_problem* p) {
   const int64_t hit = n < p->E ? n : p->E;
   const double avg = hit > 0 ? static_cast<double>(n) / static_cast<double>(hit) : 1.0;
   if (p->mode == MOE_MODE_AUTO) {
-    if (p->block_m == 128)
+    if (p->block_m >= 128)
       p->mode = MOE_MODE_NORMAL;
     else if (p->block_m != 0)
       p->mode = MOE_MODE_SWAP_AB;
@@ -106,7 +109,7 @@ void resolve(moe_problem* p) {
   }
   if (p->block_m == 0) {
     if (p->mode == MOE_MODE_NORMAL)
-      p->block_m = 128;
+      p->block_m = 128;  // the two-SM FP8 tiles (block_m 256) are opt-in: slower so far
     else
       p->block_m = avg <= 8.0 ? 16 : (avg <= 20.0 ? 32 : 64);
   }

@@ -60,6 +60,10 @@ def test_resolve_problem_auto_modes(L):
     assert q.mode == ops.MODE_SWAP_AB and q.block_m == 16
     q = ops.resolve_problem(ops.problem(16384, 128, 8, 4096, 1536, fp8=True))
     assert q.mode == ops.MODE_NORMAL and q.block_m == 128
+    q = ops.resolve_problem(ops.problem(16384, 128, 8, 4096, 1536, fp8=True, block_m=256))
+    assert q.mode == ops.MODE_NORMAL and q.block_m == 256
+    q = ops.resolve_problem(ops.problem(16384, 128, 8, 4096, 1536, fp8=False))
+    assert q.mode == ops.MODE_NORMAL and q.block_m == 128
     q = ops.resolve_problem(ops.problem(64, 128, 8, 4096, 1536, mode=ops.MODE_NORMAL))
     assert q.block_m == 128
     q = ops.resolve_problem(ops.problem(64, 128, 8, 4096, 1536, block_m=32))
@@ -69,7 +73,7 @@ def test_resolve_problem_auto_modes(L):
 @pytest.mark.parametrize("bad", [
     dict(T=-1), dict(E=0), dict(E=2000), dict(topk=0), dict(topk=9, E=8), dict(H=100), dict(I=0), dict(I=200),
     dict(mode=7), dict(mode=ops.MODE_NORMAL, block_m=16), dict(mode=ops.MODE_SWAP_AB, block_m=128),
-    dict(block_m=48),
+    dict(block_m=48), dict(mode=ops.MODE_NORMAL, block_m=256),
 ])
 def test_invalid_problems_are_rejected(L, bad):
     kw = dict(T=16, E=8, topk=2, H=256, I=128)

@@ -186,6 +186,15 @@ def test_tiny_layer_all_modes(mode, bm):
     assert_close(out.float().cpu().numpy(), ref["out"], fp8=False)
 
 
+@pytest.mark.parametrize("T", [1, 37, 700, 3000])
+def test_mid_layer_fp8_two_sm_tiles(T):
+    """FP8 normal orientation with 256-row blocks: two SMs per tile (cta_group::2)."""
+    c = Case(MID_FP8, T, seed=T + 1, mode=ops.MODE_NORMAL, block_m=256)
+    out = c.run()
+    assert c.status() == ops.MOE_STATUS_OK
+    assert_close(out.float().cpu().numpy(), c.oracle()["out"], fp8=True)
+
+
 @pytest.mark.parametrize("cfg", [MID_BF16, MID_FP8], ids=["bf16", "fp8"])
 @pytest.mark.parametrize("T", [1, 37, 700])
 @pytest.mark.parametrize("mode,bm", MODES)
