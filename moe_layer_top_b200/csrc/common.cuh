@@ -404,9 +404,13 @@ __device__ __forceinline__ uint16_t f32x2_to_e4m3x2(float lo, float hi) {
   return static_cast<uint16_t>(__nv_cvt_float2_to_fp8x2(make_float2(lo, hi), __NV_SATFINITE, __NV_E4M3));
 }
 
-// y = silu(g) rounded to bf16, times u, rounded to bf16 (g, u already bf16 values)
+// y = silu(g) rounded to bf16, times u, rounded to bf16 (g, u already bf16 values).
+// The fast exponential and division (a few ulp of fp32) are far below the
+// bf16 rounding that follows; this runs 64 times per row in the GEMM1
+// epilogue, where it is not hidden behind the MMA.  For g < -88, exp(-g) is
+// +inf and the quotient is -0.
 __device__ __forceinline__ float silu_mul_bf16(float g, float u) {
-  const float s = bf16_round(__fdiv_rn(g, 1.0f + expf(-g)));
+  const float s = bf16_round(__fdividef(g, 1.0f + __expf(-g)));
   return bf16_round(s * u);
 }
 
