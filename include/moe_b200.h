@@ -259,6 +259,17 @@ MOE_API int moe_forward_stages(const moe_problem* p, const void* x, const float*
  */
 MOE_API int moe_read_status(const moe_problem* p, void* ws, int32_t clear, int32_t* status, void* stream);
 
+/*
+ * Failure-detection self-test (no counterpart on the pages).  Launches one
+ * kernel whose only wait -- on an mbarrier nothing arrives at -- goes through
+ * the same bounded wait the pipeline kernels use, limited to timeout_us
+ * (1 .. 1 000 000).  It must give up: *status (device int32, cleared first)
+ * receives MOE_STATUS_WAIT_TIMEOUT | 0x7F and *waited_ns (device uint64) the
+ * time it waited; the kernel then returns normally and the context stays
+ * usable.  Nothing faults, traps or hangs.
+ */
+MOE_API int moe_selftest_wait_timeout(uint32_t timeout_us, int32_t* status, uint64_t* waited_ns, void* stream);
+
 /* Library version: major * 10000 + minor * 100 + patch. */
 MOE_API int32_t moe_version(void);
 

@@ -330,6 +330,21 @@ const char* moe_last_error_string(void) { return g_last_error.c_str(); }
 
 int32_t moe_version(void) { return 100; }
 
+int moe_selftest_wait_timeout(uint32_t timeout_us, int32_t* status, uint64_t* waited_ns, void* stream) {
+  if (timeout_us < 1 || timeout_us > 1000000)
+    return fail(MOE_ERR_INVALID, "selftest: timeout_us %u outside [1, 1000000]", timeout_us);
+  if (!status || !waited_ns) return fail(MOE_ERR_INVALID, "selftest: NULL pointer");
+  if (!aligned(status, 4) || !aligned(waited_ns, 8)) return fail(MOE_ERR_INVALID, "selftest: misaligned pointer");
+  int rc = device_check(nullptr);
+  if (rc != MOE_OK) return rc;
+  cudaStream_t s = static_cast<cudaStream_t>(stream);
+  cudaError_t e = cudaMemsetAsync(status, 0, sizeof(int32_t), s);
+  if (e == cudaSuccess)
+    e = moe::launch_wait_selftest(reinterpret_cast<int*>(status), 1000ull * timeout_us,
+                                  reinterpret_cast<unsigned long long*>(waited_ns), s);
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "selftest");
+}
+
 int moe_route(const float* logits, int32_t T, int32_t E, int32_t topk, int32_t renormalize, int32_t* topk_ids,
               float* topk_weights, void* stream) {
   if (T < 0 || E < 1 || E > 1024 || topk < 1 || topk > E || topk > 32)

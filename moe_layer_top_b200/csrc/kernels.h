@@ -89,6 +89,10 @@ cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const float* a1_s
 cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const float* a2_scale_t, const void* w2,
                          const float* w2_scale, void* y, cudaStream_t stream);
 
+// failure-detection self-test: one bounded wait that must time out
+cudaError_t launch_wait_selftest(int* status, unsigned long long timeout_ns, unsigned long long* waited_ns,
+                                 cudaStream_t stream);
+
 // set the per-thread error message returned by moe_last_error_string(); returns code
 int record_error(int code, const char* msg);
 

@@ -43,6 +43,7 @@ EXPORTED = (
     "moe_last_error_string", "moe_route", "moe_align_capacity", "moe_align_workspace_size", "moe_align",
     "moe_quantize_weights_fp8", "moe_resolve_problem", "moe_workspace_size", "moe_get_workspace_layout",
     "moe_fused_forward", "moe_forward_stages", "moe_read_status", "moe_version", "moe_align_noalloc",
+    "moe_selftest_wait_timeout",
 )
 
 
@@ -99,6 +100,7 @@ def lib():
             "moe_fused_forward": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, vp]),
             "moe_forward_stages": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i32, i32, vp]),
             "moe_read_status": (ctypes.c_int, [P, vp, i32, ctypes.POINTER(i32), vp]),
+            "moe_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, vp, vp, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -264,3 +266,12 @@ def workspace_views(p: MoeProblem, ws: torch.Tensor) -> dict:
         "layout": L,
         "problem": q,
     }
+
+
+def selftest_wait_timeout(timeout_us: int, stream=None):
+    """Run the bounded-wait self-test; returns (status, waited_ns) after a sync."""
+    st = torch.zeros((1,), dtype=torch.int32, device="cuda")
+    waited = torch.zeros((1,), dtype=torch.int64, device="cuda")
+    _check(lib().moe_selftest_wait_timeout(int(timeout_us), _ptr(st), _ptr(waited), _stream(stream)))
+    torch.cuda.synchronize()
+    return int(st.item()), int(waited.item())

@@ -143,3 +143,10 @@ def test_product_path_has_no_fallback(tmp_path, monkeypatch):
     monkeypatch.setattr(ops, "_lib", None)
     with pytest.raises(RuntimeError):
         ops.lib()
+
+
+def test_selftest_argument_errors(L):
+    g = _fake(1 << 20)
+    assert L.moe_selftest_wait_timeout(0, g, g, None) == ops.MOE_ERR_INVALID
+    assert L.moe_selftest_wait_timeout(2_000_000, g, g, None) == ops.MOE_ERR_INVALID
+    assert L.moe_selftest_wait_timeout(100, None, g, None) == ops.MOE_ERR_INVALID
