@@ -250,10 +250,30 @@ class Workload:
 def kernels_per_forward(cfg, T, has_logits):
     """Kernels of this library one moe_fused_forward launches: a single-CTA
     route+align for T*topk <= 8192 and E <= 256, else route + 3 align passes;
-    then gather, GEMM1, GEMM2, combine."""
+    then gather, GEMM1, GEMM2, combine (not counting a split-K reduce, which
+    only small swap-AB problems launch).  Used only when the captured graph
+    cannot be inspected."""
     small = T * cfg.topk <= 8192 and cfg.E <= 256
     head = 1 if small else (1 if has_logits else 0) + 3
     return head + 4
+
+
+def graph_kernel_count(g):
+    """Kernel nodes of a captured CUDA graph (None if it cannot be read).  The
+    forward graph captures nothing but this library's launches."""
+    try:
+        import cuda.bindings.runtime as rt
+        graph = rt.cudaGraph_t(init_value=g.raw_cuda_graph())
+        err, _, n = rt.cudaGraphGetNodes(graph, 0)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        err, nodes, n = rt.cudaGraphGetNodes(graph, n)
+        if err != rt.cudaError_t.cudaSuccess:
+            return None
+        kernel = rt.cudaGraphNodeType.cudaGraphNodeTypeKernel
+        return sum(1 for nd in nodes[:n] if rt.cudaGraphNodeGetType(nd)[1] == kernel)
+    except Exception:
+        return None
 
 
 def make_weights(cfg, seed):
@@ -311,15 +331,20 @@ class StageEvents:
         return [self.ev[i].elapsed_time(self.ev[i + 1]) for i in range(len(self.ev) - 1)]
 
 
-def capture(fn):
-    """Capture fn() into a CUDA graph (after it has run once eagerly)."""
+def capture(fn, count_kernels=False):
+    """Capture fn() into a CUDA graph (after it has run once eagerly); with
+    count_kernels, also return the number of kernel nodes in it."""
     fn()
     torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph()
+    g = torch.cuda.CUDAGraph(keep_graph=count_kernels)
     with torch.cuda.graph(g):
         fn()
     torch.cuda.synchronize()
-    return g
+    if not count_kernels:
+        return g
+    n = graph_kernel_count(g)
+    g.instantiate()
+    return g, n
 
 
 def time_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor, world: int):
@@ -328,7 +353,7 @@ def time_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor, world
     B) a CUDA graph of the same stages with event nodes between them -> per-stage times."""
     ops = wl.ops
     stream = torch.cuda.current_stream()
-    g_fwd = capture(wl.forward)
+    g_fwd, n_kernels = capture(wl.forward, count_kernels=True)
     se = StageEvents(ops.NUM_STAGES + 1)
 
     def staged():
@@ -363,7 +388,7 @@ def time_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor, world
         g_stg.replay()
         torch.cuda.synchronize()
         per_stage.append(se.elapsed())
-    return step_ms, np.array(per_stage), wall
+    return step_ms, np.array(per_stage), wall, n_kernels
 
 
 def e2e_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor):
@@ -477,9 +502,10 @@ def run_ours(args, rank, world, local):
         for T in sweep_T:
             wl = Workload(cfg, T, args.seed, weights)
             steps = args.steps if T == T_head else max(3, args.steps // 2)
-            step_ms, per_stage, wall = time_steps(wl, steps, args.warmup, flush, world)
+            step_ms, per_stage, wall, n_kernels = time_steps(wl, steps, args.warmup, flush, world)
             total_ms = max_over_ranks(float(step_ms.sum()), world)
-            results[T] = {"wl": wl, "per_stage": per_stage, "total_ms": total_ms, "steps": steps, "wall_s": wall}
+            results[T] = {"wl": wl, "per_stage": per_stage, "total_ms": total_ms, "steps": steps, "wall_s": wall,
+                          "kernels": n_kernels}
     clk = clocks.summary()
     head = results[T_head]
     wl = head["wl"]
@@ -494,11 +520,23 @@ def run_ours(args, rank, world, local):
     dom_bytes = {"gemm1": alg["gemm1_bytes"], "gemm2": alg["gemm2_bytes"]}.get(dom_name)
     if dom_bytes is None:
         dom_bytes = alg["layer_bytes"]
-    achieved = dom_bytes / (stage_ms[dom] / 1e3) / 1e9
     traffic = traffic_record(dom_name, args.workload, T_head)
-    roofline = {"bound": "hbm", "kernel": dom_name, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
-                "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
-                "peak_source": peaks["source"], "algorithmic_bytes": dom_bytes}
+    # FLOPs of the dominant GEMM (GEMM1 = 2/3 of the layer, GEMM2 = 1/3)
+    dom_flops = alg["flops"] * {"gemm1": 2.0 / 3.0, "gemm2": 1.0 / 3.0}.get(dom_name, 1.0)
+    # tensor-core peak for the arithmetic dtype: measured bf16 (burst: the kernel
+    # is timed on its own inside a short step); FP8 = 2x that, the nominal ratio
+    tc_peak = peaks["bf16_tflops"] * (2.0 if cfg.fp8 else 1.0)
+    tc_source = f"{peaks['source']} bf16 burst" + (" x 2 (nominal FP8/bf16 ratio)" if cfg.fp8 else "")
+    if dom_flops / (tc_peak * 1e12) > dom_bytes / (peaks["hbm_gbs"] * 1e9):
+        achieved = dom_flops / (stage_ms[dom] / 1e3) / 1e12
+        roofline = {"bound": "tensor", "kernel": dom_name, "achieved": round(achieved, 1), "peak": round(tc_peak, 1),
+                    "unit": "TFLOP/s", "frac": round(achieved / tc_peak, 4), "traffic": traffic,
+                    "peak_source": tc_source, "algorithmic_flops": dom_flops, "algorithmic_bytes": dom_bytes}
+    else:
+        achieved = dom_bytes / (stage_ms[dom] / 1e3) / 1e9
+        roofline = {"bound": "hbm", "kernel": dom_name, "achieved": round(achieved, 1), "peak": peaks["hbm_gbs"],
+                    "unit": "GB/s", "frac": round(achieved / peaks["hbm_gbs"], 4), "traffic": traffic,
+                    "peak_source": peaks["source"], "algorithmic_bytes": dom_bytes}
     sweep = []
     for T in sweep_T:
         r = results[T]
@@ -507,9 +545,13 @@ def run_ours(args, rank, world, local):
         sm = r["per_stage"].mean(axis=0)
         sweep.append({"T": T, "tokens_per_s": round(world * T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
                       "layer_hbm_frac": round(a["layer_bytes"] / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
-                      "tflops": round(a["flops"] / (ms / 1e3) / 1e12, 2), "hit_experts": a["hit_experts"],
+                      "tflops": round(a["flops"] / (ms / 1e3) / 1e12, 2),
+                      "layer_tc_frac": round(a["flops"] / (ms / 1e3) / 1e12 /
+                                             (peaks["bf16_tflops"] * (2.0 if cfg.fp8 else 1.0)), 4),
+                      "hit_experts": a["hit_experts"],
                       "stage_us": {ops.STAGE_NAMES[s]: round(float(sm[s]) * 1e3, 1) for s in range(ops.NUM_STAGES)},
                       "mode": "swap_ab" if r["wl"].q.mode == ops.MODE_SWAP_AB else "normal",
+                      "kernels_per_step": r["kernels"],
                       "block_m": r["wl"].q.block_m})
     e2e_ms, h2d, d2h = e2e_steps(wl, K, args.warmup, flush)
     e2e_ms = max_over_ranks(e2e_ms, world)
@@ -531,7 +573,8 @@ def run_ours(args, rank, world, local):
         "stage_us": {ops.STAGE_NAMES[s]: round(float(stage_ms[s]) * 1e3, 1) for s in range(ops.NUM_STAGES)},
         "sweep": sweep,
         "e2e": e2e,
-        "gpu_launches": K * kernels_per_forward(cfg, T_head, "logits" in wl.routing),
+        "gpu_launches": K * (head["kernels"] or kernels_per_forward(cfg, T_head, "logits" in wl.routing)),
+        "gpu_launches_source": "kernel nodes of the captured forward graph" if head["kernels"] else "formula",
         "clocks": clk,
     }
     if rank == 0 and world == 1 and not args.no_cpu_baseline:

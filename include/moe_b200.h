@@ -127,7 +127,6 @@ typedef struct moe_workspace_layout {
   int64_t a2_scale;         /* fp32 [I/128, capacity] (FP8 only; K-block major) */
   int64_t y;                /* bf16 [T*topk, H] weighted expert outputs */
   int64_t partials;         /* fp32 split-K partial sums of the swap-AB GEMMs (swap-AB only) */
-  int64_t tile_counters;    /* int32 per-tile split-K arrival counters (swap-AB only) */
   int64_t total_bytes;
   int32_t capacity;         /* rows of sorted_token_ids */
   int32_t block_m;

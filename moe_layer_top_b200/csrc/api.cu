@@ -166,11 +166,8 @@ int make_plan(const moe_problem* in, Plan* plan) {
     // one buffer serves both GEMMs (they run one after the other); GEMM1's
     // units hold 2*block_m accumulator columns, GEMM2's block_m
     L.partials = take(static_cast<int64_t>(moe::kMaxSplitUnits) * 128 * 2 * p.block_m * 4);
-    const int64_t blocks = cap / p.block_m;
-    L.tile_counters = take((blocks * (p.I / 128) + blocks * (p.H / 128)) * 4);
   } else {
     L.partials = -1;
-    L.tile_counters = -1;
   }
   L.total_bytes = off;
   L.capacity = static_cast<int32_t>(cap);
@@ -223,7 +220,6 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
   const int cap = L.capacity;
   const bool small = moe::route_align_small_fits(plan.nflat, p.E);
   const bool swap = p.mode == MOE_MODE_SWAP_AB;
-  const int n_counters = swap ? (cap / p.block_m) * (p.I / 128 + p.H / 128) : 0;
   bool aligned_already = false;
   cudaError_t e;
 
@@ -268,8 +264,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
       case MOE_STAGE_GATHER:
         e = moe::launch_gather(x, p.H, p.topk, nflat, at<int32_t>(ws, L.sorted_token_ids),
                                at<int32_t>(ws, L.num_tokens_post_padded), cap, plan.fp8, at<void>(ws, L.a1),
-                               plan.fp8 ? at<float>(ws, L.a1_scale) : nullptr,
-                               swap ? at<int>(ws, L.tile_counters) : nullptr, swap ? n_counters : 0, stream);
+                               plan.fp8 ? at<float>(ws, L.a1_scale) : nullptr, stream);
         if (e != cudaSuccess) return cuda_fail(e, "gather");
         break;
       case MOE_STAGE_GEMM1:
@@ -283,7 +278,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
         gp.block_m = p.block_m;
         gp.capacity = cap;
         gp.fp8 = plan.fp8;
-        gp.swap = p.mode == MOE_MODE_SWAP_AB;
+        gp.swap = swap;
         gp.ntpp = at<int32_t>(ws, L.num_tokens_post_padded);
         gp.expert_ids = at<int32_t>(ws, L.expert_ids);
         gp.sorted_ids = at<int32_t>(ws, L.sorted_token_ids);
@@ -291,10 +286,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
         gp.status = status;
         gp.num_sms = sms;
         gp.split_mode = p.split_k;
-        gp.partials1 = swap ? at<float>(ws, L.partials) : nullptr;
-        gp.partials2 = gp.partials1;
-        gp.counters1 = swap ? at<int>(ws, L.tile_counters) : nullptr;
-        gp.counters2 = swap ? at<int>(ws, L.tile_counters) + (cap / p.block_m) * (p.I / 128) : nullptr;
+        gp.partials = swap ? at<float>(ws, L.partials) : nullptr;
         if (s == MOE_STAGE_GEMM1) {
           e = moe::launch_gemm1(gp, at<void>(ws, L.a1), plan.fp8 ? at<float>(ws, L.a1_scale) : nullptr, w13,
                                 w13_scale, at<void>(ws, L.a2), plan.fp8 ? at<float>(ws, L.a2_scale) : nullptr,

@@ -44,10 +44,9 @@ template <bool FP8>
 __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* x, int H, int topk,
                                                      int nflat, const int32_t* sorted_ids,
                                                      const int32_t* ntpp_ptr, int capacity,
-                                                     void* a1, float* a1_scale_t, int* zero, int zero_n) {
+                                                     void* a1, float* a1_scale_t) {
   pdl_launch_dependents();
   pdl_wait();
-  for (int i = blockIdx.x * blockDim.x + threadIdx.x; i < zero_n; i += gridDim.x * blockDim.x) zero[i] = 0;
   const int ntpp = *ntpp_ptr;
   const int vecs = H / 8;
   const int iters = (vecs + blockDim.x - 1) / blockDim.x;
@@ -89,16 +88,16 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* x, int
 }
 
 cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32_t* sorted_ids,
-                          const int32_t* ntpp, int capacity, bool fp8, void* a1, float* a1_scale_t, int* zero,
-                          int zero_n, cudaStream_t stream) {
+                          const int32_t* ntpp, int capacity, bool fp8, void* a1, float* a1_scale_t,
+                          cudaStream_t stream) {
   if (capacity == 0) return cudaSuccess;
   int blocks = capacity < 148 * 8 ? capacity : 148 * 8;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (fp8)
     return launch_pdl(gather_kernel<true>, blocks, 256, 0, stream, xb, H, topk, nflat, sorted_ids, ntpp, capacity, a1,
-                      a1_scale_t, zero, zero_n);
+                      a1_scale_t);
   return launch_pdl(gather_kernel<false>, blocks, 256, 0, stream, xb, H, topk, nflat, sorted_ids, ntpp, capacity, a1,
-                    a1_scale_t, zero, zero_n);
+                    a1_scale_t);
 }
 
 // ----------------------------------------------------------------------------

@@ -40,7 +40,7 @@ constexpr int kThreads = 320;
 constexpr int kEpiWarps = 8;
 constexpr int kSmemLimit = 232448;  // max dynamic shared memory per block on sm_100
 constexpr int kSmemReserve = 4096;  // barriers, TMEM slot, exchange buffers
-constexpr int kXchgOffset = 512;    // exchange buffers (2 x 256 floats) and the split-K ticket start here
+constexpr int kXchgOffset = 512;    // exchange buffers (2 x 256 floats) start here
 
 // wait-site codes reported in the status word (low byte)
 constexpr int kWhereProducer = 1, kWhereMma = 2, kWhereEpiAcc = 3, kWhereEpiXchg = 4, kWhereDrain = 5;
@@ -85,28 +85,26 @@ struct Args {
   float* out_scale_t;      // GEMM1 FP8: a2 scale [I/128, capacity]
   int* status;
   float* partials;         // swap-AB split-K: [unit][acc column][128] fp32 partial sums
-  int* tile_counters;      // swap-AB split-K: arrivals per tile (zero between launches)
-  int split_mode;          // 0: chosen from the tile count, 1: no split
+  int splits;              // swap-AB split-K factor S (1: no split); chosen on the host
 };
 
-// Split-K for the swap-AB tiles: when so few tiles are in flight that most
-// SMs would idle, the K range of every tile is cut in S pieces.  The splits
-// publish fp32 partial sums and the last one to arrive adds them in split
-// order (fence, barrier, atomic ticket, barrier, fence, reload): under full
-// HBM load that hand-off costs several microseconds per tile, more than the
-// balance it buys once at least half of the SMs have a tile, so it is used
-// only below that.  S is a pure function of (tiles, CTAs, K stages), so every
-// role and CTA agree on it and the result is deterministic.  A split needs
-// >= 4 stages and the launch at most kMaxSplitUnits units (the buffer).
+// Split-K for the swap-AB tiles: when at most half the SMs would have a tile
+// (few experts hit and small H or I), the K range of every tile is cut in S
+// pieces so that more SMs stream weights.  Each split stores fp32 partial
+// sums; a reduce kernel adds them in split order (deterministic) and runs the
+// epilogue.  S is chosen on the host from the tile count bound that the
+// capacity gives (capacity / block_m blocks), so the host knows whether the
+// reduce kernel is needed.  A split needs >= 4 K stages, and a launch at most
+// kMaxSplitUnits units (the partial-sum buffer).
 constexpr int kMaxSplits = 4;
 
-__device__ __forceinline__ int choose_splits(int tiles, int ctas, int k_stages, int mode) {
-  if (mode == 1 || tiles <= 0 || 2 * tiles > ctas) return 1;
+int choose_splits(long long tiles, int ctas, int k_stages) {
+  if (tiles <= 0 || 2 * tiles > ctas) return 1;
   int best = 1;
   long long best_u = tiles, best_w = (tiles + ctas - 1) / ctas;  // efficiency = u / (ctas * w)
   for (int sp = 2; sp <= kMaxSplits; ++sp) {
-    if (k_stages / sp < 4 || static_cast<long long>(tiles) * sp > kMaxSplitUnits) break;
-    const long long u = static_cast<long long>(tiles) * sp, w = (u + ctas - 1) / ctas;
+    if (k_stages / sp < 4 || tiles * sp > kMaxSplitUnits) break;
+    const long long u = tiles * sp, w = (u + ctas - 1) / ctas;
     if (u * best_w * 100 > best_u * w * 105) {  // at least 5 % better
       best = sp;
       best_u = u;
@@ -186,7 +184,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   const int num_mblocks = (*(args.ntpp)) / rows_per_block;
   const int num_tiles = num_mblocks * n_tiles;
   const int k_stages = K / C::kKElems;
-  const int splits = kSwap ? choose_splits(num_tiles, gridDim.x, k_stages, args.split_mode) : 1;
+  const int splits = kSwap ? args.splits : 1;
   const int num_units = num_tiles * splits;
 
   if (warp == 0) {
@@ -622,8 +620,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
 
         if (splits > 1) {
-          // ---- split-K: publish this split's partial sums; the last split of
-          // the tile to arrive adds all of them in split order and goes on.
+          // ---- split-K: store this split's fp32 partial sums; the reduce
+          // kernel that follows adds the splits in order and runs the epilogue
           constexpr int kAccW = kDown ? kBM : 2 * kBM;
           float* part = args.partials + static_cast<size_t>(unit) * (kAccW * 128);
 #pragma unroll
@@ -631,41 +629,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             part[(col_a + j) * 128 + row] = acc_a[j];
             if constexpr (!kDown) part[(col_b + j) * 128 + row] = acc_b[j];
           }
-          __threadfence();
-          mbar_arrive(&xchg_bar[xbuf]);
-          if (!warp_wait(&xchg_bar[xbuf], xphase, abort_flag, args.status, kWhereEpiXchg)) {
-            ok = false;
-            break;
-          }
-          // the ticket gets a slot of its own: the exchange buffers are reused by the
-          // FP8 amax exchange right after, possibly before every warp has read it
-          volatile int* ticket_slot = reinterpret_cast<volatile int*>(xchg + 512);
-          if (warp == 2 && lane == 0) *ticket_slot = atomicAdd(args.tile_counters + tile, 1);
-          xbuf ^= 1;
-          if (xbuf == 0) xphase ^= 1u;
-          mbar_arrive(&xchg_bar[xbuf]);
-          if (!warp_wait(&xchg_bar[xbuf], xphase, abort_flag, args.status, kWhereEpiXchg)) {
-            ok = false;
-            break;
-          }
-          const int ticket = *ticket_slot;
-          xbuf ^= 1;
-          if (xbuf == 0) xphase ^= 1u;
-          if (ticket != splits - 1) continue;
-          __threadfence();
-          if (warp == 2 && lane == 0) args.tile_counters[tile] = 0;  // ready for the next launch
-          const float* tile_part = args.partials + static_cast<size_t>(tile) * splits * (kAccW * 128);
-#pragma unroll
-          for (int j = 0; j < kHT; ++j) {
-            float sa = 0.f, sb = 0.f;
-            for (int sp = 0; sp < splits; ++sp) {
-              const float* ps = tile_part + static_cast<size_t>(sp) * (kAccW * 128);
-              sa += (sp == split) ? acc_a[j] : __ldcg(ps + (col_a + j) * 128 + row);
-              if constexpr (!kDown) sb += (sp == split) ? acc_b[j] : __ldcg(ps + (col_b + j) * 128 + row);
-            }
-            acc_a[j] = sa;
-            if constexpr (!kDown) acc_b[j] = sb;
-          }
+          continue;
         }
 
         if constexpr (!kDown) {
@@ -731,6 +695,86 @@ __global__ void __launch_bounds__(kThreads, 1)
   if (warp == 1) {
     tc_fence_after();
     tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------------------
+// Split-K reduce for the swap-AB GEMMs.  One CTA of 128 threads per tile;
+// thread `row` owns weight row nt*128 + row of the tile for all kBM tokens.
+// It adds the S partial sums in split order (deterministic) and runs the
+// epilogue the unsplit GEMM would have run: SiLU(gate)*up with bf16 rounding
+// (+ per-(token,128) FP8 requantisation, amax over the 128 rows through
+// shared memory) for GEMM1, routed weight and scatter to y for GEMM2.
+// ----------------------------------------------------------------------------
+template <bool kDown, bool kFP8, int kBM>
+__global__ void __launch_bounds__(128) splitk_reduce_kernel(Args args) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int n_tiles = (kDown ? args.H : args.I) / 128;
+  const int num_tiles = (*(args.ntpp)) / kBM * n_tiles;
+  const int splits = args.splits;
+  constexpr int kAccW = kDown ? kBM : 2 * kBM;
+  constexpr size_t kUnit = static_cast<size_t>(kAccW) * 128;
+  __shared__ float red[4][kBM];
+  const int row = threadIdx.x, warp = row >> 5, lane = row & 31;
+  for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+    const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
+    const int tok0 = mb * kBM;
+    const float* part = args.partials + static_cast<size_t>(tile) * splits * kUnit + row;
+    float a[kBM], b[kDown ? 1 : kBM];
+#pragma unroll
+    for (int j = 0; j < kBM; ++j) {
+      a[j] = __ldcg(part + j * 128);
+      if constexpr (!kDown) b[j] = __ldcg(part + (kBM + j) * 128);
+    }
+    for (int sp = 1; sp < splits; ++sp) {
+      const float* ps = part + sp * kUnit;
+#pragma unroll
+      for (int j = 0; j < kBM; ++j) {
+        a[j] += __ldcg(ps + j * 128);
+        if constexpr (!kDown) b[j] += __ldcg(ps + (kBM + j) * 128);
+      }
+    }
+    if constexpr (!kDown) {
+      const int icol = nt * 128 + row;
+#pragma unroll
+      for (int j = 0; j < kBM; ++j) a[j] = silu_mul_bf16(bf16_round(a[j]), bf16_round(b[j]));
+      if constexpr (!kFP8) {
+        __nv_bfloat16* a2 = static_cast<__nv_bfloat16*>(args.out);
+#pragma unroll
+        for (int j = 0; j < kBM; ++j) a2[static_cast<size_t>(tok0 + j) * args.I + icol] = __float2bfloat16_rn(a[j]);
+      } else {
+#pragma unroll
+        for (int j = 0; j < kBM; ++j) {
+          float m = fabsf(a[j]);
+#pragma unroll
+          for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+          if (lane == 0) red[warp][j] = m;
+        }
+        __syncthreads();
+        uint8_t* a2 = static_cast<uint8_t*>(args.out);
+#pragma unroll
+        for (int j = 0; j < kBM; ++j) {
+          const float m = fmaxf(fmaxf(red[0][j], red[1][j]), fmaxf(red[2][j], red[3][j]));
+          const float scale = act_scale_from_amax(m);
+          a2[static_cast<size_t>(tok0 + j) * args.I + icol] =
+              static_cast<uint8_t>(f32x2_to_e4m3x2(a[j] * pow2_recip(scale), 0.f) & 0xFFu);
+          if (row == 0) args.out_scale_t[static_cast<size_t>(nt) * args.capacity + tok0 + j] = scale;
+        }
+        __syncthreads();  // red is reused by the next tile
+      }
+    } else {
+      __nv_bfloat16* y = static_cast<__nv_bfloat16*>(args.out);
+      const int hcol = nt * 128 + row;
+#pragma unroll
+      for (int j = 0; j < kBM; ++j) {
+        const int flat = (*(args.sorted_ids + tok0 + j));
+        if (flat < args.nflat) {
+          const float wt = (*(args.topk_weights + flat));
+          y[static_cast<size_t>(flat) * args.H + hcol] = __float2bfloat16_rn(a[j] * wt);
+        }
+      }
+    }
   }
 }
 
@@ -1108,11 +1152,22 @@ cudaError_t launch_on(const GemmProblem& p, const void* tok, const void* w, cons
   if (!make_map(&tm_tok, tok, p.capacity, K, elem, C::kTokRows)) return cudaErrorInvalidValue;
   if (!make_map(&tm_w, w, wrows, K, elem, kDown ? C::kWRows : 128)) return cudaErrorInvalidValue;
   const int n_tiles = (kDown ? p.H : p.I) / C::kTileN;
-  const long long max_units = static_cast<long long>(p.capacity / C::kTokRows) * n_tiles * (kSwap ? kMaxSplits : 1);
+  const long long max_tiles = static_cast<long long>(p.capacity / C::kTokRows) * n_tiles;
   int grid = p.num_sms;
-  if (max_units < grid) grid = static_cast<int>(max_units);
+  if (kSwap && p.split_mode == 0) {
+    Args a = args;
+    a.splits = choose_splits(max_tiles, p.num_sms, static_cast<int>(K / C::kKElems));
+    if (max_tiles * a.splits < grid) grid = static_cast<int>(max_tiles * a.splits);
+    if (grid <= 0) return cudaSuccess;
+    cudaError_t e = launch_pdl(kern, grid, kThreads, C::kSmemBytes, s, tm_tok, tm_w, a);
+    if (e != cudaSuccess || a.splits == 1) return e;
+    return launch_pdl(splitk_reduce_kernel<kDown, kFP8, kBM>, static_cast<int>(max_tiles), 128, 0, s, a);
+  }
+  if (max_tiles < grid) grid = static_cast<int>(max_tiles);
   if (grid <= 0) return cudaSuccess;
-  return launch_pdl(kern, grid, kThreads, C::kSmemBytes, s, tm_tok, tm_w, args);
+  Args a = args;
+  a.splits = 1;
+  return launch_pdl(kern, grid, kThreads, C::kSmemBytes, s, tm_tok, tm_w, a);
 }
 
 template <bool kDown>
@@ -1193,9 +1248,8 @@ cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const float* a1_s
   args.out = a2;
   args.out_scale_t = a2_scale_t;
   args.status = p.status;
-  args.partials = p.partials1;
-  args.tile_counters = p.counters1;
-  args.split_mode = p.split_mode;
+  args.partials = p.partials;
+  args.splits = 1;
   return p.fp8 ? dispatch<false, true>(p, a1, w13, args, stream) : dispatch<false, false>(p, a1, w13, args, stream);
 }
 
@@ -1216,9 +1270,8 @@ cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const float* a2_s
   args.out = y;
   args.out_scale_t = nullptr;
   args.status = p.status;
-  args.partials = p.partials2;
-  args.tile_counters = p.counters2;
-  args.split_mode = p.split_mode;
+  args.partials = p.partials;
+  args.splits = 1;
   return p.fp8 ? dispatch<true, true>(p, a2, w2, args, stream) : dispatch<true, false>(p, a2, w2, args, stream);
 }
 

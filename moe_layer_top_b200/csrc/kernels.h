@@ -48,11 +48,10 @@ cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in,
                                      int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp, int32_t* counts,
                                      int32_t* offsets, int* status, cudaStream_t stream);
 
-// gather x rows into sorted order (bf16 copy, or FP8 per-(row,128) quantisation);
-// also zeroes `zero_n` ints at `zero` (the split-K tile counters of the GEMMs)
+// gather x rows into sorted order (bf16 copy, or FP8 per-(row,128) quantisation)
 cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32_t* sorted_ids,
-                          const int32_t* ntpp, int capacity, bool fp8, void* a1, float* a1_scale_t, int* zero,
-                          int zero_n, cudaStream_t stream);
+                          const int32_t* ntpp, int capacity, bool fp8, void* a1, float* a1_scale_t,
+                          cudaStream_t stream);
 
 // out[t] = sum_j y[t*topk + j]
 cudaError_t launch_combine(const void* y, int T, int topk, int H, void* out, cudaStream_t stream);
@@ -71,21 +70,21 @@ struct GemmProblem {
   const float* topk_weights;  // [nflat]
   int* status;
   int num_sms;
-  int split_mode;      // 0 auto, 1 off (swap-AB split-K)
-  float* partials1;    // split-K partial sums of GEMM1 / GEMM2 (swap-AB)
-  float* partials2;
-  int* counters1;      // per-tile arrival counters, zero before the launch
-  int* counters2;
+  int split_mode;      // swap-AB split-K: 0 when few tiles are in flight, 1 never
+  float* partials;     // swap-AB split-K partial sums [unit][acc column][128] (reused by both GEMMs)
 };
 
 // swap-AB split-K: at most this many (tile, split) units per launch
-constexpr int kMaxSplitUnits = 1024;
+constexpr int kMaxSplitUnits = 320;  // >= 4 splits x (148 SMs / 2) tiles
 
-// GEMM1 + fused SiLU*up (+ FP8 requant): a1 [cap, H] -> a2 [cap, I] (+ a2_scale_t [I/128, cap])
+// GEMM1 + fused SiLU*up (+ FP8 requant): a1 [cap, H] -> a2 [cap, I] (+ a2_scale_t [I/128, cap]).
+// In swap-AB mode with split-K allowed this launches the GEMM and then the
+// split-K reduce kernel (which exits at once when the GEMM did not split).
 cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const float* a1_scale_t, const void* w13,
                          const float* w13_scale, void* a2, float* a2_scale_t, cudaStream_t stream);
 
-// GEMM2 + routed weight: a2 [cap, I] -> y [nflat, H] bf16 (rows scattered by sorted_ids)
+// GEMM2 + routed weight: a2 [cap, I] -> y [nflat, H] bf16 (rows scattered by sorted_ids);
+// swap-AB split-K launches the reduce kernel after it, as for GEMM1
 cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const float* a2_scale_t, const void* w2,
                          const float* w2_scale, void* y, cudaStream_t stream);
 

@@ -63,7 +63,7 @@ class MoeWorkspaceLayout(ctypes.Structure):
         ("num_tokens_post_padded", ctypes.c_int64), ("expert_counts", ctypes.c_int64),
         ("expert_offsets", ctypes.c_int64), ("align_scratch", ctypes.c_int64), ("a1", ctypes.c_int64),
         ("a1_scale", ctypes.c_int64), ("a2", ctypes.c_int64), ("a2_scale", ctypes.c_int64), ("y", ctypes.c_int64),
-        ("partials", ctypes.c_int64), ("tile_counters", ctypes.c_int64), ("total_bytes", ctypes.c_int64), ("capacity", ctypes.c_int32), ("block_m", ctypes.c_int32),
+        ("partials", ctypes.c_int64), ("total_bytes", ctypes.c_int64), ("capacity", ctypes.c_int32), ("block_m", ctypes.c_int32),
         ("mode", ctypes.c_int32), ("align_chunks", ctypes.c_int32),
     ]
 
@@ -263,6 +263,7 @@ def workspace_views(p: MoeProblem, ws: torch.Tensor) -> dict:
         "a2": view(L.a2, cap * q.I, torch.uint8 if fp8 else torch.bfloat16, (cap, q.I)),
         "a2_scale_t": view(L.a2_scale, cap * (q.I // 128), torch.float32, (q.I // 128, cap)),
         "y": view(L.y, nflat * q.H, torch.bfloat16, (nflat, q.H)),
+        "partials": view(L.partials, (L.total_bytes - L.partials) // 4, torch.float32, (-1,)),
         "layout": L,
         "problem": q,
     }

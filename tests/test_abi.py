@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_struct_sizes_match_header():
     assert ctypes.sizeof(ops.MoeProblem) == 16 * 4
-    assert ctypes.sizeof(ops.MoeWorkspaceLayout) == 17 * 8 + 4 * 4
+    assert ctypes.sizeof(ops.MoeWorkspaceLayout) == 16 * 8 + 4 * 4
 
 
 def test_align_capacity_formula(L):

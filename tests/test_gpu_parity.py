@@ -260,18 +260,24 @@ def test_block_size_invariance(cfg):
     assert nr <= (2e-2 if cfg.fp8 else 5e-3) and mr <= 0.05
 
 
-@pytest.mark.parametrize("name,T", [("mid_bf16", 1), ("mid_bf16", 3), ("mid_fp8", 2)])
+@pytest.mark.parametrize("name,T", [("mid_bf16", 1), ("mid_bf16", 3), ("mid_fp8", 2), ("mid_fp8", 9),
+                                    ("mid_bf16", 5)])
 def test_split_k_matches_oracle_and_unsplit(name, T):
-    """With fewer tiles than half the SMs the swap-AB GEMMs split K; the split
-    result matches the oracle and the unsplit kernel within tolerance, and is
-    itself run-to-run deterministic."""
+    """With at most half as many tiles as SMs the swap-AB GEMMs split K and a reduce kernel
+    adds the splits; the result matches the oracle and the unsplit kernel
+    within tolerance, and is itself run-to-run deterministic.  The partial-sum
+    buffer is written only when a split happened."""
     cfg = {"mid_bf16": MID_BF16, "mid_fp8": MID_FP8}[name]
     w = inputs.make_weights(cfg, 0, device="cuda")
     a = Case(cfg, T, seed=0, weights=w)
+    a.views()["partials"].fill_(float("nan"))
     out_split = a.run().clone()
+    assert not torch.all(torch.isnan(a.views()["partials"]))   # the GEMMs did split
     assert torch.equal(out_split, a.run())
     b = Case(cfg, T, seed=0, weights=w, split_k=False)
+    b.views()["partials"].fill_(float("nan"))
     out_plain = b.run().clone()
+    assert torch.all(torch.isnan(b.views()["partials"]))
     ref = a.oracle()
     assert_close(out_split.float().cpu().numpy(), ref["out"], fp8=cfg.fp8)
     assert_close(out_plain.float().cpu().numpy(), ref["out"], fp8=cfg.fp8)
