@@ -331,20 +331,27 @@ class StageEvents:
         return [self.ev[i].elapsed_time(self.ev[i + 1]) for i in range(len(self.ev) - 1)]
 
 
-def capture(fn, count_kernels=False):
-    """Capture fn() into a CUDA graph (after it has run once eagerly); with
-    count_kernels, also return the number of kernel nodes in it."""
+def capture(fn):
+    """Capture fn() into a CUDA graph (after it has run once eagerly)."""
     fn()
     torch.cuda.synchronize()
-    g = torch.cuda.CUDAGraph(keep_graph=count_kernels)
+    g = torch.cuda.CUDAGraph()
     with torch.cuda.graph(g):
         fn()
     torch.cuda.synchronize()
-    if not count_kernels:
-        return g
+    return g
+
+
+def count_kernels(fn):
+    """Kernel launches of one fn() call, read from a separate capture that is
+    never replayed (the timed graph is captured the ordinary way)."""
+    g = torch.cuda.CUDAGraph(keep_graph=True)
+    with torch.cuda.graph(g):
+        fn()
+    torch.cuda.synchronize()
     n = graph_kernel_count(g)
-    g.instantiate()
-    return g, n
+    del g
+    return n
 
 
 def time_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor, world: int):
@@ -353,7 +360,8 @@ def time_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor, world
     B) a CUDA graph of the same stages with event nodes between them -> per-stage times."""
     ops = wl.ops
     stream = torch.cuda.current_stream()
-    g_fwd, n_kernels = capture(wl.forward, count_kernels=True)
+    n_kernels = count_kernels(wl.forward)
+    g_fwd = capture(wl.forward)
     se = StageEvents(ops.NUM_STAGES + 1)
 
     def staged():

@@ -1188,11 +1188,7 @@ cudaError_t launch_fp8_pair(const GemmProblem& p, const void* tok, const void* w
   if (!make_map(&tm_w, w, wrows, K, 1, 128)) return cudaErrorInvalidValue;
   const int n_tiles = (kDown ? p.H : p.I) / C::kTileN;
   const long long max_tiles = static_cast<long long>(p.capacity / 256) * n_tiles;
-  long long grid = p.num_sms / 2 * 2;
-  if (2 * max_tiles < grid) grid = 2 * max_tiles;
-  if (grid <= 0) return cudaSuccess;
   cudaLaunchConfig_t cfg = {};
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
   cfg.blockDim = dim3(kThreads);
   cfg.dynamicSmemBytes = C::kSmemBytes;
   cfg.stream = s;
@@ -1205,6 +1201,23 @@ cudaError_t launch_fp8_pair(const GemmProblem& p, const void* tok, const void* w
   attr[1].val.clusterDim.z = 1;
   cfg.attrs = attr;
   cfg.numAttrs = 2;
+  // The kernel is persistent: every cluster must be resident at once, or the
+  // clusters that do not fit run their whole share of tiles after the others.
+  // Not every SM can pair up (the SM count per GPC need not be even), so the
+  // grid is the number of clusters that fit, not num_sms / 2.
+  static int max_clusters = 0;
+  if (max_clusters == 0) {
+    cfg.gridDim = dim3(static_cast<unsigned>(p.num_sms / 2 * 2));
+    int n = 0;
+    cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
+    if (e != cudaSuccess) return e;
+    max_clusters = n > 0 ? n : 1;
+  }
+  long long grid = 2LL * max_clusters;
+  if (grid > p.num_sms / 2 * 2) grid = p.num_sms / 2 * 2;
+  if (2 * max_tiles < grid) grid = 2 * max_tiles;
+  if (grid <= 0) return cudaSuccess;
+  cfg.gridDim = dim3(static_cast<unsigned>(grid));
   return cudaLaunchKernelEx(&cfg, kern, tm_tok, tm_w, args);
 }
 
