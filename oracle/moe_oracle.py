@@ -31,6 +31,8 @@ Readings where the pages are silent (each also listed in the design doc):
   ``e4m3(fp32(w / scale))``.
 * combine: ``out[t] = sum_j w[t,j] * y[t,j]`` exactly (float64 here), rounded
   once to bf16; duplicate expert ids in a row are independent assignments.
+* MXFP8: one E8M0 scale per 32 consecutive elements of a row, chosen by the
+  same power-of-two rule as the per-(row,128) activation scale.
 
 Parity pins for every function live in ``tests/test_oracle_*.py``.
 """
@@ -69,6 +71,10 @@ _F32_INV_448 = np.float32(1.0 / 448.0)
 # ----------------------------------------------------------------------------
 # number formats
 # ----------------------------------------------------------------------------
+
+MX_GROUP = 32          # elements per MXFP8 scale
+E8M0_BIAS = 127        # E8M0 byte of the scale 2**0
+
 
 def round_bf16(x) -> np.ndarray:
     """Round to the nearest bfloat16 value, ties to even; result as float64.
@@ -226,6 +232,48 @@ def dequantize_weight_block128(codes, scales) -> np.ndarray:
     return vals * full
 
 
+def quantize_mx_group32(v):
+    """MXFP8: E4M3 elements with one power-of-two (E8M0) scale per 32 consecutive
+    elements of a row.
+
+    [PPLX] "Quantisierung": Blackwell's micro-scaling formats; Qwen3-235B is
+    served with MXFP8 weights.  The page names the scheme but not its scale
+    rule.  Reading: the power-of-two rule of [PR] §1.2 (raw scale
+    ``max(amax, 1e-10) * (1/448)`` in fp32, scale = the smallest power of two
+    at or above it) on 32-element groups -- an E8M0 byte holds exactly the
+    powers of two, and this choice never clips the group maximum.  The same
+    rule serves weights (groups along K of each row) and activations.
+
+    v: float64 [..., K] holding fp32-representable values, K % 32 == 0.
+    Returns (codes uint8 [..., K], e8m0 uint8 [..., K // 32]) with
+    scale = 2 ** (e8m0 - 127).
+    """
+    v = np.asarray(v, dtype=np.float64)
+    *lead, k = v.shape
+    if k % MX_GROUP:
+        raise ValueError("K must be a multiple of 32")
+    g = v.reshape(*lead, k // MX_GROUP, MX_GROUP)
+    amax = np.abs(g).max(axis=-1).astype(np.float32)
+    raw = np.maximum(amax, _F32_1E_10) * _F32_INV_448          # one fp32 rounding
+    scale = pow2_ceil(raw.astype(np.float64))
+    q = np.clip(g / scale[..., None], -E4M3_MAX, E4M3_MAX)     # exact: scale is 2**n
+    codes = e4m3_encode(q).reshape(*lead, k)
+    exponent = np.frexp(scale)[1] - 1                           # scale == 2**exponent
+    return codes, (exponent + E8M0_BIAS).astype(np.uint8)
+
+
+def mx_scale(e8m0) -> np.ndarray:
+    """E8M0 byte -> its power-of-two value (the NaN byte 0xFF is never produced)."""
+    return np.ldexp(1.0, np.asarray(e8m0).astype(np.int64) - E8M0_BIAS)
+
+
+def dequantize_mx_group32(codes, e8m0) -> np.ndarray:
+    codes = np.asarray(codes)
+    *lead, k = codes.shape
+    vals = e4m3_decode(codes).reshape(*lead, k // MX_GROUP, MX_GROUP)
+    return (vals * mx_scale(e8m0)[..., None]).reshape(*lead, k)
+
+
 # ----------------------------------------------------------------------------
 # routing and alignment
 # ----------------------------------------------------------------------------
@@ -309,14 +357,15 @@ def align(topk_ids, E: int, block_m: int):
 # expert MLP and the layer
 # ----------------------------------------------------------------------------
 
-def expert_mlp(x_hat, w13_hat, w2_hat, requant: bool, return_intermediates: bool = False):
+def expert_mlp(x_hat, w13_hat, w2_hat, requant, return_intermediates: bool = False):
     """One expert's SiLU-gated MLP on a batch of rows.
 
     [PR] §1.1/§1.2: ``h = x · w13ᵀ`` held in bf16 (``intermediate_cache1``);
     gate = columns [0, I), up = columns [I, 2I); ``silu(gate)`` rounded to
     bf16 before it multiplies ``up``; the product rounded to bf16; for the
     FP8 path it is re-quantised per (row, 128) before the down projection
-    ``y = a2 · w2ᵀ``.
+    ``y = a2 · w2ᵀ`` (``requant=True``), for MXFP8 per (row, 32) with an E8M0
+    scale (``requant="mx"``), for bf16 kept as is (``requant=False``).
 
     x_hat [n, H], w13_hat [2I, H], w2_hat [H, I]: float64.  Returns y [n, H].
     """
@@ -325,7 +374,10 @@ def expert_mlp(x_hat, w13_hat, w2_hat, requant: bool, return_intermediates: bool
     gate, up = h[:, :i], h[:, i:]
     act = round_bf16(gate / (1.0 + np.exp(-gate)))
     p = round_bf16(act * up)
-    if requant:
+    if requant == "mx":
+        codes, scales = quantize_mx_group32(p)
+        p_hat = dequantize_mx_group32(codes, scales)
+    elif requant:
         codes, scales = quantize_act_group128(p)
         p_hat = dequantize_act_group128(codes, scales)
     else:
@@ -348,8 +400,10 @@ def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weigh
 
     x:   [T, H] float (bf16 values).
     w13: [E, 2I, H] bf16 values (float) -- or E4M3 codes (uint8) with
-         ``w13_scale`` [E, 2I/128, H/128] for the FP8 block-quantised path.
-    w2:  [E, H, I] likewise with ``w2_scale`` [E, H/128, I/128].
+         ``w13_scale`` [E, 2I/128, H/128] float32 for the FP8 block-quantised
+         path, or ``w13_scale`` [E, 2I, H/32] uint8 (E8M0) for MXFP8, where x
+         and the intermediate are MX-quantised too.
+    w2:  [E, H, I] likewise with ``w2_scale`` [E, H/128, I/128] or [E, H, I/32].
     Routing: ``logits`` [T, E] float32, or ``topk_ids``/``topk_weights``.
     tokens: optional subset of token indices to evaluate (each output row
     depends only on its own token, its routing and the weights).
@@ -362,6 +416,7 @@ def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weigh
     fp8 = w13_scale is not None
     if fp8 != (w2_scale is not None):
         raise ValueError("w13_scale and w2_scale go together")
+    mx = fp8 and np.asarray(w13_scale).dtype == np.uint8
     if logits is not None:
         topk_ids, topk_weights = route(logits, topk, renormalize)
     topk_ids = np.asarray(topk_ids).astype(np.int64)
@@ -370,7 +425,10 @@ def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weigh
     tokens = np.arange(t_all) if tokens is None else np.asarray(tokens, dtype=np.int64)
 
     xs = x[tokens]
-    if fp8:
+    if mx:
+        qx, sx = quantize_mx_group32(xs)
+        x_hat = dequantize_mx_group32(qx, sx)
+    elif fp8:
         qx, sx = quantize_act_group128(xs)
         x_hat = dequantize_act_group128(qx, sx)
     else:
@@ -382,13 +440,16 @@ def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weigh
     y_all = np.zeros((tokens.size, topk, h_dim), dtype=np.float64) if return_y else None
     for e in np.unique(ids):
         rows, cols = np.nonzero(ids == e)                        # (token, slot) pairs on expert e
-        if fp8:
+        if mx:
+            w13_e = dequantize_mx_group32(w13[e], w13_scale[e])
+            w2_e = dequantize_mx_group32(w2[e], w2_scale[e])
+        elif fp8:
             w13_e = dequantize_weight_block128(w13[e], w13_scale[e])
             w2_e = dequantize_weight_block128(w2[e], w2_scale[e])
         else:
             w13_e = np.asarray(w13[e], dtype=np.float64)
             w2_e = np.asarray(w2[e], dtype=np.float64)
-        y = expert_mlp(x_hat[rows], w13_e, w2_e, requant=fp8)
+        y = expert_mlp(x_hat[rows], w13_e, w2_e, requant="mx" if mx else fp8)
         for r, c, yr in zip(rows, cols, y):
             acc[r] += wts[r, c] * yr
             if return_y:

@@ -156,6 +156,36 @@ def test_weight_block_quant_properties_and_torch_path():
     assert np.all(np.abs(deq - w) <= bound)
 
 
+def test_mx_quant_properties_and_independent_torch_path():
+    rng = np.random.default_rng(7)
+    p = O.round_bf16(rng.standard_normal((16, 256)) * np.exp(rng.uniform(-6, 3, (16, 1))))
+    p[2, 32:64] = 0.0                                         # an all-zero 32-group
+    p[5, 100] = 1000.0                                        # one large value: only its group's scale moves
+    codes, e8m0 = O.quantize_mx_group32(p)
+    assert codes.shape == p.shape and e8m0.shape == (16, 8) and e8m0.dtype == np.uint8
+    s = O.mx_scale(e8m0)
+    assert np.all(np.frexp(s)[0] == 0.5), "scales must be powers of two"
+    amax = np.abs(p.reshape(16, 8, 32)).max(-1)
+    nz = amax > 0
+    ratio = amax[nz] / s[nz]
+    assert np.all(ratio <= 448.0) and np.all(ratio > 224.0)
+    assert e8m0[5, 3] > e8m0[5, 2] and e8m0[5, 3] > e8m0[5, 4]
+    floor = np.float32(np.float32(1e-10) * np.float32(1.0 / 448.0))
+    assert s[2, 1] >= floor and s[2, 1] < 2 * floor
+    # the E8M0 byte is the biased exponent of the scale
+    np.testing.assert_array_equal(e8m0.astype(np.int64) - 127, np.frexp(s)[1] - 1)
+    # independent path: torch amax over 32-groups, log2/ceil/exp2, float8 cast
+    pt = torch.from_numpy(p).reshape(16, 8, 32)
+    raw = torch.clamp(pt.abs().amax(-1).float(), min=1e-10) * torch.tensor(1.0 / 448.0, dtype=torch.float32)
+    sc = torch.exp2(torch.ceil(torch.log2(raw.double())))
+    q = torch.clamp(pt / sc[..., None], -448, 448).float().to(torch.float8_e4m3fn)
+    np.testing.assert_array_equal(codes, q.view(torch.uint8).reshape(16, 256).numpy())
+    np.testing.assert_array_equal(s, sc.numpy())
+    deq = O.dequantize_mx_group32(codes, e8m0)
+    err = np.abs(deq - p).reshape(16, 8, 32)
+    assert np.all(err <= np.maximum(np.abs(p).reshape(16, 8, 32) * 2.0 ** -4, 2.0 ** -10 * s[..., None]))
+
+
 def test_page_constants_fixture():
     with open(os.path.join(GOLDEN, "pr64760_quant_constants.json")) as f:
         gold = json.load(f)

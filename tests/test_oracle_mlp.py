@@ -66,6 +66,62 @@ def test_expert_mlp_closed_form_fp8_requant():
     np.testing.assert_array_equal(y, ref)
 
 
+def test_expert_mlp_closed_form_mx_requant():
+    H, I = 256, 128
+    w13, w2, perm, perm2 = _selection_weights(H, I, 4)
+    rng = np.random.default_rng(5)
+    x = O.round_bf16(rng.standard_normal((5, H)) * np.exp(rng.uniform(-3, 3, (5, H))))
+    y = O.expert_mlp(x, w13, w2, requant="mx")
+    g = torch.from_numpy(x[:, perm[:I]])
+    u = torch.from_numpy(x[:, perm[I:2 * I]])
+    p = ((F.silu(g).to(torch.bfloat16).double() * u).to(torch.bfloat16)).float().reshape(5, I // 32, 32)
+    raw = torch.clamp(p.abs().amax(-1, keepdim=True), min=1e-10) * torch.tensor(1 / 448.0)
+    sc = torch.exp2(torch.ceil(torch.log2(raw.double())))
+    q = ((p.double() / sc).float().to(torch.float8_e4m3fn).double() * sc).reshape(5, I)
+    ref = np.zeros_like(y)
+    ref[:, perm2[:I]] = q.numpy()
+    np.testing.assert_array_equal(y, ref)
+
+
+def _mx_torch(t, group=32):
+    """Independent MX quantise-dequantise of the last dim with torch ops."""
+    shp = t.shape
+    g = t.reshape(*shp[:-1], shp[-1] // group, group).float()
+    raw = torch.clamp(g.abs().amax(-1), min=1e-10) * torch.tensor(1 / 448.0)
+    sc = torch.exp2(torch.ceil(torch.log2(raw.double())))
+    q = torch.clamp(g.double() / sc[..., None], -448, 448).float().to(torch.float8_e4m3fn).double()
+    return (q * sc[..., None]).reshape(shp)
+
+
+def test_forward_matches_dense_bruteforce_mx_with_duplicate_ids():
+    cfg = inputs.make_custom_config("tiny_mx", E=5, topk=3, H=256, I=128, fp8=True,
+                                    routing="uniform_ids", tokens=(10,))
+    w13, w2 = inputs.make_weights(cfg, 6)
+    x = inputs.make_tokens(cfg, 10, 6)
+    r = inputs.make_routing(cfg, 10, 6)
+    ids = r["topk_ids"].numpy().copy()
+    ids[1] = [4, 4, 0]
+    wts = r["topk_weights"].numpy()
+    q13, s13 = O.quantize_mx_group32(w13.double().numpy())
+    q2, s2 = O.quantize_mx_group32(w2.double().numpy())
+    assert s13.shape == (5, 256, 8) and s2.shape == (5, 256, 4)
+    xn = x.double().numpy()
+    res = O.moe_forward(xn, q13, q2, cfg.topk, topk_ids=ids, topk_weights=wts, w13_scale=s13, w2_scale=s2)
+    # dense torch evaluation: weights MX-quantised by torch from the same draw
+    xt = _mx_torch(torch.from_numpy(xn))
+    W13 = _mx_torch(w13.double())
+    W2 = _mx_torch(w2.double())
+    h = torch.einsum("th,enh->etn", xt, W13).to(torch.bfloat16).double()
+    I = 128
+    p = (F.silu(h[..., :I]).to(torch.bfloat16).double() * h[..., I:]).to(torch.bfloat16).double()
+    y = torch.einsum("eti,ehi->eth", _mx_torch(p), W2)
+    mask = torch.zeros(10, 5, dtype=torch.float64)
+    mask.scatter_add_(1, torch.from_numpy(ids).long(), torch.from_numpy(wts).double())
+    ref = torch.einsum("te,eth->th", mask, y).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(res["out"], ref)
+    assert np.abs(res["out"]).max() > 0
+
+
 def _dense_reference(x, w13, w2, ids, wts, fp8, w13_scale=None, w2_scale=None):
     """Every expert on every token with torch ops, combined through a dense
     [T, E] weight mask; rounding points from torch's casts."""
