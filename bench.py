@@ -210,7 +210,7 @@ class Workload:
         self.w13, self.w2, self.s13, self.s2 = weights
         self.x = inputs.make_tokens(cfg, T, seed, device=dev)
         self.routing = inputs.make_routing(cfg, T, seed, device=dev)
-        self.p = ops.problem(T, cfg.E, cfg.topk, cfg.H, cfg.I, fp8=cfg.fp8)
+        self.p = ops.problem(T, cfg.E, cfg.topk, cfg.H, cfg.I, fp8=cfg.fp8, mx=cfg.mx)
         self.q = ops.resolve_problem(self.p)
         self.ws = ops.alloc_workspace(self.p)
         self.out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
@@ -234,8 +234,12 @@ class Workload:
         hit = int((counts > 0).sum())
         cfg = self.cfg
         elem = 1 if cfg.fp8 else 2
-        w13_e = 2 * cfg.I * cfg.H * elem + (2 * cfg.I // 128) * (cfg.H // 128) * 4 * cfg.fp8
-        w2_e = cfg.H * cfg.I * elem + (cfg.H // 128) * (cfg.I // 128) * 4 * cfg.fp8
+        if cfg.mx:   # one E8M0 byte per 32 weights
+            w13_e = 2 * cfg.I * cfg.H * (1 + 1 / 32)
+            w2_e = cfg.H * cfg.I * (1 + 1 / 32)
+        else:
+            w13_e = 2 * cfg.I * cfg.H * elem + (2 * cfg.I // 128) * (cfg.H // 128) * 4 * cfg.fp8
+            w2_e = cfg.H * cfg.I * elem + (cfg.H // 128) * (cfg.I // 128) * 4 * cfg.fp8
         nflat = self.T * cfg.topk
         route_io = self.T * cfg.E * 4 if "logits" in self.routing else nflat * 8
         rows = ntpp
@@ -280,8 +284,9 @@ def make_weights(cfg, seed):
     from moe_layer_top_b200 import ops
     w13, w2 = inputs.make_weights(cfg, seed, device="cuda")
     if cfg.fp8:
-        q13, s13 = ops.quantize_weights_fp8(w13)
-        q2, s2 = ops.quantize_weights_fp8(w2)
+        quant = ops.quantize_weights_mxfp8 if cfg.mx else ops.quantize_weights_fp8
+        q13, s13 = quant(w13)
+        q2, s2 = quant(w2)
         del w13, w2
         torch.cuda.empty_cache()
         return q13, q2, s13, s2
@@ -462,8 +467,12 @@ def cpu_baseline(cfg, T, seed, budget_s):
                 a, b = inputs.make_expert_weights(cfg, e, seed, device=dev)
                 a = a.float().cpu().double().numpy()
                 b = b.float().cpu().double().numpy()
-                host[e] = (*O.quantize_weight_block128(a), *O.quantize_weight_block128(b)) if cfg.fp8 \
-                    else (a, None, b, None)
+                if cfg.mx:
+                    host[e] = (*O.quantize_mx_group32(a), *O.quantize_mx_group32(b))
+                elif cfg.fp8:
+                    host[e] = (*O.quantize_weight_block128(a), *O.quantize_weight_block128(b))
+                else:
+                    host[e] = (a, None, b, None)
 
     class View:
         def __init__(self, i):
@@ -479,7 +488,8 @@ def cpu_baseline(cfg, T, seed, budget_s):
         prepare(tok)
         t0 = time.perf_counter()
         if cfg.fp8:
-            O.moe_forward(x, View(0), View(2), cfg.topk, w13_scale=View(1), w2_scale=View(3), tokens=tok, **rkw)
+            O.moe_forward(x, View(0), View(2), cfg.topk, w13_scale=View(1), w2_scale=View(3), tokens=tok,
+                          mx=cfg.mx, **rkw)
         else:
             O.moe_forward(x, View(0), View(2), cfg.topk, tokens=tok, **rkw)
         t_spent += time.perf_counter() - t0
@@ -569,10 +579,11 @@ def run_ours(args, rank, world, local):
         "metric": "fused-MoE tokens/s; % HBM roofline (decode), % FP8/BF16 TC peak (prefill)",
         "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
         "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
-        "dtype": "fp8_e4m3" if cfg.fp8 else "bf16", "data": "synthetic",
+        "dtype": ("mxfp8_e4m3" if cfg.mx else "fp8_e4m3") if cfg.fp8 else "bf16", "data": "synthetic",
         "config": {"workload": f"{cfg.name}: H={cfg.H} E={cfg.E} topk={cfg.topk} I={cfg.I} T={T_head}",
                    "global_batch": world * T_head, "tokens_per_gpu": T_head, "parallelism": f"replicas{world}",
-                   "weights": "fp8 e4m3 + 128x128 fp32 scales" if cfg.fp8 else "bf16",
+                   "weights": ("mxfp8 e4m3 + per-32 e8m0 scales" if cfg.mx else "fp8 e4m3 + 128x128 fp32 scales")
+                   if cfg.fp8 else "bf16",
                    "routing": cfg.routing, "l2": "flushed (256 MiB write) before every step, outside the timing",
                    "launch": "CUDA graph of moe_fused_forward (PDL between kernels)",
                    "layer_bytes_per_step": alg["layer_bytes"], "hit_experts": alg["hit_experts"]},

@@ -70,6 +70,19 @@ extern "C" {
 /* weight types */
 #define MOE_DTYPE_BF16 0
 #define MOE_DTYPE_FP8_E4M3 1 /* E4M3 codes + one fp32 scale per 128 x 128 block */
+#define MOE_DTYPE_MXFP8_E4M3 2 /* E4M3 codes + one E8M0 (power-of-two) scale per 32 elements of a row;
+                                 normal tiles only (mode NORMAL, block_m 128) */
+
+/*
+ * MXFP8 scale-factor layout ("SF atoms"), used for MXFP8 weights and for the
+ * activation scales the library writes.  For a matrix [.., N, K] (K the
+ * reduction axis) the E8M0 byte of element (n, k) of batch b lives at
+ *   ((b * (N/128) + n/128) * (K/128) + k/128) * 512
+ *     + (n % 32) * 16 + ((n % 128) / 32) * 4 + (k % 128) / 32,
+ * i.e. one contiguous 512-byte atom per 128 rows x 128 columns, in the order
+ * the tensor cores read scale factors (tcgen05.cp 32x128b, 4 warps).  E8M0
+ * byte v encodes 2^(v - 127).
+ */
 
 /* tile orientation of the two grouped GEMMs */
 #define MOE_MODE_AUTO 0    /* chosen from the expected tokens per expert */
@@ -122,9 +135,9 @@ typedef struct moe_workspace_layout {
   int64_t expert_offsets;   /* int32 [E + 1] */
   int64_t align_scratch;    /* int32 [chunks * E] */
   int64_t a1;               /* bf16 or E4M3 [capacity, H] x rows in sorted order (padding rows unspecified) */
-  int64_t a1_scale;         /* fp32 [H/128, capacity] (FP8 only; K-block major) */
+  int64_t a1_scale;         /* fp32 [H/128, capacity] (FP8, K-block major); E8M0 SF atoms of [capacity, H] (MXFP8) */
   int64_t a2;               /* bf16 or E4M3 [capacity, I] activation in sorted order (padding rows unspecified) */
-  int64_t a2_scale;         /* fp32 [I/128, capacity] (FP8 only; K-block major) */
+  int64_t a2_scale;         /* fp32 [I/128, capacity] (FP8, K-block major); E8M0 SF atoms of [capacity, I] (MXFP8) */
   int64_t y;                /* bf16 [T*topk, H] weighted expert outputs */
   int64_t partials;         /* fp32 split-K partial sums of the swap-AB GEMMs (swap-AB only) */
   int64_t total_bytes;
@@ -216,6 +229,19 @@ MOE_API int moe_align_noalloc(const int32_t* topk_ids, int32_t T, int32_t topk, 
 MOE_API int moe_quantize_weights_fp8(const void* w, int64_t batches, int32_t rows, int32_t cols, uint8_t* codes,
                              float* scales, void* stream);
 
+/*
+ * MXFP8 weight preparation ("Hosting von Qwen auf Blackwell", section
+ * "Quantisierung": micro-scaled FP8 weights on Blackwell).  w [batches, rows,
+ * cols] bf16 -> codes [batches, rows, cols] E4M3 and E8M0 scale factors in the
+ * SF-atom layout above (batches * rows * cols / 32 bytes).  Per row and 32
+ * consecutive columns: scale = the smallest power of two >= fp32(max(amax,
+ * 1e-10)) * fp32(1/448), code = e4m3(w / scale) (exact division, round to
+ * nearest even, saturating).  rows and cols must be multiples of 128; codes
+ * 16-byte and sf 16-byte aligned.
+ */
+MOE_API int moe_quantize_weights_mxfp8(const void* w, int64_t batches, int32_t rows, int32_t cols, uint8_t* codes,
+                                       uint8_t* sf, void* stream);
+
 /* Fill in mode and block_m when they are left to the library; validates p. */
 MOE_API int moe_resolve_problem(moe_problem* p);
 
@@ -230,8 +256,11 @@ MOE_API int moe_get_workspace_layout(const moe_problem* p, moe_workspace_layout*
  *   x             [T, H] bf16.
  *   router_logits [T, E] fp32, or NULL to use topk_ids / topk_weights
  *                 ([T, topk] int32 / fp32), which are then required.
- *   w13           [E, 2I, H]: bf16, or E4M3 codes with w13_scale [E, 2I/128, H/128] fp32.
- *   w2            [E, H, I]:  bf16, or E4M3 codes with w2_scale  [E, H/128, I/128] fp32.
+ *   w13           [E, 2I, H]: bf16, or E4M3 codes with w13_scale [E, 2I/128, H/128] fp32
+ *                 (MOE_DTYPE_FP8_E4M3), or E4M3 codes with w13_scale as E8M0 SF atoms
+ *                 of [E, 2I, H] (MOE_DTYPE_MXFP8_E4M3; x and the intermediate are then
+ *                 MX-quantised the same way, per row and 32 columns).
+ *   w2            [E, H, I]:  likewise, w2_scale [E, H/128, I/128] fp32 or SF atoms of [E, H, I].
  *   out           [T, H] bf16.
  *   ws            device scratch of at least moe_workspace_size(p) bytes,
  *                 256-byte aligned; the call clears what must start at zero.
@@ -239,8 +268,8 @@ MOE_API int moe_get_workspace_layout(const moe_problem* p, moe_workspace_layout*
  * All pointers 16-byte aligned.  T = 0 is a no-op (its buffers may be NULL).
  */
 MOE_API int moe_fused_forward(const moe_problem* p, const void* x, const float* router_logits, const int32_t* topk_ids,
-                      const float* topk_weights, const void* w13, const void* w2, const float* w13_scale,
-                      const float* w2_scale, void* out, void* ws, size_t ws_bytes, void* stream);
+                      const float* topk_weights, const void* w13, const void* w2, const void* w13_scale,
+                      const void* w2_scale, void* out, void* ws, size_t ws_bytes, void* stream);
 
 /*
  * The same pipeline restricted to stages [stage_begin, stage_end) (MOE_STAGE_*),
@@ -248,8 +277,8 @@ MOE_API int moe_fused_forward(const moe_problem* p, const void* x, const float* 
  * partition in order is exactly moe_fused_forward.
  */
 MOE_API int moe_forward_stages(const moe_problem* p, const void* x, const float* router_logits, const int32_t* topk_ids,
-                       const float* topk_weights, const void* w13, const void* w2, const float* w13_scale,
-                       const float* w2_scale, void* out, void* ws, size_t ws_bytes, int32_t stage_begin,
+                       const float* topk_weights, const void* w13, const void* w2, const void* w13_scale,
+                       const void* w2_scale, void* out, void* ws, size_t ws_bytes, int32_t stage_begin,
                        int32_t stage_end, void* stream);
 
 /*

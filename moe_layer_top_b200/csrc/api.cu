@@ -72,7 +72,8 @@ int validate_problem(const moe_problem* p) {
   if (static_cast<int64_t>(p->E) * 2 * p->I >= (int64_t(1) << 31) ||
       static_cast<int64_t>(p->E) * p->H >= (int64_t(1) << 31))
     return fail(MOE_ERR_INVALID, "E * 2I or E * H overflows int32");
-  if (p->weight_dtype != MOE_DTYPE_BF16 && p->weight_dtype != MOE_DTYPE_FP8_E4M3)
+  if (p->weight_dtype != MOE_DTYPE_BF16 && p->weight_dtype != MOE_DTYPE_FP8_E4M3 &&
+      p->weight_dtype != MOE_DTYPE_MXFP8_E4M3)
     return fail(MOE_ERR_UNSUPPORTED, "weight_dtype %d", p->weight_dtype);
   if (p->mode < MOE_MODE_AUTO || p->mode > MOE_MODE_SWAP_AB) return fail(MOE_ERR_INVALID, "mode %d", p->mode);
   if (p->renormalize != 0 && p->renormalize != 1) return fail(MOE_ERR_INVALID, "renormalize must be 0 or 1");
@@ -80,6 +81,11 @@ int validate_problem(const moe_problem* p) {
   for (int i = 0; i < 6; ++i)
     if (p->reserved[i] != 0) return fail(MOE_ERR_INVALID, "reserved fields must be zero");
   const bool fp8 = p->weight_dtype == MOE_DTYPE_FP8_E4M3;
+  if (p->weight_dtype == MOE_DTYPE_MXFP8_E4M3) {
+    if (p->mode == MOE_MODE_SWAP_AB) return fail(MOE_ERR_UNSUPPORTED, "MXFP8 weights run normal tiles only");
+    if (p->block_m != 0 && p->block_m != 128)
+      return fail(MOE_ERR_INVALID, "MXFP8 weights use block_m = 128 (got %d)", p->block_m);
+  }
   if (p->block_m == 256 && !fp8)
     return fail(MOE_ERR_INVALID, "block_m = 256 (two-SM tiles) needs FP8 weights");
   if (p->mode == MOE_MODE_NORMAL && p->block_m != 0 && p->block_m != 128 && p->block_m != 256)
@@ -96,6 +102,11 @@ int validate_problem(const moe_problem* p) {
 // few tokens (the MMA M dimension is then filled by weight rows); the block
 // is the smallest of 16/32/64 that usually holds an expert's tokens whole.
 void resolve(moe_problem* p) {
+  if (p->weight_dtype == MOE_DTYPE_MXFP8_E4M3) {  // block-scaled MMA: normal tiles only
+    p->mode = MOE_MODE_NORMAL;
+    p->block_m = 128;
+    return;
+  }
   const int64_t n = static_cast<int64_t>(p->T) * p->topk;
   const int64_t hit = n < p->E ? n : p->E;
   const double avg = hit > 0 ? static_cast<double>(n) / static_cast<double>(hit) : 1.0;
@@ -126,7 +137,8 @@ struct Plan {
   moe_problem p;
   moe_workspace_layout L;
   int64_t nflat;
-  bool fp8;
+  bool fp8;  // 8-bit weights and activations (block-128 or MX scales)
+  bool mx;   // MXFP8: E8M0 scale factors per 32 elements
 };
 
 int make_plan(const moe_problem* in, Plan* plan) {
@@ -135,7 +147,8 @@ int make_plan(const moe_problem* in, Plan* plan) {
   plan->p = *in;
   resolve(&plan->p);
   const moe_problem& p = plan->p;
-  plan->fp8 = p.weight_dtype == MOE_DTYPE_FP8_E4M3;
+  plan->mx = p.weight_dtype == MOE_DTYPE_MXFP8_E4M3;
+  plan->fp8 = p.weight_dtype == MOE_DTYPE_FP8_E4M3 || plan->mx;
   plan->nflat = static_cast<int64_t>(p.T) * p.topk;
   const int64_t cap = capacity_of(p.T, p.topk, p.E, p.block_m);
   if (cap >= (int64_t(1) << 31)) return fail(MOE_ERR_INVALID, "padded row capacity overflows int32");
@@ -158,6 +171,7 @@ int make_plan(const moe_problem* in, Plan* plan) {
   L.expert_offsets = take(static_cast<int64_t>(p.E + 1) * 4);
   L.align_scratch = take(chunks * p.E * 4);
   L.a1 = take(cap * p.H * elem);
+  // FP8: fp32 [K/128, cap]; MXFP8: E8M0 SF atoms, (cap/128) * (K/128) * 512 bytes -- the same size
   L.a1_scale = plan->fp8 ? take(cap * (p.H / 128) * 4) : -1;
   L.a2 = take(cap * p.I * elem);
   L.a2_scale = plan->fp8 ? take(cap * (p.I / 128) * 4) : -1;
@@ -183,8 +197,8 @@ T* at(void* ws, int64_t off) {
 }
 
 int run_stages(const moe_problem* prob, const void* x, const float* logits, const int32_t* topk_ids,
-               const float* topk_weights, const void* w13, const void* w2, const float* w13_scale,
-               const float* w2_scale, void* out, void* ws, size_t ws_bytes, int stage_begin, int stage_end,
+               const float* topk_weights, const void* w13, const void* w2, const void* w13_scale,
+               const void* w2_scale, void* out, void* ws, size_t ws_bytes, int stage_begin, int stage_end,
                cudaStream_t stream) {
   Plan plan;
   int rc = make_plan(prob, &plan);
@@ -198,6 +212,8 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
   if (!logits && (!topk_ids || !topk_weights))
     return fail(MOE_ERR_INVALID, "give router_logits, or topk_ids and topk_weights");
   if (plan.fp8 && (!w13_scale || !w2_scale)) return fail(MOE_ERR_INVALID, "FP8 weights need w13_scale and w2_scale");
+  if (plan.mx && (!aligned(w13_scale, 16) || !aligned(w2_scale, 16)))
+    return fail(MOE_ERR_INVALID, "MXFP8 scale factors must be 16-byte aligned");
   if (!aligned(x, 16) || !aligned(w13, 16) || !aligned(w2, 16) || !aligned(out, 16))
     return fail(MOE_ERR_INVALID, "x, w13, w2 and out must be 16-byte aligned");
   if ((logits && !aligned(logits, 4)) || (topk_ids && !aligned(topk_ids, 4)) ||
@@ -263,8 +279,8 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
         break;
       case MOE_STAGE_GATHER:
         e = moe::launch_gather(x, p.H, p.topk, nflat, at<int32_t>(ws, L.sorted_token_ids),
-                               at<int32_t>(ws, L.num_tokens_post_padded), cap, plan.fp8, at<void>(ws, L.a1),
-                               plan.fp8 ? at<float>(ws, L.a1_scale) : nullptr, stream);
+                               at<int32_t>(ws, L.num_tokens_post_padded), cap, plan.fp8, plan.mx,
+                               at<void>(ws, L.a1), plan.fp8 ? at<void>(ws, L.a1_scale) : nullptr, stream);
         if (e != cudaSuccess) return cuda_fail(e, "gather");
         break;
       case MOE_STAGE_GEMM1:
@@ -278,6 +294,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
         gp.block_m = p.block_m;
         gp.capacity = cap;
         gp.fp8 = plan.fp8;
+        gp.mx = plan.mx;
         gp.swap = swap;
         gp.ntpp = at<int32_t>(ws, L.num_tokens_post_padded);
         gp.expert_ids = at<int32_t>(ws, L.expert_ids);
@@ -288,12 +305,12 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
         gp.split_mode = p.split_k;
         gp.partials = swap ? at<float>(ws, L.partials) : nullptr;
         if (s == MOE_STAGE_GEMM1) {
-          e = moe::launch_gemm1(gp, at<void>(ws, L.a1), plan.fp8 ? at<float>(ws, L.a1_scale) : nullptr, w13,
-                                w13_scale, at<void>(ws, L.a2), plan.fp8 ? at<float>(ws, L.a2_scale) : nullptr,
+          e = moe::launch_gemm1(gp, at<void>(ws, L.a1), plan.fp8 ? at<void>(ws, L.a1_scale) : nullptr, w13,
+                                w13_scale, at<void>(ws, L.a2), plan.fp8 ? at<void>(ws, L.a2_scale) : nullptr,
                                 stream);
           if (e != cudaSuccess) return cuda_fail(e, "gemm1");
         } else {
-          e = moe::launch_gemm2(gp, at<void>(ws, L.a2), plan.fp8 ? at<float>(ws, L.a2_scale) : nullptr, w2,
+          e = moe::launch_gemm2(gp, at<void>(ws, L.a2), plan.fp8 ? at<void>(ws, L.a2_scale) : nullptr, w2,
                                 w2_scale, at<void>(ws, L.y), stream);
           if (e != cudaSuccess) return cuda_fail(e, "gemm2");
         }
@@ -423,6 +440,20 @@ int moe_quantize_weights_fp8(const void* w, int64_t batches, int32_t rows, int32
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "quantize");
 }
 
+int moe_quantize_weights_mxfp8(const void* w, int64_t batches, int32_t rows, int32_t cols, uint8_t* codes,
+                               uint8_t* sf, void* stream) {
+  if (batches < 0 || rows <= 0 || cols <= 0 || rows % 128 || cols % 128)
+    return fail(MOE_ERR_INVALID, "quantize: batches=%lld rows=%d cols=%d (rows, cols multiples of 128)",
+                static_cast<long long>(batches), rows, cols);
+  if (batches > 0 && (!w || !codes || !sf)) return fail(MOE_ERR_INVALID, "quantize: NULL pointer");
+  if (!aligned(w, 16) || !aligned(codes, 16) || !aligned(sf, 16))
+    return fail(MOE_ERR_INVALID, "quantize: w, codes and sf must be 16-byte aligned");
+  int rc = device_check(nullptr);
+  if (rc != MOE_OK) return rc;
+  cudaError_t e = moe::launch_quantize_weights_mx(w, batches, rows, cols, codes, sf, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "quantize");
+}
+
 int moe_resolve_problem(moe_problem* p) {
   int rc = validate_problem(p);
   if (rc != MOE_OK) return rc;
@@ -446,15 +477,15 @@ int moe_get_workspace_layout(const moe_problem* p, moe_workspace_layout* layout)
 }
 
 int moe_fused_forward(const moe_problem* p, const void* x, const float* router_logits, const int32_t* topk_ids,
-                      const float* topk_weights, const void* w13, const void* w2, const float* w13_scale,
-                      const float* w2_scale, void* out, void* ws, size_t ws_bytes, void* stream) {
+                      const float* topk_weights, const void* w13, const void* w2, const void* w13_scale,
+                      const void* w2_scale, void* out, void* ws, size_t ws_bytes, void* stream) {
   return run_stages(p, x, router_logits, topk_ids, topk_weights, w13, w2, w13_scale, w2_scale, out, ws, ws_bytes, 0,
                     MOE_NUM_STAGES, static_cast<cudaStream_t>(stream));
 }
 
 int moe_forward_stages(const moe_problem* p, const void* x, const float* router_logits, const int32_t* topk_ids,
-                       const float* topk_weights, const void* w13, const void* w2, const float* w13_scale,
-                       const float* w2_scale, void* out, void* ws, size_t ws_bytes, int32_t stage_begin,
+                       const float* topk_weights, const void* w13, const void* w2, const void* w13_scale,
+                       const void* w2_scale, void* out, void* ws, size_t ws_bytes, int32_t stage_begin,
                        int32_t stage_end, void* stream) {
   return run_stages(p, x, router_logits, topk_ids, topk_weights, w13, w2, w13_scale, w2_scale, out, ws, ws_bytes,
                     stage_begin, stage_end, static_cast<cudaStream_t>(stream));

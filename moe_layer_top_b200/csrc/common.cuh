@@ -121,6 +121,16 @@ __device__ __forceinline__ void tma_load_2d(void* smem_dst, const void* map, uin
       : "memory");
 }
 
+// untiled bulk copy global -> this CTA's shared memory (16-byte aligned
+// addresses, size a multiple of 16); completes `bytes` on the mbarrier
+__device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint32_t bytes, uint64_t* bar) {
+  asm volatile(
+      "cp.async.bulk.shared::cluster.global.mbarrier::complete_tx::bytes [%0], [%1], %2, [%3];" ::"r"(
+          smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(src)), "r"(bytes), "r"(smem_u32(bar))
+      : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));
@@ -256,6 +266,40 @@ __device__ __forceinline__ void mma_fp8(uint32_t d_tmem, uint64_t a_desc, uint64
       "tcgen05.mma.cta_group::1.kind::f8f6f4 [%0], %1, %2, %3, p;\n\t}" ::"r"(d_tmem),
       "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate)
       : "memory");
+}
+
+// MXFP8 block-scaled MMA (kind::mxf8f6f4, one E8M0 scale per 32 K elements):
+// D[tmem] (+)= (A * sfa) x (B * sfb)^T with the scale factors read from TMEM at
+// tsfa / tsfb; bits 30-31 of those addresses select the byte (the 32-element
+// K block inside a 4-byte TMEM cell) and must equal the ids in the descriptor.
+__device__ __forceinline__ void mma_mxf8(uint32_t d_tmem, uint64_t a_desc, uint64_t b_desc, uint32_t idesc,
+                                         uint32_t accumulate, uint32_t tsfa, uint32_t tsfb) {
+  asm volatile(
+      "{\n\t.reg .pred p;\n\t"
+      "setp.ne.b32 p, %4, 0;\n\t"
+      "tcgen05.mma.cta_group::1.kind::mxf8f6f4.block_scale [%0], %1, %2, %3, [%5], [%6], p;\n\t}" ::"r"(d_tmem),
+      "l"(a_desc), "l"(b_desc), "r"(idesc), "r"(accumulate), "r"(tsfa), "r"(tsfb)
+      : "memory");
+}
+
+// Instruction descriptor of the block-scaled MMA: E4M3 A and B, E8M0 scales
+// (bit 23), N >> 3 at bit 17, M >> 4 at bit 24, scale-factor byte ids of B at
+// bits 4-5 and of A at bits 29-30.
+__host__ __device__ constexpr uint32_t make_idesc_mx(int M, int N, int sf_id) {
+  return (static_cast<uint32_t>(sf_id) << 4) | (static_cast<uint32_t>(N >> 3) << 17) | (1u << 23) |
+         (static_cast<uint32_t>(M >> 4) << 24) | (static_cast<uint32_t>(sf_id) << 29);
+}
+
+// shared-memory descriptor of a non-swizzled K-major operand whose 8-row core
+// matrices (8 x 16 bytes) lie 128 bytes apart: a 512-byte SF atom = 32 rows x 16 B
+__device__ __forceinline__ uint64_t smem_desc_sf_atom(uint32_t smem_addr) {
+  return static_cast<uint64_t>((smem_addr >> 4) & 0x3FFF) | (static_cast<uint64_t>(128 >> 4) << 32) | (1ull << 46);
+}
+
+// copy one SF atom (32 lanes x 128 bits) from shared memory into TMEM columns
+// [taddr, taddr + 4), replicated to the four lane quarters
+__device__ __forceinline__ void tmem_cp_sf_atom(uint32_t taddr, uint64_t sdesc) {
+  asm volatile("tcgen05.cp.cta_group::1.32x128b.warpx4 [%0], %1;" ::"r"(taddr), "l"(sdesc) : "memory");
 }
 
 // arrive on `bar` once every tcgen05.mma issued so far by this thread is done
@@ -397,6 +441,21 @@ __device__ __forceinline__ float pow2_recip(float p) {
 // per-(row,128) activation scale: pow2 ceiling of max(amax, 1e-10) * (1/448) in fp32
 __device__ __forceinline__ float act_scale_from_amax(float amax) {
   return pow2_ceil(__fmul_rn(fmaxf(amax, 1e-10f), 1.0f / 448.0f));
+}
+
+// E8M0 byte of a power-of-two float (its biased exponent; normal range only)
+__device__ __forceinline__ uint8_t e8m0_of_pow2(float s) {
+  return static_cast<uint8_t>((__float_as_uint(s) >> 23) & 0xFFu);
+}
+
+// Byte offset of the E8M0 scale of element (n, k) of an [N, K] matrix in the
+// MXFP8 SF-atom layout: one 512-byte atom per 128 rows x 128 columns, atoms
+// K-block-fastest; inside an atom row n sits at (n % 32) * 16 + ((n % 128) / 32) * 4
+// and the 32-column group at + (k % 128) / 32.  For a batch of [N, K]
+// matrices pass n = batch * N + row (N is a multiple of 128).
+__device__ __forceinline__ size_t sf_atom_offset(long long n, int k, int K) {
+  return (static_cast<size_t>(n >> 7) * static_cast<size_t>(K >> 7) + static_cast<size_t>(k >> 7)) * 512 +
+         static_cast<size_t>(n & 31) * 16 + static_cast<size_t>((n & 127) >> 5) * 4 + static_cast<size_t>((k & 127) >> 5);
 }
 
 // two floats -> two E4M3 codes (round to nearest even, saturating); lo in the low byte

@@ -37,14 +37,19 @@ __device__ __forceinline__ uint4 pack8(const float (&f)[8]) {
 // num_tokens_post_padded; padding rows are not written.  FP8: per (row, 128 columns) the power-of-two
 // scale of the vLLM PR #64760 analysis §1.2 rule, codes into a1 [cap, H],
 // scales into a1_scale_t [H/128, cap] (K-block major for the GEMM epilogue).
-// A block walks rows; a thread owns 8 consecutive columns, 16 threads one
-// 128-column group.
+// MXFP8 ("Hosting von Qwen auf Blackwell", "Quantisierung"): the same rule
+// per (row, 32 columns), E8M0 scale bytes into the SF-atom layout the
+// block-scaled MMA reads.  A block walks rows; a thread owns 8 consecutive
+// columns, 16 threads one 128-column group (4 threads one 32-column group).
 // ----------------------------------------------------------------------------
-template <bool FP8>
+// quantisation of the gathered rows
+enum GatherQ { kGatherBf16 = 0, kGatherFp8 = 1, kGatherMx = 2 };
+
+template <int Q>
 __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* x, int H, int topk,
                                                      int nflat, const int32_t* sorted_ids,
                                                      const int32_t* ntpp_ptr, int capacity,
-                                                     void* a1, float* a1_scale_t) {
+                                                     void* a1, void* a1_scale) {
   pdl_launch_dependents();
   pdl_wait();
   const int ntpp = *ntpp_ptr;
@@ -61,7 +66,7 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* x, int
       const bool in = v < vecs;
       uint4 u = make_uint4(0, 0, 0, 0);
       if (in) u = (*(reinterpret_cast<const uint4*>(src) + v));
-      if constexpr (!FP8) {
+      if constexpr (Q == kGatherBf16) {
         if (in) reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a1) + static_cast<size_t>(row) * H)[v] = u;
       } else {
         float f[8];
@@ -69,8 +74,10 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* x, int
         float amax = 0.f;
 #pragma unroll
         for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+        // group of 128 columns = 16 threads (FP8), of 32 columns = 4 threads (MXFP8)
 #pragma unroll
-        for (int off = 8; off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+        for (int off = (Q == kGatherFp8 ? 8 : 2); off > 0; off >>= 1)
+          amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
         const float scale = act_scale_from_amax(amax);
         const float inv = pow2_recip(scale);
         uint2 q;
@@ -80,7 +87,11 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* x, int
               (static_cast<uint32_t>(f32x2_to_e4m3x2(f[6] * inv, f[7] * inv)) << 16);
         if (in) {
           reinterpret_cast<uint2*>(static_cast<uint8_t*>(a1) + static_cast<size_t>(row) * H)[v] = q;
-          if ((v & 15) == 0) a1_scale_t[static_cast<size_t>(v >> 4) * capacity + row] = scale;
+          if constexpr (Q == kGatherFp8) {
+            if ((v & 15) == 0) static_cast<float*>(a1_scale)[static_cast<size_t>(v >> 4) * capacity + row] = scale;
+          } else {
+            if ((v & 3) == 0) static_cast<uint8_t*>(a1_scale)[sf_atom_offset(row, v * 8, H)] = e8m0_of_pow2(scale);
+          }
         }
       }
     }
@@ -88,16 +99,19 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* x, int
 }
 
 cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32_t* sorted_ids,
-                          const int32_t* ntpp, int capacity, bool fp8, void* a1, float* a1_scale_t,
+                          const int32_t* ntpp, int capacity, bool fp8, bool mx, void* a1, void* a1_scale,
                           cudaStream_t stream) {
   if (capacity == 0) return cudaSuccess;
   int blocks = capacity < 148 * 8 ? capacity : 148 * 8;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (mx)
+    return launch_pdl(gather_kernel<kGatherMx>, blocks, 256, 0, stream, xb, H, topk, nflat, sorted_ids, ntpp,
+                      capacity, a1, a1_scale);
   if (fp8)
-    return launch_pdl(gather_kernel<true>, blocks, 256, 0, stream, xb, H, topk, nflat, sorted_ids, ntpp, capacity, a1,
-                      a1_scale_t);
-  return launch_pdl(gather_kernel<false>, blocks, 256, 0, stream, xb, H, topk, nflat, sorted_ids, ntpp, capacity, a1,
-                    a1_scale_t);
+    return launch_pdl(gather_kernel<kGatherFp8>, blocks, 256, 0, stream, xb, H, topk, nflat, sorted_ids, ntpp,
+                      capacity, a1, a1_scale);
+  return launch_pdl(gather_kernel<kGatherBf16>, blocks, 256, 0, stream, xb, H, topk, nflat, sorted_ids, ntpp,
+                    capacity, a1, a1_scale);
 }
 
 // ----------------------------------------------------------------------------
@@ -199,6 +213,67 @@ cudaError_t launch_quantize_weights(const void* w, long long batches, int rows, 
   if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
   return launch_pdl(quantize_weights_kernel, static_cast<unsigned>(blocks), 256, 0, stream,
                     static_cast<const __nv_bfloat16*>(w), rows, cols, codes, scales);
+}
+
+// ----------------------------------------------------------------------------
+// MXFP8 weight quantisation: one CTA per 128x128 block, thread = (row, 64
+// columns) = two 32-column groups.  scale = pow2 ceiling of fp32(max(amax,
+// 1e-10)) * fp32(1/448); code = e4m3(w * 2^-e) (exact scaling, RNE,
+// saturating); the E8M0 bytes go to the SF-atom layout.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) quantize_weights_mx_kernel(const __nv_bfloat16* w, int rows, int cols,
+                                                                  uint8_t* codes, uint8_t* sf) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int nbc = cols / 128, nbr = rows / 128;
+  const long long blk = blockIdx.x;
+  const long long b = blk / (static_cast<long long>(nbr) * nbc);
+  const int rem = static_cast<int>(blk - b * nbr * nbc);
+  const int br = rem / nbc, bc = rem - br * nbc;
+  const int r = threadIdx.x >> 1, half = threadIdx.x & 1;
+  const long long grow = b * rows + static_cast<long long>(br) * 128 + r;  // row in the batch of matrices
+  const int col0 = bc * 128 + half * 64;
+  const size_t row_off = static_cast<size_t>(grow) * cols + col0;
+  const uint4* src = reinterpret_cast<const uint4*>(w + row_off);
+  uint4* dst = reinterpret_cast<uint4*>(codes + row_off);
+  uint8_t e8[2];
+#pragma unroll
+  for (int grp = 0; grp < 2; ++grp) {
+    float f[32];
+    float amax = 0.f;
+#pragma unroll
+    for (int i = 0; i < 4; ++i) {
+      float t[8];
+      unpack8((*(src + 4 * grp + i)), t);
+#pragma unroll
+      for (int k = 0; k < 8; ++k) {
+        f[8 * i + k] = t[k];
+        amax = fmaxf(amax, fabsf(t[k]));
+      }
+    }
+    const float scale = act_scale_from_amax(amax);
+    const float inv = pow2_recip(scale);
+    uint32_t wds[8];
+#pragma unroll
+    for (int i = 0; i < 8; ++i)
+      wds[i] = static_cast<uint32_t>(f32x2_to_e4m3x2(f[4 * i] * inv, f[4 * i + 1] * inv)) |
+               (static_cast<uint32_t>(f32x2_to_e4m3x2(f[4 * i + 2] * inv, f[4 * i + 3] * inv)) << 16);
+    dst[2 * grp] = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+    dst[2 * grp + 1] = make_uint4(wds[4], wds[5], wds[6], wds[7]);
+    e8[grp] = e8m0_of_pow2(scale);
+  }
+  // the thread's two groups are adjacent bytes of one SF-atom row
+  *reinterpret_cast<uint16_t*>(sf + sf_atom_offset(grow, col0, cols)) =
+      static_cast<uint16_t>(e8[0] | (static_cast<uint16_t>(e8[1]) << 8));
+}
+
+cudaError_t launch_quantize_weights_mx(const void* w, long long batches, int rows, int cols, uint8_t* codes,
+                                       uint8_t* sf, cudaStream_t stream) {
+  const long long blocks = batches * (rows / 128) * (cols / 128);
+  if (blocks == 0) return cudaSuccess;
+  if (blocks > 0x7fffffffLL) return cudaErrorInvalidValue;
+  return launch_pdl(quantize_weights_mx_kernel, static_cast<unsigned>(blocks), 256, 0, stream,
+                    static_cast<const __nv_bfloat16*>(w), rows, cols, codes, sf);
 }
 
 }  // namespace moe

@@ -86,6 +86,9 @@ struct Args {
   int* status;
   float* partials;         // swap-AB split-K: [unit][acc column][128] fp32 partial sums
   int splits;              // swap-AB split-K factor S (1: no split); chosen on the host
+  const uint8_t* a_sf;     // MXFP8: E8M0 SF atoms of the activation rows [capacity, K]
+  const uint8_t* w_sf;     // MXFP8: E8M0 SF atoms of the weights [E * Nw, K]
+  uint8_t* out_sf;         // MXFP8 GEMM1: SF atoms of a2 [capacity, I]
 };
 
 // Split-K for the swap-AB tiles: when at most half the SMs would have a tile
@@ -779,6 +782,286 @@ __global__ void __launch_bounds__(128) splitk_reduce_kernel(Args args) {
 }
 
 // ----------------------------------------------------------------------------
+// MXFP8 normal tiles ("Hosting von Qwen auf Blackwell", "Quantisierung":
+// micro-scaling is what Blackwell's tensor cores consume natively).
+//
+// tcgen05.mma kind::mxf8f6f4.block_scale: the E8M0 scale of every 32-element K
+// block is applied inside the MMA, so the accumulator stays in TMEM for the
+// whole K loop -- no per-K-block promotion.  Per K block the producer loads
+// the 128 x 128 token tile, the 256 x 128 weight tile (two 128-row boxes for
+// GEMM1: gate and up) and three 512-byte SF atoms (tokens; two weight row
+// blocks); the MMA thread copies the atoms into TMEM (tcgen05.cp 32x128b,
+// replicated to the four lane quarters; 16 columns per stage) and issues four
+// K=32 MMAs whose scale-factor byte id walks the atom's four K blocks.
+// TMEM: one 256-column accumulator + 4 x 16 SF columns.  The epilogue reads
+// its whole share of the accumulator into registers, releases TMEM at once
+// (the next tile's MMAs start) and then runs SiLU*up + MX requantisation
+// (GEMM1) or the routed weight + scatter (GEMM2).
+// ----------------------------------------------------------------------------
+template <bool kDown>
+struct CfgMx {
+  static constexpr int kTokBytes = 128 * 128;
+  static constexpr int kWBytes = 256 * 128;
+  static constexpr int kSfOffset = kTokBytes + kWBytes;  // three 512-byte atoms
+  static constexpr int kStageBytes = 51200;              // 48 KB + 1.5 KB, kept 1024-aligned
+  static constexpr int kStages = 4;
+  static constexpr int kAccCols = 256;
+  static constexpr int kSfCol0 = 256;                    // stage s: columns kSfCol0 + 16 s + [0, 12)
+  static constexpr int kTmemCols = 512;
+  static constexpr int kTileN = kDown ? 256 : 128;       // output columns per tile
+  static constexpr size_t kSmemBytes = static_cast<size_t>(kStages) * kStageBytes + kSmemReserve + 1024;
+  static_assert(kSfOffset + 3 * 512 <= kStageBytes, "stage layout");
+  static_assert(kSmemBytes <= static_cast<size_t>(kSmemLimit), "shared memory");
+};
+
+template <bool kDown>
+__global__ void __launch_bounds__(kThreads, 1)
+    moe_gemm_mx_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant__ CUtensorMap tm_w,
+                       const Args args) {
+  using C = CfgMx<kDown>;
+  extern __shared__ uint8_t smem_raw[];
+  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
+  uint8_t* reserve = smem + static_cast<size_t>(C::kStages) * C::kStageBytes;
+  uint64_t* full = reinterpret_cast<uint64_t*>(reserve);
+  uint64_t* empty = full + C::kStages;
+  uint64_t* acc_full = empty + C::kStages;
+  uint64_t* acc_empty = acc_full + 1;
+  uint64_t* drain = acc_empty + 1;
+  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
+  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
+
+  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
+  pdl_launch_dependents();
+  if (threadIdx.x == 0) {
+    for (int s = 0; s < C::kStages; ++s) {
+      mbar_init(&full[s], 1);
+      mbar_init(&empty[s], 1);
+    }
+    mbar_init(acc_full, 1);
+    mbar_init(acc_empty, kEpiWarps);
+    mbar_init(drain, 1);
+    *abort_flag = 0;
+    fence_mbar_init();
+  }
+  if (warp == 0 && lane == 0) {
+    tma_prefetch_desc(&tm_tok);
+    tma_prefetch_desc(&tm_w);
+  }
+  if (warp == 1) {
+    tmem_alloc(tmem_slot, C::kTmemCols);
+    tmem_relinquish();
+  }
+  tc_fence_before();
+  __syncthreads();
+  tc_fence_after();
+  const uint32_t tmem_base = *tmem_slot;
+  pdl_wait();
+
+  const int H = args.H, I = args.I;
+  const int K = kDown ? I : H;
+  const int kb_n = K / 128;
+  const int n_tiles = (kDown ? H : I) / C::kTileN;
+  const int num_tiles = ((*(args.ntpp)) / 128) * n_tiles;
+
+  if (warp == 0) {
+    // ------------------------------------------------------------------ producer
+    if (lane == 0) {
+      const uint64_t pol_w = policy_evict_first();
+      const uint64_t pol_a = policy_evict_last();
+      int stage = 0;
+      uint32_t phase = 0;
+      long long fills = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
+        const int e = (*(args.expert_ids + mb));
+        // weight rows of the two 128-row blocks of this tile (global row index in [E * Nw, K])
+        int w_row0, w_row1;
+        if constexpr (kDown) {
+          w_row0 = e * H + nt * 256;
+          w_row1 = w_row0 + 128;
+        } else {
+          w_row0 = e * 2 * I + nt * 128;  // gate rows
+          w_row1 = w_row0 + I;            // up rows
+        }
+        const uint8_t* sfa = args.a_sf + static_cast<size_t>(mb) * kb_n * 512;
+        const uint8_t* sfb0 = args.w_sf + static_cast<size_t>(w_row0 / 128) * kb_n * 512;
+        const uint8_t* sfb1 = args.w_sf + static_cast<size_t>(w_row1 / 128) * kb_n * 512;
+        for (int kb = 0; kb < kb_n; ++kb) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status,
+                         MOE_STATUS_WAIT_TIMEOUT | kWhereProducer)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + static_cast<size_t>(stage) * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], C::kTokBytes + C::kWBytes + 3 * 512);
+          const int kx = kb * 128;
+          tma_load_2d(st, &tm_tok, &full[stage], kx, mb * 128, pol_a);
+          if constexpr (kDown) {
+            tma_load_2d(st + C::kTokBytes, &tm_w, &full[stage], kx, w_row0, pol_w);
+          } else {
+            tma_load_2d(st + C::kTokBytes, &tm_w, &full[stage], kx, w_row0, pol_w);
+            tma_load_2d(st + C::kTokBytes + 16384, &tm_w, &full[stage], kx, w_row1, pol_w);
+          }
+          bulk_load(st + C::kSfOffset, sfa + static_cast<size_t>(kb) * 512, 512, &full[stage]);
+          bulk_load(st + C::kSfOffset + 512, sfb0 + static_cast<size_t>(kb) * 512, 512, &full[stage]);
+          bulk_load(st + C::kSfOffset + 1024, sfb1 + static_cast<size_t>(kb) * 512, 512, &full[stage]);
+          ++fills;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+      }
+      if (!ok) {
+        // let every copy already issued land before the CTA tears down
+        for (int s = 0; s < C::kStages; ++s) {
+          const long long n_s = fills / C::kStages + (s < fills % C::kStages ? 1 : 0);
+          if (n_s > 0) {
+            const uint64_t t0 = globaltimer_ns();
+            while (!mbar_try_wait(&full[s], static_cast<uint32_t>((n_s - 1) & 1)) &&
+                   globaltimer_ns() - t0 < kWaitTimeoutNs) {
+            }
+          }
+        }
+      }
+    }
+  } else if (warp == 1) {
+    // ------------------------------------------------------------------ MMA issuer
+    if (lane == 0) {
+      int stage = 0;
+      uint32_t phase = 0, aphase = 0;
+      bool ok = true;
+      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+        if (!mbar_wait(acc_empty, aphase ^ 1u, abort_flag, args.status, MOE_STATUS_WAIT_TIMEOUT | kWhereMma)) {
+          ok = false;
+          break;
+        }
+        tc_fence_after();
+        for (int kb = 0; kb < kb_n; ++kb) {
+          if (!mbar_wait(&full[stage], phase, abort_flag, args.status, MOE_STATUS_WAIT_TIMEOUT | kWhereMma)) {
+            ok = false;
+            break;
+          }
+          tc_fence_after();
+          const uint32_t st = smem_u32(smem + static_cast<size_t>(stage) * C::kStageBytes);
+          const uint32_t sf_t = tmem_base + static_cast<uint32_t>(C::kSfCol0 + 16 * stage);
+          tmem_cp_sf_atom(sf_t, smem_desc_sf_atom(st + C::kSfOffset));
+          tmem_cp_sf_atom(sf_t + 4, smem_desc_sf_atom(st + C::kSfOffset + 512));
+          tmem_cp_sf_atom(sf_t + 8, smem_desc_sf_atom(st + C::kSfOffset + 1024));
+#pragma unroll
+          for (int k = 0; k < 4; ++k) {
+            const uint32_t koff = k * 32;  // 32 E4M3 elements
+            const uint32_t sel = static_cast<uint32_t>(k) << 30;
+            mma_mxf8(tmem_base, smem_desc_sw128(st + koff), smem_desc_sw128(st + C::kTokBytes + koff),
+                     make_idesc_mx(128, 256, k), (kb > 0 || k > 0) ? 1u : 0u, sf_t | sel, (sf_t + 4) | sel);
+          }
+          mma_commit(&empty[stage]);
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) break;
+        mma_commit(acc_full);
+        aphase ^= 1u;
+      }
+      mma_commit(drain);
+      const uint64_t t0 = globaltimer_ns();
+      while (!mbar_try_wait(drain, 0)) {
+        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
+          report_status(args.status, MOE_STATUS_WAIT_TIMEOUT | kWhereDrain);
+          break;
+        }
+      }
+    }
+  } else {
+    // ------------------------------------------------------------------ epilogue
+    const int q = warp & 3;
+    const int g = (warp - 2) >> 2;
+    const int row = 32 * q + lane;
+    const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
+    uint32_t aphase = 0;
+    for (int tile = blockIdx.x; tile < num_tiles; tile += gridDim.x) {
+      const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
+      const int grow = mb * 128 + row;
+      if (!warp_wait(acc_full, aphase, abort_flag, args.status, kWhereEpiAcc)) break;
+      aphase ^= 1u;
+      tc_fence_after();
+      float v[128];  // GEMM1: gate [0, 64) and up [64, 128) of this group; GEMM2: 128 output columns
+      const uint32_t t0 = tmem_base + lane_addr;
+#pragma unroll
+      for (int c = 0; c < 4; ++c) {
+        float a[16], b[16];
+        tmem_ld16(t0 + (kDown ? g * 128 + 16 * c : g * 64 + 16 * c), a);
+        tmem_ld16(t0 + (kDown ? g * 128 + 64 + 16 * c : 128 + g * 64 + 16 * c), b);
+#pragma unroll
+        for (int i = 0; i < 16; ++i) {
+          v[16 * c + i] = a[i];
+          v[64 + 16 * c + i] = b[i];
+        }
+      }
+      tmem_wait_ld();
+      tc_fence_before();
+      __syncwarp();
+      if (lane == 0) mbar_arrive(acc_empty);  // the next tile's MMAs may overwrite the accumulator now
+      if constexpr (!kDown) {
+        // SiLU(gate) * up (bf16 rounding points as the oracle), MX requant per 32 columns
+        const int col0 = nt * 128 + g * 64;
+        uint8_t* dst = static_cast<uint8_t*>(args.out) + static_cast<size_t>(grow) * I + col0;
+        uint8_t e8[2];
+#pragma unroll
+        for (int grp = 0; grp < 2; ++grp) {
+          float p[32];
+          float amax = 0.f;
+#pragma unroll
+          for (int i = 0; i < 32; ++i) {
+            p[i] = silu_mul_bf16(bf16_round(v[32 * grp + i]), bf16_round(v[64 + 32 * grp + i]));
+            amax = fmaxf(amax, fabsf(p[i]));
+          }
+          const float scale = act_scale_from_amax(amax);
+          const float inv = pow2_recip(scale);
+          uint32_t wds[8];
+#pragma unroll
+          for (int i = 0; i < 8; ++i)
+            wds[i] = static_cast<uint32_t>(f32x2_to_e4m3x2(p[4 * i] * inv, p[4 * i + 1] * inv)) |
+                     (static_cast<uint32_t>(f32x2_to_e4m3x2(p[4 * i + 2] * inv, p[4 * i + 3] * inv)) << 16);
+          uint4* d4 = reinterpret_cast<uint4*>(dst + 32 * grp);
+          d4[0] = make_uint4(wds[0], wds[1], wds[2], wds[3]);
+          d4[1] = make_uint4(wds[4], wds[5], wds[6], wds[7]);
+          e8[grp] = e8m0_of_pow2(scale);
+        }
+        *reinterpret_cast<uint16_t*>(args.out_sf + sf_atom_offset(grow, col0, I)) =
+            static_cast<uint16_t>(e8[0] | (static_cast<uint16_t>(e8[1]) << 8));
+      } else {
+        // routed weight, scatter the row to y[flat]
+        const int flat = (*(args.sorted_ids + grow));
+        if (flat < args.nflat) {
+          const float wt = (*(args.topk_weights + flat));
+          __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(flat) * H + nt * 256 +
+                                g * 128;
+#pragma unroll
+          for (int c = 0; c < 8; ++c) {
+            float o[16];
+#pragma unroll
+            for (int i = 0; i < 16; ++i) o[i] = v[16 * c + i] * wt;
+            store_bf16x16(yrow + 16 * c, o);
+          }
+        }
+      }
+    }
+  }
+
+  __syncwarp();
+  tc_fence_before();
+  __syncthreads();
+  if (warp == 1) {
+    tc_fence_after();
+    tmem_dealloc(tmem_base, C::kTmemCols);
+  }
+}
+
+// ----------------------------------------------------------------------------
 // Normal orientation, FP8, two SMs per tile (tcgen05 cta_group::2).
 //
 // A cluster of two CTAs computes a 256 x 256 tile: CTA r holds token rows
@@ -1221,8 +1504,35 @@ cudaError_t launch_fp8_pair(const GemmProblem& p, const void* tok, const void* w
   return cudaLaunchKernelEx(&cfg, kern, tm_tok, tm_w, args);
 }
 
+template <bool kDown>
+cudaError_t launch_mx(const GemmProblem& p, const void* tok, const void* w, const Args& args, cudaStream_t s) {
+  using C = CfgMx<kDown>;
+  auto kern = moe_gemm_mx_kernel<kDown>;
+  static bool attr_set = false;
+  if (!attr_set) {
+    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
+                                         static_cast<int>(C::kSmemBytes));
+    if (e != cudaSuccess) return e;
+    attr_set = true;
+  }
+  const long long K = kDown ? p.I : p.H;
+  const long long wrows = kDown ? static_cast<long long>(p.E) * p.H : static_cast<long long>(p.E) * 2 * p.I;
+  CUtensorMap tm_tok, tm_w;
+  if (!make_map(&tm_tok, tok, p.capacity, K, 1, 128)) return cudaErrorInvalidValue;
+  if (!make_map(&tm_w, w, wrows, K, 1, kDown ? 256 : 128)) return cudaErrorInvalidValue;
+  const int n_tiles = (kDown ? p.H : p.I) / C::kTileN;
+  const long long max_tiles = static_cast<long long>(p.capacity / 128) * n_tiles;
+  int grid = p.num_sms;
+  if (max_tiles < grid) grid = static_cast<int>(max_tiles);
+  if (grid <= 0) return cudaSuccess;
+  return launch_pdl(kern, grid, kThreads, C::kSmemBytes, s, tm_tok, tm_w, args);
+}
+
 template <bool kDown, bool kFP8>
 cudaError_t dispatch(const GemmProblem& p, const void* tok, const void* w, const Args& args, cudaStream_t s) {
+  if constexpr (kFP8) {
+    if (p.mx) return launch_mx<kDown>(p, tok, w, args, s);
+  }
   if (!p.swap) {
     if constexpr (kFP8) {
       if (p.block_m == 256) return launch_fp8_pair<kDown>(p, tok, w, args, s);
@@ -1244,8 +1554,8 @@ size_t smem_of() {
 
 }  // namespace
 
-cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const float* a1_scale_t, const void* w13,
-                         const float* w13_scale, void* a2, float* a2_scale_t, cudaStream_t stream) {
+cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const void* a1_scale, const void* w13,
+                         const void* w13_scale, void* a2, void* a2_scale, cudaStream_t stream) {
   Args args{};
   args.E = p.E;
   args.H = p.H;
@@ -1256,18 +1566,24 @@ cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const float* a1_s
   args.expert_ids = p.expert_ids;
   args.sorted_ids = p.sorted_ids;
   args.topk_weights = p.topk_weights;
-  args.a_scale_t = a1_scale_t;
-  args.w_scale = w13_scale;
+  if (p.mx) {
+    args.a_sf = static_cast<const uint8_t*>(a1_scale);
+    args.w_sf = static_cast<const uint8_t*>(w13_scale);
+    args.out_sf = static_cast<uint8_t*>(a2_scale);
+  } else {
+    args.a_scale_t = static_cast<const float*>(a1_scale);
+    args.w_scale = static_cast<const float*>(w13_scale);
+    args.out_scale_t = static_cast<float*>(a2_scale);
+  }
   args.out = a2;
-  args.out_scale_t = a2_scale_t;
   args.status = p.status;
   args.partials = p.partials;
   args.splits = 1;
   return p.fp8 ? dispatch<false, true>(p, a1, w13, args, stream) : dispatch<false, false>(p, a1, w13, args, stream);
 }
 
-cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const float* a2_scale_t, const void* w2,
-                         const float* w2_scale, void* y, cudaStream_t stream) {
+cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const void* a2_scale, const void* w2,
+                         const void* w2_scale, void* y, cudaStream_t stream) {
   Args args{};
   args.E = p.E;
   args.H = p.H;
@@ -1278,8 +1594,13 @@ cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const float* a2_s
   args.expert_ids = p.expert_ids;
   args.sorted_ids = p.sorted_ids;
   args.topk_weights = p.topk_weights;
-  args.a_scale_t = a2_scale_t;
-  args.w_scale = w2_scale;
+  if (p.mx) {
+    args.a_sf = static_cast<const uint8_t*>(a2_scale);
+    args.w_sf = static_cast<const uint8_t*>(w2_scale);
+  } else {
+    args.a_scale_t = static_cast<const float*>(a2_scale);
+    args.w_scale = static_cast<const float*>(w2_scale);
+  }
   args.out = y;
   args.out_scale_t = nullptr;
   args.status = p.status;

@@ -48,9 +48,11 @@ cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in,
                                      int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp, int32_t* counts,
                                      int32_t* offsets, int* status, cudaStream_t stream);
 
-// gather x rows into sorted order (bf16 copy, or FP8 per-(row,128) quantisation)
+// gather x rows into sorted order: bf16 copy, FP8 per-(row,128) quantisation
+// (a1_scale: fp32 [H/128, capacity]) or MXFP8 per-(row,32) quantisation
+// (a1_scale: E8M0 SF atoms of [capacity, H])
 cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32_t* sorted_ids,
-                          const int32_t* ntpp, int capacity, bool fp8, void* a1, float* a1_scale_t,
+                          const int32_t* ntpp, int capacity, bool fp8, bool mx, void* a1, void* a1_scale,
                           cudaStream_t stream);
 
 // out[t] = sum_j y[t*topk + j]
@@ -60,10 +62,15 @@ cudaError_t launch_combine(const void* y, int T, int topk, int H, void* out, cud
 cudaError_t launch_quantize_weights(const void* w, long long batches, int rows, int cols, uint8_t* codes,
                                     float* scales, cudaStream_t stream);
 
+// MXFP8 weight quantisation: per (row, 32 columns) E8M0 scale, SF-atom layout
+cudaError_t launch_quantize_weights_mx(const void* w, long long batches, int rows, int cols, uint8_t* codes,
+                                       uint8_t* sf, cudaStream_t stream);
+
 // grouped GEMMs ----------------------------------------------------------------
 struct GemmProblem {
   int E, H, I, topk, nflat, block_m, capacity;
   bool fp8, swap;
+  bool mx;             // MXFP8 (with fp8): block-scaled MMA, E8M0 SF atoms
   const int32_t* ntpp;
   const int32_t* expert_ids;
   const int32_t* sorted_ids;
@@ -80,13 +87,15 @@ constexpr int kMaxSplitUnits = 320;  // >= 4 splits x (148 SMs / 2) tiles
 // GEMM1 + fused SiLU*up (+ FP8 requant): a1 [cap, H] -> a2 [cap, I] (+ a2_scale_t [I/128, cap]).
 // In swap-AB mode with split-K allowed this launches the GEMM and then the
 // split-K reduce kernel (which exits at once when the GEMM did not split).
-cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const float* a1_scale_t, const void* w13,
-                         const float* w13_scale, void* a2, float* a2_scale_t, cudaStream_t stream);
+// Scale arguments: FP8 -- fp32 (activation scales K-block major, weight scales
+// per 128x128 block); MXFP8 -- E8M0 SF atoms.
+cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const void* a1_scale, const void* w13,
+                         const void* w13_scale, void* a2, void* a2_scale, cudaStream_t stream);
 
 // GEMM2 + routed weight: a2 [cap, I] -> y [nflat, H] bf16 (rows scattered by sorted_ids);
 // swap-AB split-K launches the reduce kernel after it, as for GEMM1
-cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const float* a2_scale_t, const void* w2,
-                         const float* w2_scale, void* y, cudaStream_t stream);
+cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const void* a2_scale, const void* w2,
+                         const void* w2_scale, void* y, cudaStream_t stream);
 
 // failure-detection self-test: one bounded wait that must time out
 cudaError_t launch_wait_selftest(int* status, unsigned long long timeout_ns, unsigned long long* waited_ns,

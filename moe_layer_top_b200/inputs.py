@@ -29,13 +29,14 @@ class MoEConfig:
     topk: int
     H: int
     I: int
-    fp8: bool
+    fp8: bool             # 8-bit E4M3 weights (with mx: MXFP8 scales, else 128x128 fp32 block scales)
     routing: str          # "logits" | "biased_logits" | "uniform_ids" | "zipf"
     tokens: tuple         # the batch sizes T of the family
     zipf_s: float = 1.2
     bias_std: float = 0.5
     w_std: float = 0.02
     x_scale: float = 0.1
+    mx: bool = False
 
 
 CONFIGS = {
@@ -51,6 +52,11 @@ CONFIGS = {
     # prefill: 16384 tokens, logits plus a per-expert bias for moderate imbalance
     "prefill_fp8": MoEConfig("prefill_fp8", E=128, topk=8, H=4096, I=1536, fp8=True,
                              routing="biased_logits", tokens=(16384,)),
+    # the prefill and decode layers with MXFP8 weights (E4M3, one E8M0 scale per 32 elements)
+    "prefill_mxfp8": MoEConfig("prefill_mxfp8", E=128, topk=8, H=4096, I=1536, fp8=True,
+                               routing="biased_logits", tokens=(16384,), mx=True),
+    "decode_mxfp8": MoEConfig("decode_mxfp8", E=128, topk=8, H=4096, I=1536, fp8=True,
+                              routing="logits", tokens=(1, 4, 16, 64), mx=True),
     # large experts with Zipf(1.2)-skewed choice without replacement
     "skewed_fp8": MoEConfig("skewed_fp8", E=256, topk=8, H=7168, I=2048, fp8=True,
                             routing="zipf", tokens=(1, 32, 512, 8192)),

@@ -30,6 +30,7 @@ MOE_STATUS_WAIT_TIMEOUT = 0x100
 
 DTYPE_BF16 = 0
 DTYPE_FP8_E4M3 = 1
+DTYPE_MXFP8_E4M3 = 2
 
 MODE_AUTO = 0
 MODE_NORMAL = 1
@@ -43,7 +44,7 @@ EXPORTED = (
     "moe_last_error_string", "moe_route", "moe_align_capacity", "moe_align_workspace_size", "moe_align",
     "moe_quantize_weights_fp8", "moe_resolve_problem", "moe_workspace_size", "moe_get_workspace_layout",
     "moe_fused_forward", "moe_forward_stages", "moe_read_status", "moe_version", "moe_align_noalloc",
-    "moe_selftest_wait_timeout",
+    "moe_selftest_wait_timeout", "moe_quantize_weights_mxfp8",
 )
 
 
@@ -94,6 +95,7 @@ def lib():
             "moe_align": (ctypes.c_int, [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp, sz, vp]),
             "moe_align_noalloc": (ctypes.c_int, [vp, i32, i32, i32, i32, vp, vp, vp, vp, vp, vp]),
             "moe_quantize_weights_fp8": (ctypes.c_int, [vp, i64, i32, i32, vp, vp, vp]),
+            "moe_quantize_weights_mxfp8": (ctypes.c_int, [vp, i64, i32, i32, vp, vp, vp]),
             "moe_resolve_problem": (ctypes.c_int, [P]),
             "moe_workspace_size": (sz, [P]),
             "moe_get_workspace_layout": (ctypes.c_int, [P, ctypes.POINTER(MoeWorkspaceLayout)]),
@@ -130,10 +132,13 @@ def _stream(stream=None):
     return ctypes.c_void_p(s.cuda_stream)
 
 
-def problem(T, E, topk, H, I, fp8=False, mode=MODE_AUTO, block_m=0, renormalize=True, split_k=True) -> MoeProblem:
+def problem(T, E, topk, H, I, fp8=False, mode=MODE_AUTO, block_m=0, renormalize=True, split_k=True,
+            mx=False) -> MoeProblem:
+    """A moe_problem; ``fp8`` selects E4M3 weights with 128x128 fp32 block scales, ``mx`` MXFP8
+    (E4M3 with per-32 E8M0 scales)."""
     p = MoeProblem()
     p.T, p.E, p.topk, p.H, p.I = int(T), int(E), int(topk), int(H), int(I)
-    p.weight_dtype = DTYPE_FP8_E4M3 if fp8 else DTYPE_BF16
+    p.weight_dtype = DTYPE_MXFP8_E4M3 if mx else (DTYPE_FP8_E4M3 if fp8 else DTYPE_BF16)
     p.mode, p.block_m, p.renormalize = int(mode), int(block_m), 1 if renormalize else 0
     p.split_k = 0 if split_k else 1
     return p
@@ -205,6 +210,28 @@ def quantize_weights_fp8(w: torch.Tensor, stream=None):
     return codes, scales
 
 
+def quantize_weights_mxfp8(w: torch.Tensor, stream=None):
+    """bf16 [..., rows, cols] -> (E4M3 codes uint8 [..., rows, cols], E8M0 scale factors uint8
+    [..., rows * cols / 32] in the SF-atom layout of the header)."""
+    w = w.contiguous()
+    *lead, rows, cols = w.shape
+    batches = 1
+    for d in lead:
+        batches *= d
+    codes = torch.empty(w.shape, dtype=torch.uint8, device=w.device)
+    sf = torch.empty((*lead, rows * cols // 32), dtype=torch.uint8, device=w.device)
+    _check(lib().moe_quantize_weights_mxfp8(_ptr(w), batches, rows, cols, _ptr(codes), _ptr(sf), _stream(stream)))
+    return codes, sf
+
+
+def sf_atoms_to_rows(sf_atoms: torch.Tensor, rows: int, cols: int) -> torch.Tensor:
+    """Re-index SF atoms of [.., rows, cols] into the natural [.., rows, cols/32] order (for tests and tools)."""
+    lead = sf_atoms.shape[:-1]
+    a = sf_atoms.reshape(*lead, rows // 128, cols // 128, 32, 4, 4)      # [rb, kb, n%32, (n%128)/32, k-group]
+    a = a.permute(*range(len(lead)), len(lead), len(lead) + 3, len(lead) + 2, len(lead) + 1, len(lead) + 4)
+    return a.reshape(*lead, rows, cols // 32)
+
+
 def _forward_args(p, x, logits, topk_ids, topk_weights, w13, w2, w13_scale, w2_scale, out, ws):
     return (ctypes.byref(p), _ptr(x), _ptr(logits), _ptr(topk_ids), _ptr(topk_weights), _ptr(w13), _ptr(w2),
             _ptr(w13_scale), _ptr(w2_scale), _ptr(out), _ptr(ws), ws.numel())
@@ -241,7 +268,8 @@ def workspace_views(p: MoeProblem, ws: torch.Tensor) -> dict:
     L = workspace_layout(q)
     nflat = q.T * q.topk
     cap = L.capacity
-    fp8 = q.weight_dtype == DTYPE_FP8_E4M3
+    mx = q.weight_dtype == DTYPE_MXFP8_E4M3
+    fp8 = q.weight_dtype == DTYPE_FP8_E4M3 or mx
 
     def view(off, n, dtype, shape):
         if off < 0:
@@ -259,9 +287,11 @@ def workspace_views(p: MoeProblem, ws: torch.Tensor) -> dict:
         "expert_counts": view(L.expert_counts, q.E, torch.int32, (q.E,)),
         "expert_offsets": view(L.expert_offsets, q.E + 1, torch.int32, (q.E + 1,)),
         "a1": view(L.a1, cap * q.H, torch.uint8 if fp8 else torch.bfloat16, (cap, q.H)),
-        "a1_scale_t": view(L.a1_scale, cap * (q.H // 128), torch.float32, (q.H // 128, cap)),
+        "a1_scale_t": None if mx else view(L.a1_scale, cap * (q.H // 128), torch.float32, (q.H // 128, cap)),
+        "a1_sf": view(L.a1_scale, cap * q.H // 32, torch.uint8, (cap * q.H // 32,)) if mx else None,
         "a2": view(L.a2, cap * q.I, torch.uint8 if fp8 else torch.bfloat16, (cap, q.I)),
-        "a2_scale_t": view(L.a2_scale, cap * (q.I // 128), torch.float32, (q.I // 128, cap)),
+        "a2_scale_t": None if mx else view(L.a2_scale, cap * (q.I // 128), torch.float32, (q.I // 128, cap)),
+        "a2_sf": view(L.a2_scale, cap * q.I // 32, torch.uint8, (cap * q.I // 32,)) if mx else None,
         "y": view(L.y, nflat * q.H, torch.bfloat16, (nflat, q.H)),
         "partials": view(L.partials, (L.total_bytes - L.partials) // 4, torch.float32, (-1,)),
         "layout": L,

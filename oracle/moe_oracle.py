@@ -391,7 +391,7 @@ def expert_mlp(x_hat, w13_hat, w2_hat, requant, return_intermediates: bool = Fal
 
 def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weights=None,
                 w13_scale=None, w2_scale=None, renormalize: bool = True, tokens=None,
-                return_y: bool = False):
+                return_y: bool = False, mx=None):
     """The fused MoE layer: route -> experts -> top-k weighted combine.
 
     [AWS] "Warum MoE-Kernel so wichtig sind": one operation that routes each
@@ -407,6 +407,7 @@ def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weigh
     Routing: ``logits`` [T, E] float32, or ``topk_ids``/``topk_weights``.
     tokens: optional subset of token indices to evaluate (each output row
     depends only on its own token, its routing and the weights).
+    mx: MXFP8 scales (taken from the scale dtype, uint8, when not given).
 
     Returns a dict with ``out`` [len(tokens), H] (float64 holding bf16
     values), ``topk_ids``, ``topk_weights`` and, when asked, ``y``
@@ -416,7 +417,7 @@ def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weigh
     fp8 = w13_scale is not None
     if fp8 != (w2_scale is not None):
         raise ValueError("w13_scale and w2_scale go together")
-    mx = fp8 and np.asarray(w13_scale).dtype == np.uint8
+    mx = fp8 and (bool(mx) if mx is not None else np.asarray(w13_scale).dtype == np.uint8)
     if logits is not None:
         topk_ids, topk_weights = route(logits, topk, renormalize)
     topk_ids = np.asarray(topk_ids).astype(np.int64)

@@ -18,18 +18,22 @@ TOL_MAX_REL = 0.05
 
 class LazyExperts:
     """Per-expert host copies of the generator's bf16 weights, and the
-    oracle's own FP8 block quantisation of them, made on first access."""
+    oracle's own FP8 (block-128 or MX) quantisation of them, made on first access."""
 
-    def __init__(self, w_dev: torch.Tensor, fp8: bool):
+    def __init__(self, w_dev: torch.Tensor, fp8: bool, mx: bool = False):
         self.w_dev = w_dev
         self.fp8 = fp8
+        self.mx = mx
         self._cache = {}
 
     def _get(self, e):
         e = int(e)
         if e not in self._cache:
             w = self.w_dev[e].float().cpu().double().numpy()
-            self._cache[e] = O.quantize_weight_block128(w) if self.fp8 else (w, None)
+            if self.mx:
+                self._cache[e] = O.quantize_mx_group32(w)
+            else:
+                self._cache[e] = O.quantize_weight_block128(w) if self.fp8 else (w, None)
         return self._cache[e]
 
     @property
@@ -63,14 +67,17 @@ class Case:
         self.w13_bf16, self.w2_bf16 = weights
         self.x = inputs.make_tokens(cfg, T, seed, device=dev)
         self.routing = inputs.make_routing(cfg, T, seed, device=dev)
-        if cfg.fp8:
+        if cfg.mx:
+            self.w13, self.w13_scale = ops.quantize_weights_mxfp8(self.w13_bf16)
+            self.w2, self.w2_scale = ops.quantize_weights_mxfp8(self.w2_bf16)
+        elif cfg.fp8:
             self.w13, self.w13_scale = ops.quantize_weights_fp8(self.w13_bf16)
             self.w2, self.w2_scale = ops.quantize_weights_fp8(self.w2_bf16)
         else:
             self.w13, self.w2 = self.w13_bf16, self.w2_bf16
             self.w13_scale = self.w2_scale = None
         self.p = ops.problem(T, cfg.E, cfg.topk, cfg.H, cfg.I, fp8=cfg.fp8, mode=mode, block_m=block_m,
-                             split_k=split_k)
+                             split_k=split_k, mx=cfg.mx)
         self.q = ops.resolve_problem(self.p)
         self.ws = ops.alloc_workspace(self.p)
         self.out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
@@ -96,11 +103,11 @@ class Case:
         else:
             kw["topk_ids"] = self.routing["topk_ids"].cpu().numpy()
             kw["topk_weights"] = self.routing["topk_weights"].cpu().numpy()
-        l13 = LazyExperts(self.w13_bf16, self.cfg.fp8)
-        l2 = LazyExperts(self.w2_bf16, self.cfg.fp8)
+        l13 = LazyExperts(self.w13_bf16, self.cfg.fp8, self.cfg.mx)
+        l2 = LazyExperts(self.w2_bf16, self.cfg.fp8, self.cfg.mx)
         if self.cfg.fp8:
             return O.moe_forward(x, l13.codes, l2.codes, self.cfg.topk, w13_scale=l13.scales, w2_scale=l2.scales,
-                                 tokens=tokens, return_y=return_y, **kw)
+                                 tokens=tokens, return_y=return_y, mx=self.cfg.mx, **kw)
         return O.moe_forward(x, l13.codes, l2.codes, self.cfg.topk, tokens=tokens, return_y=return_y, **kw)
 
 

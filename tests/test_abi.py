@@ -70,6 +70,32 @@ def test_resolve_problem_auto_modes(L):
     assert q.mode == ops.MODE_SWAP_AB and q.block_m == 32
 
 
+def test_resolve_problem_mxfp8_is_normal_128(L):
+    for T in (1, 64, 16384):
+        q = ops.resolve_problem(ops.problem(T, 128, 8, 4096, 1536, mx=True))
+        assert q.weight_dtype == ops.DTYPE_MXFP8_E4M3 and q.mode == ops.MODE_NORMAL and q.block_m == 128
+    p = ops.problem(16, 8, 2, 256, 128, mx=True, mode=ops.MODE_SWAP_AB)
+    assert L.moe_workspace_size(ctypes.byref(p)) == 0
+    p = ops.problem(16, 8, 2, 256, 128, mx=True, block_m=64)
+    assert L.moe_workspace_size(ctypes.byref(p)) == 0
+    # activation scale regions: the SF atoms take exactly the bytes of the fp32 K-block scales
+    lay_mx = ops.workspace_layout(ops.problem(300, 16, 4, 1024, 512, mx=True))
+    lay_f8 = ops.workspace_layout(ops.problem(300, 16, 4, 1024, 512, fp8=True, mode=ops.MODE_NORMAL))
+    assert lay_mx.total_bytes == lay_f8.total_bytes and lay_mx.a1_scale >= 0 and lay_mx.a2_scale >= 0
+
+
+def test_quantize_mxfp8_argument_errors(L):
+    g = _fake(1 << 20)
+    assert L.moe_quantize_weights_mxfp8(g, 1, 100, 128, g, g, None) == ops.MOE_ERR_INVALID
+    assert L.moe_quantize_weights_mxfp8(g, 1, 128, 128, None, g, None) == ops.MOE_ERR_INVALID
+    assert L.moe_quantize_weights_mxfp8(g, 1, 128, 128, g, _fake((1 << 20) + 4), None) == ops.MOE_ERR_INVALID
+    p = ops.problem(16, 8, 2, 256, 128, mx=True)
+    need = ops.workspace_size(p)
+    # MXFP8 scale factors must be 16-byte aligned (bulk copies read whole 512-byte atoms)
+    assert L.moe_fused_forward(ctypes.byref(p), g, g, None, None, g, g, _fake((1 << 20) + 4), g, g, g, need,
+                               None) == ops.MOE_ERR_INVALID
+
+
 @pytest.mark.parametrize("bad", [
     dict(T=-1), dict(E=0), dict(E=2000), dict(topk=0), dict(topk=9, E=8), dict(H=100), dict(I=0), dict(I=200),
     dict(mode=7), dict(mode=ops.MODE_NORMAL, block_m=16), dict(mode=ops.MODE_SWAP_AB, block_m=128),
