@@ -116,7 +116,15 @@ typedef struct moe_problem {
   int32_t block_m;      /* rows per expert block: 16, 32, 64 (swap-AB); 128, or 256 for FP8 two-SM tiles (normal); 0 = auto */
   int32_t renormalize;  /* router: 1 = renormalise the chosen softmax weights (default), 0 = keep them */
   int32_t split_k;      /* swap-AB GEMMs: 0 = split K when few tiles are in flight (default), 1 = never */
-  int32_t reserved[6];  /* must be zero */
+  /* 1 = scale each token row by its router weight before GEMM1 instead of the
+   * expert output after GEMM2 (vLLM's apply_router_weight_on_input, shown
+   * False in the PR analysis' test); requires topk == 1.  0 = default. */
+  int32_t router_weight_on_input;
+  /* SwiGLU clamp limit L > 0: gate = min(gate, L), up = clamp(up, -L, L) before
+   * SiLU(gate) * up (the clamp_limit that the PR analysis' sorted-A predicate
+   * excludes).  0 = no clamp (default). */
+  float swiglu_limit;
+  int32_t reserved[4];  /* must be zero */
 } moe_problem;
 
 /*

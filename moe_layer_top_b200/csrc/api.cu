@@ -1,6 +1,7 @@
 // C ABI of the fused MoE layer: argument validation, problem resolution,
 // workspace layout and the stage pipeline.  Every entry point validates all
 // of its arguments before it enqueues anything.
+#include <cmath>
 #include <cstdarg>
 #include <cstdio>
 #include <cstring>
@@ -78,8 +79,14 @@ int validate_problem(const moe_problem* p) {
   if (p->mode < MOE_MODE_AUTO || p->mode > MOE_MODE_SWAP_AB) return fail(MOE_ERR_INVALID, "mode %d", p->mode);
   if (p->renormalize != 0 && p->renormalize != 1) return fail(MOE_ERR_INVALID, "renormalize must be 0 or 1");
   if (p->split_k != 0 && p->split_k != 1) return fail(MOE_ERR_INVALID, "split_k must be 0 or 1");
-  for (int i = 0; i < 6; ++i)
+  for (int i = 0; i < 4; ++i)
     if (p->reserved[i] != 0) return fail(MOE_ERR_INVALID, "reserved fields must be zero");
+  if (p->router_weight_on_input != 0 && p->router_weight_on_input != 1)
+    return fail(MOE_ERR_INVALID, "router_weight_on_input must be 0 or 1");
+  if (p->router_weight_on_input == 1 && p->topk != 1)
+    return fail(MOE_ERR_INVALID, "router_weight_on_input needs topk == 1 (got %d)", p->topk);
+  if (!(p->swiglu_limit >= 0.0f) || p->swiglu_limit == INFINITY)
+    return fail(MOE_ERR_INVALID, "swiglu_limit must be 0 (off) or a positive finite value");
   const bool fp8 = p->weight_dtype == MOE_DTYPE_FP8_E4M3;
   if (p->weight_dtype == MOE_DTYPE_MXFP8_E4M3) {
     if (p->mode == MOE_MODE_SWAP_AB) return fail(MOE_ERR_UNSUPPORTED, "MXFP8 weights run normal tiles only");
@@ -280,7 +287,8 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
       case MOE_STAGE_GATHER:
         e = moe::launch_gather(x, p.H, p.topk, nflat, at<int32_t>(ws, L.sorted_token_ids),
                                at<int32_t>(ws, L.num_tokens_post_padded), cap, plan.fp8, plan.mx,
-                               at<void>(ws, L.a1), plan.fp8 ? at<void>(ws, L.a1_scale) : nullptr, stream);
+                               p.router_weight_on_input == 1 ? wts : nullptr, at<void>(ws, L.a1),
+                               plan.fp8 ? at<void>(ws, L.a1_scale) : nullptr, stream);
         if (e != cudaSuccess) return cuda_fail(e, "gather");
         break;
       case MOE_STAGE_GEMM1:
@@ -304,6 +312,8 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
         gp.num_sms = sms;
         gp.split_mode = p.split_k;
         gp.partials = swap ? at<float>(ws, L.partials) : nullptr;
+        gp.weight_on_input = p.router_weight_on_input == 1;
+        gp.swiglu_limit = p.swiglu_limit > 0.0f ? p.swiglu_limit : INFINITY;
         if (s == MOE_STAGE_GEMM1) {
           e = moe::launch_gemm1(gp, at<void>(ws, L.a1), plan.fp8 ? at<void>(ws, L.a1_scale) : nullptr, w13,
                                 w13_scale, at<void>(ws, L.a2), plan.fp8 ? at<void>(ws, L.a2_scale) : nullptr,

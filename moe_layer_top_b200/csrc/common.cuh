@@ -473,4 +473,15 @@ __device__ __forceinline__ float silu_mul_bf16(float g, float u) {
   return bf16_round(s * u);
 }
 
+// SwiGLU with an optional clamp (limit = +inf: none): gate = min(g, L),
+// up = clamp(u, -L, L), then silu_mul_bf16.  g, u are bf16 values.
+__device__ __forceinline__ float swiglu_bf16(float g, float u, float limit) {
+  return silu_mul_bf16(fminf(g, limit), fminf(fmaxf(u, -limit), limit));
+}
+
+// routed weight of flat assignment `flat`, or 1 when it was applied to the input
+__device__ __forceinline__ float route_weight(const float* topk_weights, int flat) {
+  return topk_weights ? (*(topk_weights + flat)) : 1.0f;
+}
+
 }  // namespace moe

@@ -49,7 +49,7 @@ template <int Q>
 __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* x, int H, int topk,
                                                      int nflat, const int32_t* sorted_ids,
                                                      const int32_t* ntpp_ptr, int capacity,
-                                                     void* a1, void* a1_scale) {
+                                                     const float* row_weight, void* a1, void* a1_scale) {
   pdl_launch_dependents();
   pdl_wait();
   const int ntpp = *ntpp_ptr;
@@ -61,11 +61,20 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* x, int
     // depends only on its own input row, and padding outputs are never stored
     if (flat >= nflat) continue;
     const __nv_bfloat16* src = x + static_cast<size_t>(flat / topk) * H;
+    // router weight applied on the input: the row is w * x, rounded to bf16
+    const float rw = row_weight ? (*(row_weight + flat)) : 1.0f;
     for (int it = 0; it < iters; ++it) {
       const int v = it * blockDim.x + threadIdx.x;  // uniform trip count: shuffles below see full warps
       const bool in = v < vecs;
       uint4 u = make_uint4(0, 0, 0, 0);
       if (in) u = (*(reinterpret_cast<const uint4*>(src) + v));
+      if (row_weight) {
+        float f[8];
+        unpack8(u, f);
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] *= rw;
+        u = pack8(f);
+      }
       if constexpr (Q == kGatherBf16) {
         if (in) reinterpret_cast<uint4*>(static_cast<__nv_bfloat16*>(a1) + static_cast<size_t>(row) * H)[v] = u;
       } else {
@@ -99,19 +108,19 @@ __global__ void __launch_bounds__(256) gather_kernel(const __nv_bfloat16* x, int
 }
 
 cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32_t* sorted_ids,
-                          const int32_t* ntpp, int capacity, bool fp8, bool mx, void* a1, void* a1_scale,
-                          cudaStream_t stream) {
+                          const int32_t* ntpp, int capacity, bool fp8, bool mx, const float* row_weight, void* a1,
+                          void* a1_scale, cudaStream_t stream) {
   if (capacity == 0) return cudaSuccess;
   int blocks = capacity < 148 * 8 ? capacity : 148 * 8;
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (mx)
     return launch_pdl(gather_kernel<kGatherMx>, blocks, 256, 0, stream, xb, H, topk, nflat, sorted_ids, ntpp,
-                      capacity, a1, a1_scale);
+                      capacity, row_weight, a1, a1_scale);
   if (fp8)
     return launch_pdl(gather_kernel<kGatherFp8>, blocks, 256, 0, stream, xb, H, topk, nflat, sorted_ids, ntpp,
-                      capacity, a1, a1_scale);
+                      capacity, row_weight, a1, a1_scale);
   return launch_pdl(gather_kernel<kGatherBf16>, blocks, 256, 0, stream, xb, H, topk, nflat, sorted_ids, ntpp,
-                    capacity, a1, a1_scale);
+                    capacity, row_weight, a1, a1_scale);
 }
 
 // ----------------------------------------------------------------------------

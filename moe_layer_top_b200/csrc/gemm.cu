@@ -86,6 +86,7 @@ struct Args {
   int* status;
   float* partials;         // swap-AB split-K: [unit][acc column][128] fp32 partial sums
   int splits;              // swap-AB split-K factor S (1: no split); chosen on the host
+  float swiglu_limit;      // GEMM1: SwiGLU clamp limit (+inf: none)
   const uint8_t* a_sf;     // MXFP8: E8M0 SF atoms of the activation rows [capacity, K]
   const uint8_t* w_sf;     // MXFP8: E8M0 SF atoms of the weights [E * Nw, K]
   uint8_t* out_sf;         // MXFP8 GEMM1: SF atoms of a2 [capacity, I]
@@ -439,8 +440,9 @@ __global__ void __launch_bounds__(kThreads, 1)
               tmem_wait_ld();
 #pragma unroll
               for (int i = 0; i < 8; ++i) {
-                const float p0 = silu_mul_bf16(bf16_round(dg[2 * i]), bf16_round(du[2 * i]));
-                const float p1 = silu_mul_bf16(bf16_round(dg[2 * i + 1]), bf16_round(du[2 * i + 1]));
+                const float p0 = swiglu_bf16(bf16_round(dg[2 * i]), bf16_round(du[2 * i]), args.swiglu_limit);
+                const float p1 =
+                    swiglu_bf16(bf16_round(dg[2 * i + 1]), bf16_round(du[2 * i + 1]), args.swiglu_limit);
                 const __nv_bfloat162 h2 = __floats2bfloat162_rn(p0, p1);
                 packed[8 * c + i] = *reinterpret_cast<const uint32_t*>(&h2);
               }
@@ -458,7 +460,7 @@ __global__ void __launch_bounds__(kThreads, 1)
             float amax = 0.f;
 #pragma unroll
             for (int i = 0; i < 64; ++i) {
-              const float p = silu_mul_bf16(bf16_round(acc_a[i]), bf16_round(acc_b[i]));
+              const float p = swiglu_bf16(bf16_round(acc_a[i]), bf16_round(acc_b[i]), args.swiglu_limit);
               acc_a[i] = p;
               amax = fmaxf(amax, fabsf(p));
             }
@@ -493,7 +495,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           // ---- GEMM2 epilogue: routed weight, scatter the row to y[flat]
           const int flat = (*(args.sorted_ids + grow));
           const bool real = flat < args.nflat;
-          const float wt = real ? (*(args.topk_weights + flat)) : 0.f;
+          const float wt = real ? route_weight(args.topk_weights, flat) : 0.f;
           __nv_bfloat16* yrow =
               static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(real ? flat : 0) * H + nt * 256 + g * 128;
           if constexpr (kFP8) {
@@ -639,7 +641,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           // ---- GEMM1: this thread owns intermediate column nt*128 + row for kHT tokens
           const int icol = nt * 128 + row;
 #pragma unroll
-          for (int j = 0; j < kHT; ++j) acc_a[j] = silu_mul_bf16(bf16_round(acc_a[j]), bf16_round(acc_b[j]));
+          for (int j = 0; j < kHT; ++j)
+            acc_a[j] = swiglu_bf16(bf16_round(acc_a[j]), bf16_round(acc_b[j]), args.swiglu_limit);
           if constexpr (!kFP8) {
             __nv_bfloat16* a2 = static_cast<__nv_bfloat16*>(args.out);
 #pragma unroll
@@ -683,7 +686,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           for (int j = 0; j < kHT; ++j) {
             const int flat = (*(args.sorted_ids + tok0 + j));
             if (flat < args.nflat) {
-              const float wt = (*(args.topk_weights + flat));
+              const float wt = route_weight(args.topk_weights, flat);
               y[static_cast<size_t>(flat) * H + hcol] = __float2bfloat16_rn(acc_a[j] * wt);
             }
           }
@@ -741,7 +744,7 @@ __global__ void __launch_bounds__(128) splitk_reduce_kernel(Args args) {
     if constexpr (!kDown) {
       const int icol = nt * 128 + row;
 #pragma unroll
-      for (int j = 0; j < kBM; ++j) a[j] = silu_mul_bf16(bf16_round(a[j]), bf16_round(b[j]));
+      for (int j = 0; j < kBM; ++j) a[j] = swiglu_bf16(bf16_round(a[j]), bf16_round(b[j]), args.swiglu_limit);
       if constexpr (!kFP8) {
         __nv_bfloat16* a2 = static_cast<__nv_bfloat16*>(args.out);
 #pragma unroll
@@ -773,7 +776,7 @@ __global__ void __launch_bounds__(128) splitk_reduce_kernel(Args args) {
       for (int j = 0; j < kBM; ++j) {
         const int flat = (*(args.sorted_ids + tok0 + j));
         if (flat < args.nflat) {
-          const float wt = (*(args.topk_weights + flat));
+          const float wt = route_weight(args.topk_weights, flat);
           y[static_cast<size_t>(flat) * args.H + hcol] = __float2bfloat16_rn(a[j] * wt);
         }
       }
@@ -1016,7 +1019,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           float amax = 0.f;
 #pragma unroll
           for (int i = 0; i < 32; ++i) {
-            p[i] = silu_mul_bf16(bf16_round(v[32 * grp + i]), bf16_round(v[64 + 32 * grp + i]));
+            p[i] = swiglu_bf16(bf16_round(v[32 * grp + i]), bf16_round(v[64 + 32 * grp + i]), args.swiglu_limit);
             amax = fmaxf(amax, fabsf(p[i]));
           }
           const float scale = act_scale_from_amax(amax);
@@ -1037,7 +1040,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         // routed weight, scatter the row to y[flat]
         const int flat = (*(args.sorted_ids + grow));
         if (flat < args.nflat) {
-          const float wt = (*(args.topk_weights + flat));
+          const float wt = route_weight(args.topk_weights, flat);
           __nv_bfloat16* yrow = static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(flat) * H + nt * 256 +
                                 g * 128;
 #pragma unroll
@@ -1331,7 +1334,8 @@ __global__ void __launch_bounds__(kThreads, 1)
         float amax = 0.f;
 #pragma unroll
         for (int i = 0; i < 64; ++i) {
-          const float p = silu_mul_bf16(bf16_round(__uint_as_float(acc_a[i])), bf16_round(__uint_as_float(acc_b[i])));
+          const float p = swiglu_bf16(bf16_round(__uint_as_float(acc_a[i])), bf16_round(__uint_as_float(acc_b[i])),
+                                      args.swiglu_limit);
           acc_a[i] = __float_as_uint(p);
           amax = fmaxf(amax, fabsf(p));
         }
@@ -1362,7 +1366,7 @@ __global__ void __launch_bounds__(kThreads, 1)
       } else {
         const int flat = *(args.sorted_ids + grow);
         if (flat < args.nflat) {
-          const float wt = *(args.topk_weights + flat);
+          const float wt = route_weight(args.topk_weights, flat);
           __nv_bfloat16* yrow =
               static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(flat) * H + nt * 256 + g * 128;
 #pragma unroll
@@ -1565,7 +1569,8 @@ cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const void* a1_sc
   args.ntpp = p.ntpp;
   args.expert_ids = p.expert_ids;
   args.sorted_ids = p.sorted_ids;
-  args.topk_weights = p.topk_weights;
+  args.topk_weights = p.weight_on_input ? nullptr : p.topk_weights;
+  args.swiglu_limit = p.swiglu_limit;
   if (p.mx) {
     args.a_sf = static_cast<const uint8_t*>(a1_scale);
     args.w_sf = static_cast<const uint8_t*>(w13_scale);
@@ -1593,7 +1598,8 @@ cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const void* a2_sc
   args.ntpp = p.ntpp;
   args.expert_ids = p.expert_ids;
   args.sorted_ids = p.sorted_ids;
-  args.topk_weights = p.topk_weights;
+  args.topk_weights = p.weight_on_input ? nullptr : p.topk_weights;
+  args.swiglu_limit = p.swiglu_limit;
   if (p.mx) {
     args.a_sf = static_cast<const uint8_t*>(a2_scale);
     args.w_sf = static_cast<const uint8_t*>(w2_scale);

@@ -51,9 +51,10 @@ cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in,
 // gather x rows into sorted order: bf16 copy, FP8 per-(row,128) quantisation
 // (a1_scale: fp32 [H/128, capacity]) or MXFP8 per-(row,32) quantisation
 // (a1_scale: E8M0 SF atoms of [capacity, H])
+// (row_weight != NULL: each row is first scaled by row_weight[flat], rounded to bf16)
 cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32_t* sorted_ids,
-                          const int32_t* ntpp, int capacity, bool fp8, bool mx, void* a1, void* a1_scale,
-                          cudaStream_t stream);
+                          const int32_t* ntpp, int capacity, bool fp8, bool mx, const float* row_weight, void* a1,
+                          void* a1_scale, cudaStream_t stream);
 
 // out[t] = sum_j y[t*topk + j]
 cudaError_t launch_combine(const void* y, int T, int topk, int H, void* out, cudaStream_t stream);
@@ -71,6 +72,8 @@ struct GemmProblem {
   int E, H, I, topk, nflat, block_m, capacity;
   bool fp8, swap;
   bool mx;             // MXFP8 (with fp8): block-scaled MMA, E8M0 SF atoms
+  bool weight_on_input;  // the router weight was applied in the gather: GEMM2 stores y unweighted
+  float swiglu_limit;  // SwiGLU clamp limit (+inf: none)
   const int32_t* ntpp;
   const int32_t* expert_ids;
   const int32_t* sorted_ids;

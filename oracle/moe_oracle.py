@@ -357,7 +357,7 @@ def align(topk_ids, E: int, block_m: int):
 # expert MLP and the layer
 # ----------------------------------------------------------------------------
 
-def expert_mlp(x_hat, w13_hat, w2_hat, requant, return_intermediates: bool = False):
+def expert_mlp(x_hat, w13_hat, w2_hat, requant, return_intermediates: bool = False, swiglu_limit=None):
     """One expert's SiLU-gated MLP on a batch of rows.
 
     [PR] §1.1/§1.2: ``h = x · w13ᵀ`` held in bf16 (``intermediate_cache1``);
@@ -367,11 +367,19 @@ def expert_mlp(x_hat, w13_hat, w2_hat, requant, return_intermediates: bool = Fal
     ``y = a2 · w2ᵀ`` (``requant=True``), for MXFP8 per (row, 32) with an E8M0
     scale (``requant="mx"``), for bf16 kept as is (``requant=False``).
 
+    swiglu_limit L: [PR] names a SwiGLU ``clamp_limit`` (its presence turns the
+    fused path off) but not its formula.  Reading: gate = min(gate, L) and
+    up = clamp(up, -L, L) on the bf16 values, before the activation.
+
     x_hat [n, H], w13_hat [2I, H], w2_hat [H, I]: float64.  Returns y [n, H].
     """
     i = w13_hat.shape[0] // 2
     h = round_bf16(x_hat @ w13_hat.T)
     gate, up = h[:, :i], h[:, i:]
+    if swiglu_limit is not None:
+        lim = float(np.float32(swiglu_limit))
+        gate = np.minimum(gate, lim)
+        up = np.clip(up, -lim, lim)
     act = round_bf16(gate / (1.0 + np.exp(-gate)))
     p = round_bf16(act * up)
     if requant == "mx":
@@ -391,7 +399,7 @@ def expert_mlp(x_hat, w13_hat, w2_hat, requant, return_intermediates: bool = Fal
 
 def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weights=None,
                 w13_scale=None, w2_scale=None, renormalize: bool = True, tokens=None,
-                return_y: bool = False, mx=None):
+                return_y: bool = False, mx=None, router_weight_on_input: bool = False, swiglu_limit=None):
     """The fused MoE layer: route -> experts -> top-k weighted combine.
 
     [AWS] "Warum MoE-Kernel so wichtig sind": one operation that routes each
@@ -408,6 +416,12 @@ def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weigh
     tokens: optional subset of token indices to evaluate (each output row
     depends only on its own token, its routing and the weights).
     mx: MXFP8 scales (taken from the scale dtype, uint8, when not given).
+    router_weight_on_input: [PR]'s test passes ``apply_router_weight_on_input``
+    (False there).  Reading: with top-1 routing each token row becomes
+    bf16(fp32(x) * w) before the experts and the expert output is not weighted
+    again; top-k > 1 is rejected (a non-linear expert cannot take the weight
+    on its input without changing the layer).
+    swiglu_limit: see :func:`expert_mlp`.
 
     Returns a dict with ``out`` [len(tokens), H] (float64 holding bf16
     values), ``topk_ids``, ``topk_weights`` and, when asked, ``y``
@@ -426,6 +440,11 @@ def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weigh
     tokens = np.arange(t_all) if tokens is None else np.asarray(tokens, dtype=np.int64)
 
     xs = x[tokens]
+    if router_weight_on_input:
+        if topk != 1:
+            raise ValueError("router_weight_on_input needs topk == 1")
+        w_in = np.asarray(topk_weights, dtype=np.float32)[tokens, 0]
+        xs = round_bf16((xs.astype(np.float32) * w_in[:, None]).astype(np.float64))   # one fp32 product
     if mx:
         qx, sx = quantize_mx_group32(xs)
         x_hat = dequantize_mx_group32(qx, sx)
@@ -450,9 +469,9 @@ def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weigh
         else:
             w13_e = np.asarray(w13[e], dtype=np.float64)
             w2_e = np.asarray(w2[e], dtype=np.float64)
-        y = expert_mlp(x_hat[rows], w13_e, w2_e, requant="mx" if mx else fp8)
+        y = expert_mlp(x_hat[rows], w13_e, w2_e, requant="mx" if mx else fp8, swiglu_limit=swiglu_limit)
         for r, c, yr in zip(rows, cols, y):
-            acc[r] += wts[r, c] * yr
+            acc[r] += (1.0 if router_weight_on_input else wts[r, c]) * yr
             if return_y:
                 y_all[r, c] = yr
     result = {

@@ -84,6 +84,19 @@ def test_resolve_problem_mxfp8_is_normal_128(L):
     assert lay_mx.total_bytes == lay_f8.total_bytes and lay_mx.a1_scale >= 0 and lay_mx.a2_scale >= 0
 
 
+def test_epilogue_variant_validation(L):
+    ok = ops.problem(16, 8, 1, 256, 128, router_weight_on_input=True)
+    assert L.moe_workspace_size(ctypes.byref(ok)) > 0
+    bad = ops.problem(16, 8, 2, 256, 128, router_weight_on_input=True)      # needs top-1
+    assert L.moe_workspace_size(ctypes.byref(bad)) == 0
+    assert L.moe_workspace_size(ctypes.byref(ops.problem(16, 8, 2, 256, 128, swiglu_limit=7.0))) > 0
+    for lim in (-1.0, float("inf"), float("nan")):
+        assert L.moe_workspace_size(ctypes.byref(ops.problem(16, 8, 2, 256, 128, swiglu_limit=lim))) == 0
+    p = ops.problem(16, 8, 2, 256, 128)
+    p.router_weight_on_input = 2
+    assert L.moe_workspace_size(ctypes.byref(p)) == 0
+
+
 def test_quantize_mxfp8_argument_errors(L):
     g = _fake(1 << 20)
     assert L.moe_quantize_weights_mxfp8(g, 1, 100, 128, g, g, None) == ops.MOE_ERR_INVALID

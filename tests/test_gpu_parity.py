@@ -319,3 +319,54 @@ def test_all_tokens_on_one_expert_and_topk_equals_E():
     c1.routing["topk_ids"] = torch.full((300, 2), 1, dtype=torch.int32, device="cuda")   # duplicates in each row
     c1.run()
     assert_close(c1.out.float().cpu().numpy(), c1.oracle()["out"], fp8=False)
+
+
+# ----------------------------------------------------------------------------- epilogue variants
+TOP1_BF16 = inputs.make_custom_config("top1_bf16", E=16, topk=1, H=1024, I=512, fp8=False, routing="logits")
+TOP1_FP8 = inputs.make_custom_config("top1_fp8", E=16, topk=1, H=1024, I=512, fp8=True, routing="logits")
+TOP1_MX = inputs.make_custom_config("top1_mx", E=16, topk=1, H=1024, I=512, fp8=True, mx=True, routing="logits")
+
+
+@pytest.mark.parametrize("cfg,T,mode,bm", [(TOP1_BF16, 5, ops.MODE_AUTO, 0), (TOP1_BF16, 300, ops.MODE_NORMAL, 128),
+                                           (TOP1_FP8, 40, ops.MODE_SWAP_AB, 32), (TOP1_FP8, 300, ops.MODE_AUTO, 0),
+                                           (TOP1_MX, 100, ops.MODE_AUTO, 0)],
+                         ids=["bf16-swap", "bf16-normal", "fp8-swap", "fp8-normal", "mx"])
+def test_router_weight_on_input(cfg, T, mode, bm):
+    """Top-1 routing with the weight applied to x before GEMM1 (the gather
+    scales each row); GEMM2 then stores the expert output unweighted."""
+    c = Case(cfg, T, seed=3, mode=mode, block_m=bm, router_weight_on_input=True)
+    out = c.run()
+    assert c.status() == ops.MOE_STATUS_OK
+    ref = c.oracle()
+    assert_close(out.float().cpu().numpy(), ref["out"], fp8=cfg.fp8)
+    if not cfg.fp8:   # the gathered bf16 rows are bf16(fp32(x) * w) exactly
+        v = c.views()
+        ntpp = int(v["num_tokens_post_padded"].item())
+        ids = v["sorted_token_ids"][:ntpp].cpu().numpy()
+        rows = np.nonzero(ids < T)[0]
+        w = v["topk_weights"].cpu().numpy()[ids[rows], 0]
+        xs = (c.x.float()[torch.from_numpy(ids[rows]).cuda()] * torch.from_numpy(w).cuda()[:, None]).bfloat16()
+        assert torch.equal(v["a1"][:ntpp][torch.from_numpy(rows).cuda()], xs)
+
+
+@pytest.mark.parametrize("cfg,T,mode,bm", [(MID_BF16, 7, ops.MODE_SWAP_AB, 16), (MID_BF16, 300, ops.MODE_NORMAL, 128),
+                                           (MID_FP8, 2, ops.MODE_AUTO, 0), (MID_FP8, 500, ops.MODE_NORMAL, 128)],
+                         ids=["bf16-swap", "bf16-normal", "fp8-swap-split", "fp8-normal"])
+def test_swiglu_clamp(cfg, T, mode, bm):
+    """A SwiGLU clamp small enough to bite: gate <= L and |up| <= L before the activation."""
+    c = Case(cfg, T, seed=6, mode=mode, block_m=bm, swiglu_limit=0.05)
+    out = c.run()
+    assert c.status() == ops.MOE_STATUS_OK
+    ref = c.oracle()
+    assert_close(out.float().cpu().numpy(), ref["out"], fp8=cfg.fp8)
+    plain = Case(cfg, T, seed=6, mode=mode, block_m=bm, weights=(c.w13_bf16, c.w2_bf16)).run()
+    assert not torch.equal(out, plain)                 # the limit changed the result
+
+
+def test_swiglu_clamp_mx_and_two_sm():
+    mx_cfg = inputs.make_custom_config("mid_mx", E=16, topk=4, H=1024, I=512, fp8=True, mx=True, routing="uniform_ids")
+    for cfg, bm in ((mx_cfg, 0), (MID_FP8, 256)):
+        c = Case(cfg, 700, seed=7, block_m=bm, swiglu_limit=0.05)
+        out = c.run()
+        assert c.status() == ops.MOE_STATUS_OK
+        assert_close(out.float().cpu().numpy(), c.oracle()["out"], fp8=True)

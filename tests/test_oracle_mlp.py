@@ -83,6 +83,53 @@ def test_expert_mlp_closed_form_mx_requant():
     np.testing.assert_array_equal(y, ref)
 
 
+def test_expert_mlp_closed_form_swiglu_clamp():
+    H, I = 256, 128
+    w13, w2, perm, perm2 = _selection_weights(H, I, 6)
+    rng = np.random.default_rng(7)
+    x = O.round_bf16(rng.standard_normal((6, H)) * 4.0)
+    lim = 2.5
+    y = O.expert_mlp(x, w13, w2, requant=False, swiglu_limit=lim)
+    g = torch.clamp(torch.from_numpy(x[:, perm[:I]]), max=lim)
+    u = torch.clamp(torch.from_numpy(x[:, perm[I:2 * I]]), -lim, lim)
+    p = (F.silu(g).to(torch.bfloat16).double() * u).to(torch.bfloat16).double()
+    ref = np.zeros_like(y)
+    ref[:, perm2[:I]] = p.numpy()
+    np.testing.assert_array_equal(y, ref)
+    assert np.abs(x[:, perm[:2 * I]]).max() > lim          # the clamp is exercised
+    # no limit reproduces the unclamped rule
+    np.testing.assert_array_equal(O.expert_mlp(x, w13, w2, requant=False),
+                                  O.expert_mlp(x, w13, w2, requant=False, swiglu_limit=None))
+
+
+def test_router_weight_on_input_top1():
+    cfg = inputs.make_custom_config("tiny_top1", E=4, topk=1, H=256, I=128, routing="uniform_ids", tokens=(9,))
+    w13, w2 = inputs.make_weights(cfg, 8)
+    x = inputs.make_tokens(cfg, 9, 8).double().numpy()
+    r = inputs.make_routing(cfg, 9, 8)
+    ids = r["topk_ids"].numpy()
+    wts = (np.random.default_rng(1).uniform(0.2, 1.7, (9, 1))).astype(np.float32)
+    a, b = w13.double().numpy(), w2.double().numpy()
+    res = O.moe_forward(x, a, b, 1, topk_ids=ids, topk_weights=wts, router_weight_on_input=True)
+    # independent path: scale rows with torch's fp32 product and bf16 cast, run each expert, no output weight
+    xs = (torch.from_numpy(x).float() * torch.from_numpy(wts)).to(torch.bfloat16).double()
+    ref = np.zeros_like(x)
+    for t in range(9):
+        e = int(ids[t, 0])
+        h = (xs[t] @ torch.from_numpy(a[e]).T).to(torch.bfloat16).double()
+        p = (F.silu(h[:128]).to(torch.bfloat16).double() * h[128:]).to(torch.bfloat16).double()
+        ref[t] = (p @ torch.from_numpy(b[e]).T).to(torch.bfloat16).double().numpy()
+    np.testing.assert_array_equal(res["out"], ref)
+    # unit weights: identical to weighting the output
+    ones = np.ones((9, 1), np.float32)
+    np.testing.assert_array_equal(
+        O.moe_forward(x, a, b, 1, topk_ids=ids, topk_weights=ones, router_weight_on_input=True)["out"],
+        O.moe_forward(x, a, b, 1, topk_ids=ids, topk_weights=ones)["out"])
+    with pytest.raises(ValueError):
+        O.moe_forward(x, a, b, 2, topk_ids=np.zeros((9, 2), np.int64), topk_weights=np.ones((9, 2), np.float32),
+                      router_weight_on_input=True)
+
+
 def _mx_torch(t, group=32):
     """Independent MX quantise-dequantise of the last dim with torch ops."""
     shp = t.shape
