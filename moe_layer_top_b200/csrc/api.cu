@@ -144,8 +144,11 @@ struct Plan {
   moe_problem p;
   moe_workspace_layout L;
   int64_t nflat;
-  bool fp8;  // 8-bit weights and activations (block-128 or MX scales)
-  bool mx;   // MXFP8: E8M0 scale factors per 32 elements
+  bool fp8;   // 8-bit weights and activations (block-128 or MX scales)
+  bool mx;    // MXFP8: E8M0 scale factors per 32 elements
+  bool pair;        // two-SM FP8 tiles
+  bool tok_gather;  // swap-AB: GEMM1 gathers token rows (TMA gather4) from x or its per-token copy;
+                    // normal tiles read a sorted copy a1 [capacity, H] (gather4 is too slow for 128-row tiles)
 };
 
 int make_plan(const moe_problem* in, Plan* plan) {
@@ -156,6 +159,8 @@ int make_plan(const moe_problem* in, Plan* plan) {
   const moe_problem& p = plan->p;
   plan->mx = p.weight_dtype == MOE_DTYPE_MXFP8_E4M3;
   plan->fp8 = p.weight_dtype == MOE_DTYPE_FP8_E4M3 || plan->mx;
+  plan->pair = p.mode == MOE_MODE_NORMAL && p.block_m == 256;
+  plan->tok_gather = p.mode == MOE_MODE_SWAP_AB;
   plan->nflat = static_cast<int64_t>(p.T) * p.topk;
   const int64_t cap = capacity_of(p.T, p.topk, p.E, p.block_m);
   if (cap >= (int64_t(1) << 31)) return fail(MOE_ERR_INVALID, "padded row capacity overflows int32");
@@ -177,7 +182,17 @@ int make_plan(const moe_problem* in, Plan* plan) {
   L.expert_counts = take(static_cast<int64_t>(p.E) * 4);
   L.expert_offsets = take(static_cast<int64_t>(p.E + 1) * 4);
   L.align_scratch = take(chunks * p.E * 4);
-  L.a1 = take(cap * p.H * elem);
+  // GEMM1's token rows: normal tiles read a sorted copy [cap, H]; swap-AB tiles
+  // gather rows of x itself (bf16) or of its per-token copy [T, H] (quantised,
+  // or scaled by the router weight)
+  const bool rw = p.router_weight_on_input == 1;
+  if (!plan->tok_gather)
+    L.a1 = take(cap * p.H * elem);
+  else if (plan->fp8 || rw)
+    L.a1 = take(static_cast<int64_t>(p.T) * p.H * elem);
+  else
+    L.a1 = -1;
+  L.pos_of_flat = (plan->fp8 && plan->tok_gather) ? take(plan->nflat * 4) : -1;
   // FP8: fp32 [K/128, cap]; MXFP8: E8M0 SF atoms, (cap/128) * (K/128) * 512 bytes -- the same size
   L.a1_scale = plan->fp8 ? take(cap * (p.H / 128) * 4) : -1;
   L.a2 = take(cap * p.I * elem);
@@ -243,6 +258,9 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
   const int cap = L.capacity;
   const bool small = moe::route_align_small_fits(plan.nflat, p.E);
   const bool swap = p.mode == MOE_MODE_SWAP_AB;
+  int32_t* pos = L.pos_of_flat >= 0 ? at<int32_t>(ws, L.pos_of_flat) : nullptr;
+  // GEMM1's token source: the sorted copy (normal tiles), the per-token copy, or x
+  const void* tok_src = L.a1 >= 0 ? at<void>(ws, L.a1) : x;
   bool aligned_already = false;
   cudaError_t e;
 
@@ -258,7 +276,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
                                             cap, at<int32_t>(ws, L.sorted_token_ids), at<int32_t>(ws, L.expert_ids),
                                             at<int32_t>(ws, L.num_tokens_post_padded),
                                             at<int32_t>(ws, L.expert_counts), at<int32_t>(ws, L.expert_offsets),
-                                            status, stream);
+                                            status, pos, stream);
           if (e != cudaSuccess) return cuda_fail(e, "route+align");
           aligned_already = true;
         } else if (logits) {
@@ -274,21 +292,27 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
                                             p.block_m, cap, at<int32_t>(ws, L.sorted_token_ids),
                                             at<int32_t>(ws, L.expert_ids), at<int32_t>(ws, L.num_tokens_post_padded),
                                             at<int32_t>(ws, L.expert_counts), at<int32_t>(ws, L.expert_offsets),
-                                            status, stream);
+                                            status, pos, stream);
           if (e != cudaSuccess) return cuda_fail(e, "align");
           break;
         }
         e = moe::launch_align(ids, nflat, p.E, p.block_m, cap, at<int32_t>(ws, L.sorted_token_ids),
                               at<int32_t>(ws, L.expert_ids), at<int32_t>(ws, L.num_tokens_post_padded),
                               at<int32_t>(ws, L.expert_counts), at<int32_t>(ws, L.expert_offsets),
-                              at<int32_t>(ws, L.align_scratch), nullptr, nullptr, status, stream);
+                              at<int32_t>(ws, L.align_scratch), nullptr, nullptr, status, pos, stream);
         if (e != cudaSuccess) return cuda_fail(e, "align");
         break;
       case MOE_STAGE_GATHER:
-        e = moe::launch_gather(x, p.H, p.topk, nflat, at<int32_t>(ws, L.sorted_token_ids),
-                               at<int32_t>(ws, L.num_tokens_post_padded), cap, plan.fp8, plan.mx,
-                               p.router_weight_on_input == 1 ? wts : nullptr, at<void>(ws, L.a1),
-                               plan.fp8 ? at<void>(ws, L.a1_scale) : nullptr, stream);
+        if (!plan.tok_gather)
+          e = moe::launch_gather(x, p.H, p.topk, nflat, at<int32_t>(ws, L.sorted_token_ids),
+                                 at<int32_t>(ws, L.num_tokens_post_padded), cap, plan.fp8, plan.mx,
+                                 p.router_weight_on_input == 1 ? wts : nullptr, at<void>(ws, L.a1),
+                                 plan.fp8 ? at<void>(ws, L.a1_scale) : nullptr, stream);
+        else
+          e = moe::launch_prepare_x(x, p.T, p.H, p.topk, plan.fp8, plan.mx, pos, cap,
+                                    p.router_weight_on_input == 1 ? wts : nullptr,
+                                    L.a1 >= 0 ? at<void>(ws, L.a1) : nullptr,
+                                    plan.fp8 ? at<void>(ws, L.a1_scale) : nullptr, stream);
         if (e != cudaSuccess) return cuda_fail(e, "gather");
         break;
       case MOE_STAGE_GEMM1:
@@ -313,9 +337,11 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
         gp.split_mode = p.split_k;
         gp.partials = swap ? at<float>(ws, L.partials) : nullptr;
         gp.weight_on_input = p.router_weight_on_input == 1;
+        gp.gather_tok = plan.tok_gather;
+        gp.T = p.T;
         gp.swiglu_limit = p.swiglu_limit > 0.0f ? p.swiglu_limit : INFINITY;
         if (s == MOE_STAGE_GEMM1) {
-          e = moe::launch_gemm1(gp, at<void>(ws, L.a1), plan.fp8 ? at<void>(ws, L.a1_scale) : nullptr, w13,
+          e = moe::launch_gemm1(gp, tok_src, plan.fp8 ? at<void>(ws, L.a1_scale) : nullptr, w13,
                                 w13_scale, at<void>(ws, L.a2), plan.fp8 ? at<void>(ws, L.a2_scale) : nullptr,
                                 stream);
           if (e != cudaSuccess) return cuda_fail(e, "gemm1");
@@ -427,12 +453,12 @@ int moe_align(const int32_t* topk_ids, int32_t T, int32_t topk, int32_t E, int32
     e = moe::launch_route_align_small(nullptr, topk_ids, T, E, topk, 1, nullptr, nullptr, block_m,
                                       static_cast<int>(cap), sorted_token_ids, expert_ids, num_tokens_post_padded,
                                       expert_counts ? expert_counts : counts, expert_offsets ? expert_offsets : offs,
-                                      status, s);
+                                      status, nullptr, s);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "align");
   }
   e = moe::launch_align(topk_ids, static_cast<int>(n), E, block_m, static_cast<int>(cap), sorted_token_ids,
                         expert_ids, num_tokens_post_padded, counts, offs, scratch, expert_counts, expert_offsets,
-                        status, s);
+                        status, nullptr, s);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "align");
 }
 

@@ -131,6 +131,19 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
       : "memory");
 }
 
+// TMA gather of four rows (tile::gather4): rows y0..y3 of a 2-D tensor map whose
+// box is one row high, x the first column, into 4 consecutive box rows at
+// smem_dst (the 128-byte swizzle follows the shared-memory address, so four
+// rows land exactly as a 4-row slice of a swizzled tile)
+__device__ __forceinline__ void tma_gather4(void* smem_dst, const void* map, uint64_t* bar, int x, int y0, int y1,
+                                            int y2, int y3) {
+  asm volatile(
+      "cp.async.bulk.tensor.2d.shared::cta.global.tile::gather4.mbarrier::complete_tx::bytes"
+      " [%0], [%1, {%3, %4, %5, %6, %7}], [%2];" ::"r"(smem_u32(smem_dst)),
+      "l"(reinterpret_cast<uint64_t>(map)), "r"(smem_u32(bar)), "r"(x), "r"(y0), "r"(y1), "r"(y2), "r"(y3)
+      : "memory");
+}
+
 __device__ __forceinline__ uint64_t policy_evict_first() {
   uint64_t p;
   asm volatile("createpolicy.fractional.L2::evict_first.b64 %0, 1.0;" : "=l"(p));

@@ -124,6 +124,102 @@ cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32
 }
 
 // ----------------------------------------------------------------------------
+// Quantise x once per token (T rows, not T * topk): E4M3 codes into xq [T, H];
+// each (token, K block) scale is written to the sorted rows of the token's
+// topk assignments (pos_of_flat, the inverse of sorted_token_ids) -- fp32
+// a1_scale_t [H/128, capacity] (FP8, rule of vLLM PR #64760 analysis §1.2)
+// or E8M0 bytes in the SF-atom layout of [capacity, H] (MXFP8).  The GEMM1
+// producer gathers the code rows with TMA tile::gather4, so the sorted copy
+// of x never reaches HBM.  row_weight (top-1 only): the row is first
+// bf16(fp32(x) * w).
+// ----------------------------------------------------------------------------
+template <bool MX>
+__global__ void __launch_bounds__(256) quantize_x_kernel(const __nv_bfloat16* x, int T, int H, int topk,
+                                                         const int32_t* pos_of_flat, int capacity,
+                                                         const float* row_weight, uint8_t* xq, void* scales) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int vecs = H / 8;
+  const int iters = (vecs + blockDim.x - 1) / blockDim.x;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    const float rw = row_weight ? (*(row_weight + static_cast<size_t>(t) * topk)) : 1.0f;
+    const __nv_bfloat16* src = x + static_cast<size_t>(t) * H;
+    for (int it = 0; it < iters; ++it) {
+      const int v = it * blockDim.x + threadIdx.x;  // uniform trip count: shuffles see full warps
+      const bool in = v < vecs;
+      uint4 u = make_uint4(0, 0, 0, 0);
+      if (in) u = (*(reinterpret_cast<const uint4*>(src) + v));
+      float f[8];
+      unpack8(u, f);
+      if (row_weight) {
+#pragma unroll
+        for (int i = 0; i < 8; ++i) f[i] = bf16_round(f[i] * rw);
+      }
+      float amax = 0.f;
+#pragma unroll
+      for (int i = 0; i < 8; ++i) amax = fmaxf(amax, fabsf(f[i]));
+#pragma unroll
+      for (int off = (MX ? 2 : 8); off > 0; off >>= 1) amax = fmaxf(amax, __shfl_xor_sync(0xffffffffu, amax, off));
+      const float scale = act_scale_from_amax(amax);
+      const float inv = pow2_recip(scale);
+      uint2 q;
+      q.x = static_cast<uint32_t>(f32x2_to_e4m3x2(f[0] * inv, f[1] * inv)) |
+            (static_cast<uint32_t>(f32x2_to_e4m3x2(f[2] * inv, f[3] * inv)) << 16);
+      q.y = static_cast<uint32_t>(f32x2_to_e4m3x2(f[4] * inv, f[5] * inv)) |
+            (static_cast<uint32_t>(f32x2_to_e4m3x2(f[6] * inv, f[7] * inv)) << 16);
+      if (in) {
+        reinterpret_cast<uint2*>(xq + static_cast<size_t>(t) * H)[v] = q;
+        if ((v & (MX ? 3 : 15)) == 0) {
+          for (int j = 0; j < topk; ++j) {
+            const int r = (*(pos_of_flat + static_cast<size_t>(t) * topk + j));
+            if (r < 0) continue;  // invalid expert id: the assignment has no row
+            if constexpr (MX)
+              static_cast<uint8_t*>(scales)[sf_atom_offset(r, v * 8, H)] = e8m0_of_pow2(scale);
+            else
+              static_cast<float*>(scales)[static_cast<size_t>(v >> 4) * capacity + r] = scale;
+          }
+        }
+      }
+    }
+  }
+}
+
+// bf16 rows scaled by the router weight (top-1): out[t] = bf16(fp32(x[t]) * w[t])
+__global__ void __launch_bounds__(256) scale_rows_kernel(const __nv_bfloat16* x, int T, int H, int topk,
+                                                         const float* row_weight, __nv_bfloat16* out) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int vecs = H / 8;
+  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+    const float rw = (*(row_weight + static_cast<size_t>(t) * topk));
+    for (int v = threadIdx.x; v < vecs; v += blockDim.x) {
+      float f[8];
+      unpack8((*(reinterpret_cast<const uint4*>(x + static_cast<size_t>(t) * H) + v)), f);
+#pragma unroll
+      for (int i = 0; i < 8; ++i) f[i] *= rw;
+      reinterpret_cast<uint4*>(out + static_cast<size_t>(t) * H)[v] = pack8(f);
+    }
+  }
+}
+
+cudaError_t launch_prepare_x(const void* x, int T, int H, int topk, bool fp8, bool mx, const int32_t* pos_of_flat,
+                             int capacity, const float* row_weight, void* xq, void* scales, cudaStream_t stream) {
+  if (T == 0) return cudaSuccess;
+  const int blocks = T < 148 * 8 ? T : 148 * 8;
+  const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
+  if (mx)
+    return launch_pdl(quantize_x_kernel<true>, blocks, 256, 0, stream, xb, T, H, topk, pos_of_flat, capacity,
+                      row_weight, static_cast<uint8_t*>(xq), scales);
+  if (fp8)
+    return launch_pdl(quantize_x_kernel<false>, blocks, 256, 0, stream, xb, T, H, topk, pos_of_flat, capacity,
+                      row_weight, static_cast<uint8_t*>(xq), scales);
+  if (row_weight)
+    return launch_pdl(scale_rows_kernel, blocks, 256, 0, stream, xb, T, H, topk, row_weight,
+                      static_cast<__nv_bfloat16*>(xq));
+  return cudaSuccess;
+}
+
+// ----------------------------------------------------------------------------
 // combine ("Hosting von Qwen auf Blackwell", "MoE Dispatch - Combine": the
 // weighted accumulation; the weights were applied in the GEMM2 epilogue):
 // out[t, :] = bf16(sum_j y[t*topk + j, :]) in fp32, j ascending.

@@ -41,6 +41,7 @@ constexpr int kEpiWarps = 8;
 constexpr int kSmemLimit = 232448;  // max dynamic shared memory per block on sm_100
 constexpr int kSmemReserve = 4096;  // barriers, TMEM slot, exchange buffers
 constexpr int kXchgOffset = 512;    // exchange buffers (2 x 256 floats) start here
+constexpr int kTokRowsOffset = 3072; // token row ids of the current tile (<= 128 int32) for the TMA gather
 
 // wait-site codes reported in the status word (low byte)
 constexpr int kWhereProducer = 1, kWhereMma = 2, kWhereEpiAcc = 3, kWhereEpiXchg = 4, kWhereDrain = 5;
@@ -87,6 +88,8 @@ struct Args {
   float* partials;         // swap-AB split-K: [unit][acc column][128] fp32 partial sums
   int splits;              // swap-AB split-K factor S (1: no split); chosen on the host
   float swiglu_limit;      // GEMM1: SwiGLU clamp limit (+inf: none)
+  int gather_tok;          // GEMM1: token rows are gathered from the [T, K] source by sorted_ids / topk
+  int topk;
   const uint8_t* a_sf;     // MXFP8: E8M0 SF atoms of the activation rows [capacity, K]
   const uint8_t* w_sf;     // MXFP8: E8M0 SF atoms of the weights [E * Nw, K]
   uint8_t* out_sf;         // MXFP8 GEMM1: SF atoms of a2 [capacity, I]
@@ -193,19 +196,29 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_a = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      long long fills = 0;
-      bool ok = true;
-      for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x) {
-        const int tile = unit / splits, split = unit - tile * splits;
-        const int ks0 = split * k_stages / splits, ks1 = (split + 1) * k_stages / splits;
-        const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
+    // All 32 lanes stage the tile's token row ids (GEMM1 gathers token rows
+    // from x or its quantised copy); lane 0 issues every TMA load.
+    int32_t* tok_rows = reinterpret_cast<int32_t*>(reserve + kTokRowsOffset);
+    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_a = policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    long long fills = 0;
+    bool ok = true;
+    for (int unit = blockIdx.x; unit < num_units && ok; unit += gridDim.x) {
+      const int tile = unit / splits, split = unit - tile * splits;
+      const int ks0 = split * k_stages / splits, ks1 = (split + 1) * k_stages / splits;
+      const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
+      const int tok_row = mb * rows_per_block;
+      if (args.gather_tok) {
+        for (int i = lane; i < C::kTokRows; i += 32) {
+          const int f = (*(args.sorted_ids + tok_row + i));
+          tok_rows[i] = f < args.nflat ? f / args.topk : 0;  // padding rows read any valid row
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
         const int e = (*(args.expert_ids + mb));
-        const int tok_row = mb * rows_per_block;
         int w_row0, w_row1;
         if constexpr (kDown) {
           w_row0 = e * H + nt * C::kTileN;
@@ -223,7 +236,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* st = smem + static_cast<size_t>(stage) * C::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
           const int kx = ks * C::kKElems;
-          tma_load_2d(st, &tm_tok, &full[stage], kx, tok_row, pol_a);
+          if (args.gather_tok) {
+#pragma unroll 4
+            for (int g = 0; g < C::kTokRows / 4; ++g) {
+              const int4 r4 = reinterpret_cast<const int4*>(tok_rows)[g];
+              tma_gather4(st + 512 * g, &tm_tok, &full[stage], kx, r4.x, r4.y, r4.z, r4.w);
+            }
+          } else {
+            tma_load_2d(st, &tm_tok, &full[stage], kx, tok_row, pol_a);
+          }
           if constexpr (kDown) {
             tma_load_2d(st + C::kTokBytes, &tm_w, &full[stage], kx, w_row0, pol_w);
           } else {
@@ -237,15 +258,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok) {
-        // let every copy already issued land before the CTA tears down
-        for (int s = 0; s < C::kStages; ++s) {
-          const long long n_s = fills / C::kStages + (s < fills % C::kStages ? 1 : 0);
-          if (n_s > 0) {
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(&full[s], static_cast<uint32_t>((n_s - 1) & 1)) &&
-                   globaltimer_ns() - t0 < kWaitTimeoutNs) {
-            }
+      __syncwarp();  // the row ids are rewritten only after lane 0 issued this tile's loads
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+    if (lane == 0 && !ok) {
+      // let every copy already issued land before the CTA tears down
+      for (int s = 0; s < C::kStages; ++s) {
+        const long long n_s = fills / C::kStages + (s < fills % C::kStages ? 1 : 0);
+        if (n_s > 0) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full[s], static_cast<uint32_t>((n_s - 1) & 1)) &&
+                 globaltimer_ns() - t0 < kWaitTimeoutNs) {
           }
         }
       }
@@ -868,15 +891,25 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
-    if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_a = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      long long fills = 0;
-      bool ok = true;
-      for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
-        const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
+    // All lanes stage the tile's token row ids (GEMM1 gathers code rows of
+    // the per-token quantised x); lane 0 issues every copy.
+    int32_t* tok_rows = reinterpret_cast<int32_t*>(reserve + kTokRowsOffset);
+    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_a = policy_evict_last();
+    int stage = 0;
+    uint32_t phase = 0;
+    long long fills = 0;
+    bool ok = true;
+    for (int tile = blockIdx.x; tile < num_tiles && ok; tile += gridDim.x) {
+      const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
+      if (args.gather_tok) {
+        for (int i = lane; i < 128; i += 32) {
+          const int f = (*(args.sorted_ids + mb * 128 + i));
+          tok_rows[i] = f < args.nflat ? f / args.topk : 0;  // padding rows read any valid row
+        }
+      }
+      __syncwarp();
+      if (lane == 0) {
         const int e = (*(args.expert_ids + mb));
         // weight rows of the two 128-row blocks of this tile (global row index in [E * Nw, K])
         int w_row0, w_row1;
@@ -899,7 +932,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           uint8_t* st = smem + static_cast<size_t>(stage) * C::kStageBytes;
           mbar_arrive_expect_tx(&full[stage], C::kTokBytes + C::kWBytes + 3 * 512);
           const int kx = kb * 128;
-          tma_load_2d(st, &tm_tok, &full[stage], kx, mb * 128, pol_a);
+          if (args.gather_tok) {
+#pragma unroll 4
+            for (int g = 0; g < 32; ++g) {
+              const int4 r4 = reinterpret_cast<const int4*>(tok_rows)[g];
+              tma_gather4(st + 512 * g, &tm_tok, &full[stage], kx, r4.x, r4.y, r4.z, r4.w);
+            }
+          } else {
+            tma_load_2d(st, &tm_tok, &full[stage], kx, mb * 128, pol_a);
+          }
           if constexpr (kDown) {
             tma_load_2d(st + C::kTokBytes, &tm_w, &full[stage], kx, w_row0, pol_w);
           } else {
@@ -916,15 +957,17 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         }
       }
-      if (!ok) {
-        // let every copy already issued land before the CTA tears down
-        for (int s = 0; s < C::kStages; ++s) {
-          const long long n_s = fills / C::kStages + (s < fills % C::kStages ? 1 : 0);
-          if (n_s > 0) {
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(&full[s], static_cast<uint32_t>((n_s - 1) & 1)) &&
-                   globaltimer_ns() - t0 < kWaitTimeoutNs) {
-            }
+      __syncwarp();  // the row ids are rewritten only after lane 0 issued this tile's loads
+      ok = __shfl_sync(0xffffffffu, ok ? 1 : 0, 0) != 0;
+    }
+    if (lane == 0 && !ok) {
+      // let every copy already issued land before the CTA tears down
+      for (int s = 0; s < C::kStages; ++s) {
+        const long long n_s = fills / C::kStages + (s < fills % C::kStages ? 1 : 0);
+        if (n_s > 0) {
+          const uint64_t t0 = globaltimer_ns();
+          while (!mbar_try_wait(&full[s], static_cast<uint32_t>((n_s - 1) & 1)) &&
+                 globaltimer_ns() - t0 < kWaitTimeoutNs) {
           }
         }
       }
@@ -1436,7 +1479,10 @@ cudaError_t launch_on(const GemmProblem& p, const void* tok, const void* w, cons
   const long long K = kDown ? p.I : p.H;
   const long long wrows = kDown ? static_cast<long long>(p.E) * p.H : static_cast<long long>(p.E) * 2 * p.I;
   CUtensorMap tm_tok, tm_w;
-  if (!make_map(&tm_tok, tok, p.capacity, K, elem, C::kTokRows)) return cudaErrorInvalidValue;
+  // GEMM1 gathers token rows (one-row boxes, tile::gather4) from [T, K]; GEMM2 reads sorted a2 tiles
+  if (args.gather_tok ? !make_map(&tm_tok, tok, p.T, K, elem, 1)
+                      : !make_map(&tm_tok, tok, p.capacity, K, elem, C::kTokRows))
+    return cudaErrorInvalidValue;
   if (!make_map(&tm_w, w, wrows, K, elem, kDown ? C::kWRows : 128)) return cudaErrorInvalidValue;
   const int n_tiles = (kDown ? p.H : p.I) / C::kTileN;
   const long long max_tiles = static_cast<long long>(p.capacity / C::kTokRows) * n_tiles;
@@ -1522,7 +1568,8 @@ cudaError_t launch_mx(const GemmProblem& p, const void* tok, const void* w, cons
   const long long K = kDown ? p.I : p.H;
   const long long wrows = kDown ? static_cast<long long>(p.E) * p.H : static_cast<long long>(p.E) * 2 * p.I;
   CUtensorMap tm_tok, tm_w;
-  if (!make_map(&tm_tok, tok, p.capacity, K, 1, 128)) return cudaErrorInvalidValue;
+  if (args.gather_tok ? !make_map(&tm_tok, tok, p.T, K, 1, 1) : !make_map(&tm_tok, tok, p.capacity, K, 1, 128))
+    return cudaErrorInvalidValue;
   if (!make_map(&tm_w, w, wrows, K, 1, kDown ? 256 : 128)) return cudaErrorInvalidValue;
   const int n_tiles = (kDown ? p.H : p.I) / C::kTileN;
   const long long max_tiles = static_cast<long long>(p.capacity / 128) * n_tiles;
@@ -1571,6 +1618,8 @@ cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const void* a1_sc
   args.sorted_ids = p.sorted_ids;
   args.topk_weights = p.weight_on_input ? nullptr : p.topk_weights;
   args.swiglu_limit = p.swiglu_limit;
+  args.gather_tok = p.gather_tok ? 1 : 0;
+  args.topk = p.topk;
   if (p.mx) {
     args.a_sf = static_cast<const uint8_t*>(a1_scale);
     args.w_sf = static_cast<const uint8_t*>(w13_scale);

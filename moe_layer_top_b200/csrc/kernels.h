@@ -37,7 +37,7 @@ inline int align_chunks(long long n) { return static_cast<int>((n + kAlignChunk 
 cudaError_t launch_align(const int32_t* topk_ids, int n, int E, int block_m, int capacity,
                          int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp, int32_t* counts_ws,
                          int32_t* offsets_ws, int32_t* chunk_scratch, int32_t* user_counts,
-                         int32_t* user_offsets, int* status, cudaStream_t stream);
+                         int32_t* user_offsets, int* status, int32_t* pos_of_flat, cudaStream_t stream);
 
 // single-CTA route (optional) + align for small batches
 constexpr int kSmallAlignMaxN = 8192;  // assignments (T * topk)
@@ -46,7 +46,10 @@ bool route_align_small_fits(long long n, int E);
 cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in, int T, int E, int topk,
                                      int renormalize, int32_t* ids_out, float* weights_out, int block_m, int capacity,
                                      int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp, int32_t* counts,
-                                     int32_t* offsets, int* status, cudaStream_t stream);
+                                     int32_t* offsets, int* status, int32_t* pos_of_flat, cudaStream_t stream);
+
+// pos_of_flat (optional, both align paths): sorted position of every flat
+// assignment, -1 for an invalid expert id (the inverse of sorted_token_ids)
 
 // gather x rows into sorted order: bf16 copy, FP8 per-(row,128) quantisation
 // (a1_scale: fp32 [H/128, capacity]) or MXFP8 per-(row,32) quantisation
@@ -55,6 +58,14 @@ cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in,
 cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32_t* sorted_ids,
                           const int32_t* ntpp, int capacity, bool fp8, bool mx, const float* row_weight, void* a1,
                           void* a1_scale, cudaStream_t stream);
+
+// x once per token, for GEMM1's TMA gather of token rows: FP8 / MXFP8 codes
+// into xq [T, H] with each (token, K block) scale scattered to the sorted rows
+// of its assignments (fp32 [H/128, capacity] or E8M0 SF atoms of [capacity, H]);
+// bf16 with a router weight on the input: xq = bf16(x * w) [T, H]; plain bf16:
+// nothing (GEMM1 reads x itself)
+cudaError_t launch_prepare_x(const void* x, int T, int H, int topk, bool fp8, bool mx, const int32_t* pos_of_flat,
+                             int capacity, const float* row_weight, void* xq, void* scales, cudaStream_t stream);
 
 // out[t] = sum_j y[t*topk + j]
 cudaError_t launch_combine(const void* y, int T, int topk, int H, void* out, cudaStream_t stream);
@@ -73,6 +84,8 @@ struct GemmProblem {
   bool fp8, swap;
   bool mx;             // MXFP8 (with fp8): block-scaled MMA, E8M0 SF atoms
   bool weight_on_input;  // the router weight was applied in the gather: GEMM2 stores y unweighted
+  bool gather_tok;     // GEMM1: token rows come from a [T, H] source by sorted_ids / topk (TMA gather)
+  int T;               // rows of that source
   float swiglu_limit;  // SwiGLU clamp limit (+inf: none)
   const int32_t* ntpp;
   const int32_t* expert_ids;

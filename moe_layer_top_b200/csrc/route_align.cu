@@ -220,7 +220,7 @@ __global__ void __launch_bounds__(kAlignWarps * 32) align_scatter_kernel(
     const int32_t* ids, int n, int E, int block_m, int capacity, int nchunks,
     const int32_t* chunk_base, const int32_t* counts_ws, int32_t* sorted_ids,
     int32_t* expert_ids, int32_t* ntpp_out, int32_t* offsets_ws,
-    int32_t* user_offsets) {
+    int32_t* user_offsets, int32_t* pos_of_flat) {
   extern __shared__ int32_t smem_i32[];
   int32_t* offs = smem_i32;                    // [E + 1]
   int32_t* cnt = offs + (E + 1);               // [E]
@@ -291,6 +291,7 @@ __global__ void __launch_bounds__(kAlignWarps * 32) align_scatter_kernel(
         sorted_ids[dest] = f;
         if (lower == 0) run[e] += __popc(same);  // one lane per expert group updates the counter
       }
+      if (pos_of_flat && f < n) pos_of_flat[f] = dest;  // -1 for an invalid id
       __syncwarp();
     }
   }
@@ -315,7 +316,7 @@ __global__ void __launch_bounds__(kAlignWarps * 32) align_scatter_kernel(
 cudaError_t launch_align(const int32_t* topk_ids, int n, int E, int block_m, int capacity, int32_t* sorted_ids,
                          int32_t* expert_ids, int32_t* ntpp, int32_t* counts_ws, int32_t* offsets_ws,
                          int32_t* chunk_scratch, int32_t* user_counts, int32_t* user_offsets, int* status,
-                         cudaStream_t stream) {
+                         int32_t* pos_of_flat, cudaStream_t stream) {
   const int nchunks = align_chunks(n);
   if (nchunks == 0) return cudaSuccess;
   const int threads = kAlignWarps * 32;
@@ -332,7 +333,8 @@ cudaError_t launch_align(const int32_t* topk_ids, int n, int E, int block_m, int
   if (fill_blocks > blocks3) blocks3 = fill_blocks < 296 ? fill_blocks : 296;
   if (blocks3 < blocks) blocks3 = blocks;
   return launch_pdl(align_scatter_kernel, blocks3, threads, smem3, stream, topk_ids, n, E, block_m, capacity,
-                    nchunks, chunk_scratch, counts_ws, sorted_ids, expert_ids, ntpp, offsets_ws, user_offsets);
+                    nchunks, chunk_scratch, counts_ws, sorted_ids, expert_ids, ntpp, offsets_ws, user_offsets,
+                    pos_of_flat);
 }
 
 // ----------------------------------------------------------------------------
@@ -348,7 +350,7 @@ __global__ void __launch_bounds__(1024) route_align_small_kernel(
     const float* logits, const int32_t* ids_in, int T, int E, int topk, int renormalize,
     int32_t* ids_out, float* weights_out, int block_m, int capacity,
     int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp_out,
-    int32_t* counts_out, int32_t* offsets_out, int* status) {
+    int32_t* counts_out, int32_t* offsets_out, int* status, int32_t* pos_of_flat) {
   extern __shared__ int32_t sm_small[];
   __shared__ int32_t warp_sums[32];
   pdl_launch_dependents();
@@ -436,6 +438,7 @@ __global__ void __launch_bounds__(1024) route_align_small_kernel(
       sorted_ids[dest] = i;
       if (lower == 0) hist[warp * E + e] += __popc(same);
     }
+    if (pos_of_flat && i < end) pos_of_flat[i] = dest;  // -1 for an invalid id
     __syncwarp();
   }
   for (int p = tid; p < capacity; p += 1024) {
@@ -462,7 +465,7 @@ bool route_align_small_fits(long long n, int E) { return n > 0 && n <= kSmallAli
 cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in, int T, int E, int topk,
                                      int renormalize, int32_t* ids_out, float* weights_out, int block_m, int capacity,
                                      int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp, int32_t* counts,
-                                     int32_t* offsets, int* status, cudaStream_t stream) {
+                                     int32_t* offsets, int* status, int32_t* pos_of_flat, cudaStream_t stream) {
   const size_t smem = (static_cast<size_t>(T) * topk + 32 * static_cast<size_t>(E) + 2 * static_cast<size_t>(E) + 1) *
                       sizeof(int32_t);
   static bool attr_set[4] = {false, false, false, false};
@@ -473,7 +476,7 @@ cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in,
       attr_set[idx] = true;
     }
     return launch_pdl(kern, 1, 1024, smem, stream, logits, ids_in, T, E, topk, renormalize, ids_out, weights_out,
-                      block_m, capacity, sorted_ids, expert_ids, ntpp, counts, offsets, status);
+                      block_m, capacity, sorted_ids, expert_ids, ntpp, counts, offsets, status, pos_of_flat);
   };
   if (E <= 128) return pick(route_align_small_kernel<4>, 0);
   return pick(route_align_small_kernel<8>, 1);

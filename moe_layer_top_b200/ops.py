@@ -63,7 +63,8 @@ class MoeWorkspaceLayout(ctypes.Structure):
         ("status", ctypes.c_int64), ("topk_ids", ctypes.c_int64), ("topk_weights", ctypes.c_int64),
         ("sorted_token_ids", ctypes.c_int64), ("expert_ids", ctypes.c_int64),
         ("num_tokens_post_padded", ctypes.c_int64), ("expert_counts", ctypes.c_int64),
-        ("expert_offsets", ctypes.c_int64), ("align_scratch", ctypes.c_int64), ("a1", ctypes.c_int64),
+        ("expert_offsets", ctypes.c_int64), ("align_scratch", ctypes.c_int64), ("pos_of_flat", ctypes.c_int64),
+        ("a1", ctypes.c_int64),
         ("a1_scale", ctypes.c_int64), ("a2", ctypes.c_int64), ("a2_scale", ctypes.c_int64), ("y", ctypes.c_int64),
         ("partials", ctypes.c_int64), ("total_bytes", ctypes.c_int64), ("capacity", ctypes.c_int32), ("block_m", ctypes.c_int32),
         ("mode", ctypes.c_int32), ("align_chunks", ctypes.c_int32),
@@ -274,6 +275,7 @@ def workspace_views(p: MoeProblem, ws: torch.Tensor) -> dict:
     cap = L.capacity
     mx = q.weight_dtype == DTYPE_MXFP8_E4M3
     fp8 = q.weight_dtype == DTYPE_FP8_E4M3 or mx
+    a1_rows = q.T if q.mode == MODE_SWAP_AB else cap
 
     def view(off, n, dtype, shape):
         if off < 0:
@@ -290,7 +292,9 @@ def workspace_views(p: MoeProblem, ws: torch.Tensor) -> dict:
         "num_tokens_post_padded": view(L.num_tokens_post_padded, 1, torch.int32, (1,)),
         "expert_counts": view(L.expert_counts, q.E, torch.int32, (q.E,)),
         "expert_offsets": view(L.expert_offsets, q.E + 1, torch.int32, (q.E + 1,)),
-        "a1": view(L.a1, cap * q.H, torch.uint8 if fp8 else torch.bfloat16, (cap, q.H)),
+        # GEMM1 token rows: sorted copy [cap, H] for normal tiles, one row per token [T, H] for swap-AB
+        "a1": view(L.a1, a1_rows * q.H, torch.uint8 if fp8 else torch.bfloat16, (a1_rows, q.H)),
+        "pos_of_flat": view(L.pos_of_flat, nflat, torch.int32, (nflat,)),
         "a1_scale_t": None if mx else view(L.a1_scale, cap * (q.H // 128), torch.float32, (q.H // 128, cap)),
         "a1_sf": view(L.a1_scale, cap * q.H // 32, torch.uint8, (cap * q.H // 32,)) if mx else None,
         "a2": view(L.a2, cap * q.I, torch.uint8 if fp8 else torch.bfloat16, (cap, q.I)),

@@ -42,7 +42,7 @@ def test_library_exports_every_declared_symbol(L):
 
 def test_struct_sizes_match_header():
     assert ctypes.sizeof(ops.MoeProblem) == 16 * 4
-    assert ctypes.sizeof(ops.MoeWorkspaceLayout) == 16 * 8 + 4 * 4
+    assert ctypes.sizeof(ops.MoeWorkspaceLayout) == 17 * 8 + 4 * 4
 
 
 def test_align_capacity_formula(L):
@@ -132,8 +132,10 @@ def test_workspace_layout_is_aligned_and_ordered(L):
         offs = [lay.status, lay.topk_ids, lay.topk_weights, lay.sorted_token_ids, lay.expert_ids,
                 lay.num_tokens_post_padded, lay.expert_counts, lay.expert_offsets, lay.align_scratch, lay.a1,
                 lay.a2, lay.y]
+        offs = [o for o in offs if o >= 0]          # -1: a region this problem does not use
         assert all(o % 256 == 0 for o in offs)
         assert offs == sorted(offs)
+        assert (lay.a1 >= 0) == fp8 and (lay.pos_of_flat >= 0) == fp8   # bf16 GEMM1 gathers from x itself
         assert (lay.a1_scale >= 0) == fp8 and (lay.a2_scale >= 0) == fp8
         assert lay.total_bytes == ops.workspace_size(p)
         assert lay.y + 64 * 8 * 4096 * 2 <= lay.total_bytes

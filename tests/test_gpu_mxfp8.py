@@ -58,11 +58,11 @@ def test_mx_gather_quantises_x_bit_exact():
     sorted_ids = v["sorted_token_ids"][:ntpp].cpu().numpy()
     nflat = 37 * MID_MX.topk
     rows = np.nonzero(sorted_ids < nflat)[0]
-    x = c.x.float().cpu().double().numpy()[sorted_ids[rows] // MID_MX.topk]
-    rc, re8 = O.quantize_mx_group32(x)
-    np.testing.assert_array_equal(v["a1"][:ntpp].cpu().numpy()[rows], rc)
+    tok = sorted_ids[rows] // MID_MX.topk
+    rc, re8 = O.quantize_mx_group32(c.x.float().cpu().double().numpy())
+    np.testing.assert_array_equal(v["a1"][:ntpp].cpu().numpy()[rows], rc[tok])   # sorted copy of the codes
     sf_rows = ops.sf_atoms_to_rows(v["a1_sf"], cap, MID_MX.H).cpu().numpy()
-    np.testing.assert_array_equal(sf_rows[rows], re8)
+    np.testing.assert_array_equal(sf_rows[rows], re8[tok])
 
 
 def test_mx_gemm1_intermediate_matches_oracle():

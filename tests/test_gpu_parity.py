@@ -160,18 +160,28 @@ def test_weight_quantisation_zero_block_and_extremes():
     np.testing.assert_array_equal(scales[0].cpu().numpy(), rs)
 
 
-def test_gather_quantises_x_bit_exact():
-    c = Case(MID_FP8, 37, seed=3, mode=ops.MODE_NORMAL)
+@pytest.mark.parametrize("mode,bm", [(ops.MODE_NORMAL, 128), (ops.MODE_SWAP_AB, 32), (ops.MODE_NORMAL, 256)])
+def test_gather_quantises_x_bit_exact(mode, bm):
+    """Swap-AB: x is quantised once per token ([T, H] codes) and each scale lands
+    on the sorted rows of the token's assignments.  Normal tiles: a sorted copy."""
+    c = Case(MID_FP8, 37, seed=3, mode=mode, block_m=bm)
     c.run()
     v = c.views()
     ntpp = int(v["num_tokens_post_padded"].item())
     sorted_ids = v["sorted_token_ids"][:ntpp].cpu().numpy()
     nflat = 37 * MID_FP8.topk
     rows = np.nonzero(sorted_ids < nflat)[0]
-    x = c.x.float().cpu().double().numpy()[sorted_ids[rows] // MID_FP8.topk]
+    tok = sorted_ids[rows] // MID_FP8.topk
+    x = c.x.float().cpu().double().numpy()
     rc, rs = O.quantize_act_group128(x)
-    np.testing.assert_array_equal(v["a1"][:ntpp].cpu().numpy()[rows], rc)
-    np.testing.assert_array_equal(v["a1_scale_t"][:, :ntpp].cpu().numpy().T[rows], rs)
+    if mode == ops.MODE_NORMAL:
+        np.testing.assert_array_equal(v["a1"][:ntpp].cpu().numpy()[rows], rc[tok])
+    else:
+        np.testing.assert_array_equal(v["a1"].cpu().numpy(), rc)
+        pos = v["pos_of_flat"].cpu().numpy()
+        np.testing.assert_array_equal(np.sort(pos), np.sort(rows))           # inverse of sorted_token_ids
+        np.testing.assert_array_equal(sorted_ids[pos], np.arange(nflat))
+    np.testing.assert_array_equal(v["a1_scale_t"][:, :ntpp].cpu().numpy().T[rows], rs[tok])
 
 
 # ----------------------------------------------------------------------------- layer output
@@ -339,14 +349,16 @@ def test_router_weight_on_input(cfg, T, mode, bm):
     assert c.status() == ops.MOE_STATUS_OK
     ref = c.oracle()
     assert_close(out.float().cpu().numpy(), ref["out"], fp8=cfg.fp8)
-    if not cfg.fp8:   # the gathered bf16 rows are bf16(fp32(x) * w) exactly
+    if not cfg.fp8:   # GEMM1's token rows are bf16(fp32(x) * w) exactly
         v = c.views()
-        ntpp = int(v["num_tokens_post_padded"].item())
-        ids = v["sorted_token_ids"][:ntpp].cpu().numpy()
-        rows = np.nonzero(ids < T)[0]
-        w = v["topk_weights"].cpu().numpy()[ids[rows], 0]
-        xs = (c.x.float()[torch.from_numpy(ids[rows]).cuda()] * torch.from_numpy(w).cuda()[:, None]).bfloat16()
-        assert torch.equal(v["a1"][:ntpp][torch.from_numpy(rows).cuda()], xs)
+        scaled = (c.x.float() * v["topk_weights"][:, 0][:, None]).bfloat16()
+        if c.q.mode == ops.MODE_SWAP_AB:            # one row per token
+            assert torch.equal(v["a1"], scaled)
+        else:                                       # sorted copy
+            ntpp = int(v["num_tokens_post_padded"].item())
+            ids = v["sorted_token_ids"][:ntpp]
+            rows = torch.nonzero(ids < T).flatten()
+            assert torch.equal(v["a1"][rows], scaled[ids[rows].long()])
 
 
 @pytest.mark.parametrize("cfg,T,mode,bm", [(MID_BF16, 7, ops.MODE_SWAP_AB, 16), (MID_BF16, 300, ops.MODE_NORMAL, 128),
