@@ -103,7 +103,9 @@ extern "C" {
  * mode = MOE_MODE_AUTO and block_m = 0 let the library choose; both are
  * written back by moe_resolve_problem().
  * Constraints: T >= 0, 1 <= topk <= E <= 1024, H and I positive multiples of
- * 128, T * topk < 2^31.
+ * 128, T * topk < 2^31.  Normal tiles (and so MXFP8) cover 256 columns of H
+ * per GEMM2 tile and need H % 256 == 0; MOE_MODE_AUTO picks swap-AB tiles
+ * when H % 256 == 128.
  */
 typedef struct moe_problem {
   int32_t T;            /* tokens */

@@ -88,8 +88,12 @@ int validate_problem(const moe_problem* p) {
   if (!(p->swiglu_limit >= 0.0f) || p->swiglu_limit == INFINITY)
     return fail(MOE_ERR_INVALID, "swiglu_limit must be 0 (off) or a positive finite value");
   const bool fp8 = p->weight_dtype == MOE_DTYPE_FP8_E4M3;
+  // normal tiles cover 256 output columns of GEMM2 at a time
+  if ((p->mode == MOE_MODE_NORMAL || (p->mode == MOE_MODE_AUTO && p->block_m >= 128)) && p->H % 256)
+    return fail(MOE_ERR_INVALID, "normal tiles need H %% 256 == 0 (H = %d); use swap-AB", p->H);
   if (p->weight_dtype == MOE_DTYPE_MXFP8_E4M3) {
     if (p->mode == MOE_MODE_SWAP_AB) return fail(MOE_ERR_UNSUPPORTED, "MXFP8 weights run normal tiles only");
+    if (p->H % 256) return fail(MOE_ERR_UNSUPPORTED, "MXFP8 weights need H %% 256 == 0 (H = %d)", p->H);
     if (p->block_m != 0 && p->block_m != 128)
       return fail(MOE_ERR_INVALID, "MXFP8 weights use block_m = 128 (got %d)", p->block_m);
   }
@@ -120,7 +124,7 @@ void resolve(moe_problem* p) {
   if (p->mode == MOE_MODE_AUTO) {
     if (p->block_m >= 128)
       p->mode = MOE_MODE_NORMAL;
-    else if (p->block_m != 0)
+    else if (p->block_m != 0 || p->H % 256)  // normal tiles need H % 256 == 0
       p->mode = MOE_MODE_SWAP_AB;
     else
       p->mode = avg <= 40.0 ? MOE_MODE_SWAP_AB : MOE_MODE_NORMAL;

@@ -59,8 +59,9 @@ class Case:
     """One workload instance on the GPU plus its oracle evaluation."""
 
     def __init__(self, cfg: inputs.MoEConfig, T: int, seed: int = 0, mode=ops.MODE_AUTO, block_m=0,
-                 weights=None, split_k=True, router_weight_on_input=False, swiglu_limit=0.0):
+                 weights=None, split_k=True, router_weight_on_input=False, swiglu_limit=0.0, renormalize=True):
         self.cfg, self.T, self.seed = cfg, T, seed
+        self.renormalize = renormalize
         self.router_weight_on_input, self.swiglu_limit = router_weight_on_input, swiglu_limit
         dev = torch.device("cuda")
         if weights is None:
@@ -79,7 +80,7 @@ class Case:
             self.w13_scale = self.w2_scale = None
         self.p = ops.problem(T, cfg.E, cfg.topk, cfg.H, cfg.I, fp8=cfg.fp8, mode=mode, block_m=block_m,
                              split_k=split_k, mx=cfg.mx, router_weight_on_input=router_weight_on_input,
-                             swiglu_limit=swiglu_limit)
+                             swiglu_limit=swiglu_limit, renormalize=renormalize)
         self.q = ops.resolve_problem(self.p)
         self.ws = ops.alloc_workspace(self.p)
         self.out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
@@ -106,6 +107,7 @@ class Case:
             kw["topk_ids"] = self.routing["topk_ids"].cpu().numpy()
             kw["topk_weights"] = self.routing["topk_weights"].cpu().numpy()
         kw["router_weight_on_input"] = self.router_weight_on_input
+        kw["renormalize"] = self.renormalize
         kw["swiglu_limit"] = self.swiglu_limit if self.swiglu_limit > 0 else None
         l13 = LazyExperts(self.w13_bf16, self.cfg.fp8, self.cfg.mx)
         l2 = LazyExperts(self.w2_bf16, self.cfg.fp8, self.cfg.mx)

@@ -84,6 +84,15 @@ def test_resolve_problem_mxfp8_is_normal_128(L):
     assert lay_mx.total_bytes == lay_f8.total_bytes and lay_mx.a1_scale >= 0 and lay_mx.a2_scale >= 0
 
 
+def test_normal_tiles_need_h_multiple_of_256(L):
+    q = ops.resolve_problem(ops.problem(16384, 8, 2, 384, 128))          # many tokens, but H % 256 == 128
+    assert q.mode == ops.MODE_SWAP_AB
+    for kw in (dict(mode=ops.MODE_NORMAL), dict(block_m=128), dict(mx=True)):
+        p = ops.problem(64, 8, 2, 384, 128, **kw)
+        assert L.moe_workspace_size(ctypes.byref(p)) == 0
+    assert L.moe_workspace_size(ctypes.byref(ops.problem(64, 8, 2, 512, 128, mode=ops.MODE_NORMAL))) > 0
+
+
 def test_epilogue_variant_validation(L):
     ok = ops.problem(16, 8, 1, 256, 128, router_weight_on_input=True)
     assert L.moe_workspace_size(ctypes.byref(ok)) > 0
