@@ -105,6 +105,15 @@ __device__ __forceinline__ void pdl_launch_dependents() {
 
 __device__ __forceinline__ void pdl_wait() { asm volatile("griddepcontrol.wait;" ::: "memory"); }
 
+// L2-coherent load (bypasses L1).  Used only for data that a kernel two or
+// more launches back wrote, read before griddepcontrol.wait by a kernel whose
+// predecessor triggered its launch only after its own wait.
+__device__ __forceinline__ int ld_cg_i32(const int32_t* p) {
+  int v;
+  asm volatile("ld.global.cg.s32 %0, [%1];" : "=r"(v) : "l"(p) : "memory");
+  return v;
+}
+
 // --------------------------------------------------------------------------
 // TMA (cp.async.bulk.tensor), no multicast
 // --------------------------------------------------------------------------

@@ -155,7 +155,7 @@ __global__ void __launch_bounds__(kThreads, 1)
   float* xchg = reinterpret_cast<float*>(reserve + kXchgOffset);  // [2][2 * 128] floats
 
   const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  pdl_launch_dependents();
+  if constexpr (kDown) pdl_launch_dependents();  // GEMM1 triggers only after its own wait (below)
   if (threadIdx.x == 0) {
     for (int s = 0; s < C::kStages; ++s) {
       mbar_init(&full[s], 1);
@@ -182,13 +182,19 @@ __global__ void __launch_bounds__(kThreads, 1)
   __syncthreads();
   tc_fence_after();
   const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();  // everything above overlapped the previous kernel's tail
+  // GEMM1 waits here, then lets GEMM2 launch: GEMM2 may then read the alignment
+  // (written two or more launches back) before its own wait and start streaming
+  // its weights under GEMM1's tail.  GEMM2 waits per role.
+  if constexpr (!kDown) {
+    pdl_wait();
+    pdl_launch_dependents();
+  }
 
   const int H = args.H, I = args.I;
   const int K = kDown ? I : H;                           // reduction length
   const int rows_per_block = C::kTokRows;                // == block_m of the alignment
   const int n_tiles = (kDown ? H : I) / C::kTileN;
-  const int num_mblocks = (*(args.ntpp)) / rows_per_block;
+  const int num_mblocks = (kDown ? ld_cg_i32(args.ntpp) : (*(args.ntpp))) / rows_per_block;
   const int num_tiles = num_mblocks * n_tiles;
   const int k_stages = K / C::kKElems;
   const int splits = kSwap ? args.splits : 1;
@@ -196,6 +202,84 @@ __global__ void __launch_bounds__(kThreads, 1)
 
   if (warp == 0) {
     // ------------------------------------------------------------------ producer
+    if constexpr (kDown) {
+      // GEMM2: the weight tiles of the first kStages fills are issued before the
+      // wait (they depend only on the alignment); the a2 tiles follow after it.
+      if (lane == 0) {
+        const uint64_t pol_w = policy_evict_first();
+        const uint64_t pol_a = policy_evict_last();
+        int stage = 0;
+        uint32_t phase = 0;
+        long long fills = 0;
+        bool ok = true;
+        int unit = static_cast<int>(blockIdx.x) - static_cast<int>(gridDim.x);
+        int ks = 0, ks_end = 0, tok_row = 0, w_row = 0;
+        auto advance = [&]() -> bool {  // next (unit, K stage) of this CTA
+          if (ks + 1 < ks_end) {
+            ++ks;
+            return true;
+          }
+          unit += static_cast<int>(gridDim.x);
+          if (unit >= num_units) return false;
+          const int tile = unit / splits, split = unit - tile * splits;
+          ks = split * k_stages / splits;
+          ks_end = (split + 1) * k_stages / splits;
+          const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
+          tok_row = mb * rows_per_block;
+          w_row = ld_cg_i32(args.expert_ids + mb) * H + nt * C::kTileN;
+          return ks < ks_end;
+        };
+        int pre_kx[C::kStages], pre_row[C::kStages];
+        int npre = 0;
+        bool more = true;
+        while (npre < C::kStages && (more = advance())) {
+          uint8_t* st = smem + static_cast<size_t>(stage) * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          const int kx = ks * C::kKElems;
+          tma_load_2d(st + C::kTokBytes, &tm_w, &full[stage], kx, w_row, pol_w);
+          pre_kx[npre] = kx;
+          pre_row[npre] = tok_row;
+          ++npre;
+          ++fills;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        pdl_wait();  // a2 (GEMM1's output) is complete from here on
+        for (int i = 0; i < npre; ++i)
+          tma_load_2d(smem + static_cast<size_t>(i) * C::kStageBytes, &tm_tok, &full[i], pre_kx[i], pre_row[i],
+                      pol_a);
+        while (more && ok && (more = advance())) {
+          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status,
+                         MOE_STATUS_WAIT_TIMEOUT | kWhereProducer)) {
+            ok = false;
+            break;
+          }
+          uint8_t* st = smem + static_cast<size_t>(stage) * C::kStageBytes;
+          mbar_arrive_expect_tx(&full[stage], C::kStageBytes);
+          const int kx = ks * C::kKElems;
+          tma_load_2d(st, &tm_tok, &full[stage], kx, tok_row, pol_a);
+          tma_load_2d(st + C::kTokBytes, &tm_w, &full[stage], kx, w_row, pol_w);
+          ++fills;
+          if (++stage == C::kStages) {
+            stage = 0;
+            phase ^= 1u;
+          }
+        }
+        if (!ok) {
+          for (int s = 0; s < C::kStages; ++s) {
+            const long long n_s = fills / C::kStages + (s < fills % C::kStages ? 1 : 0);
+            if (n_s > 0) {
+              const uint64_t t0 = globaltimer_ns();
+              while (!mbar_try_wait(&full[s], static_cast<uint32_t>((n_s - 1) & 1)) &&
+                     globaltimer_ns() - t0 < kWaitTimeoutNs) {
+              }
+            }
+          }
+        }
+      }
+    } else {
     // All 32 lanes stage the tile's token row ids (GEMM1 gathers token rows
     // from x or its quantised copy); lane 0 issues every TMA load.
     int32_t* tok_rows = reinterpret_cast<int32_t*>(reserve + kTokRowsOffset);
@@ -273,8 +357,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    }  // GEMM1 producer
   } else if (warp == 1) {
     // ------------------------------------------------------------------ MMA issuer
+    if constexpr (kDown) pdl_wait();
     if (lane == 0) {
       constexpr uint32_t idesc = make_idesc(128, C::kMmaN, kFP8);
       int stage = 0, abuf = 0;
@@ -360,6 +446,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     }
   } else {
     // ------------------------------------------------------------------ epilogue
+    if constexpr (kDown) pdl_wait();
     const int q = warp & 3;                 // TMEM lane quarter this warp may access
     const int g = (warp - 2) >> 2;          // epilogue group
     const int row = 32 * q + lane;          // accumulator row (TMEM lane)
