@@ -144,7 +144,7 @@ typedef struct moe_workspace_layout {
   int64_t expert_counts;    /* int32 [E] */
   int64_t expert_offsets;   /* int32 [E + 1] */
   int64_t align_scratch;    /* int32 [chunks * E] */
-  int64_t pos_of_flat;      /* int32 [T*topk]: sorted row of each assignment, -1 for a bad id (swap-AB FP8) */
+  int64_t pos_of_flat;      /* int32 [T*topk]: sorted row of each assignment, -1 for a bad id (FP8 / MXFP8) */
   int64_t a1;               /* GEMM1 token rows.  Normal tiles: x rows in sorted order [capacity, H], bf16 or
                                E4M3 (padding rows unspecified).  Swap-AB: one row per token [T, H] -- E4M3
                                codes (FP8) or bf16(x * w) (router weight on the input) -- gathered by TMA;

@@ -196,7 +196,7 @@ int make_plan(const moe_problem* in, Plan* plan) {
     L.a1 = take(static_cast<int64_t>(p.T) * p.H * elem);
   else
     L.a1 = -1;
-  L.pos_of_flat = (plan->fp8 && plan->tok_gather) ? take(plan->nflat * 4) : -1;
+  L.pos_of_flat = (plan->fp8 && !plan->pair) ? take(plan->nflat * 4) : -1;
   // FP8: fp32 [K/128, cap]; MXFP8: E8M0 SF atoms, (cap/128) * (K/128) * 512 bytes -- the same size
   L.a1_scale = plan->fp8 ? take(cap * (p.H / 128) * 4) : -1;
   L.a2 = take(cap * p.I * elem);
@@ -307,7 +307,17 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
         if (e != cudaSuccess) return cuda_fail(e, "align");
         break;
       case MOE_STAGE_GATHER:
-        if (!plan.tok_gather)
+        if (!plan.tok_gather && plan.fp8 && !plan.pair) {
+          // normal FP8 / MXFP8 tiles: quantise once per token into the (not yet used)
+          // y region, scattering the scales to the sorted rows, then copy code rows
+          void* xq = at<void>(ws, L.y);
+          e = moe::launch_prepare_x(x, p.T, p.H, p.topk, true, plan.mx, pos, cap,
+                                    p.router_weight_on_input == 1 ? wts : nullptr, xq, at<void>(ws, L.a1_scale),
+                                    stream);
+          if (e == cudaSuccess)
+            e = moe::launch_copy_rows(xq, p.H, p.topk, nflat, at<int32_t>(ws, L.sorted_token_ids),
+                                      at<int32_t>(ws, L.num_tokens_post_padded), cap, at<void>(ws, L.a1), stream);
+        } else if (!plan.tok_gather)
           e = moe::launch_gather(x, p.H, p.topk, nflat, at<int32_t>(ws, L.sorted_token_ids),
                                  at<int32_t>(ws, L.num_tokens_post_padded), cap, plan.fp8, plan.mx,
                                  p.router_weight_on_input == 1 ? wts : nullptr, at<void>(ws, L.a1),

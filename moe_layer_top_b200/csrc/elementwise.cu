@@ -202,6 +202,36 @@ __global__ void __launch_bounds__(256) scale_rows_kernel(const __nv_bfloat16* x,
   }
 }
 
+// ----------------------------------------------------------------------------
+// Sorted copy of quantised rows: a1[r] = xq[sorted_ids[r] / topk] (E4M3 bytes)
+// for the real rows r < ntpp.  With the per-token quantiser in front, x is
+// read and quantised once per token instead of once per assignment; this
+// copy then reads the L2-resident codes.
+// ----------------------------------------------------------------------------
+__global__ void __launch_bounds__(256) copy_rows_kernel(const uint8_t* xq, int H, int topk, int nflat,
+                                                        const int32_t* sorted_ids, const int32_t* ntpp_ptr,
+                                                        uint8_t* a1) {
+  pdl_launch_dependents();
+  pdl_wait();
+  const int ntpp = *ntpp_ptr;
+  const int vecs = H / 16;
+  for (int row = blockIdx.x; row < ntpp; row += gridDim.x) {
+    const int flat = (*(sorted_ids + row));
+    if (flat >= nflat) continue;  // padding rows are never stored
+    const uint4* src = reinterpret_cast<const uint4*>(xq + static_cast<size_t>(flat / topk) * H);
+    uint4* dst = reinterpret_cast<uint4*>(a1 + static_cast<size_t>(row) * H);
+    for (int v = threadIdx.x; v < vecs; v += blockDim.x) dst[v] = (*(src + v));
+  }
+}
+
+cudaError_t launch_copy_rows(const void* xq, int H, int topk, int nflat, const int32_t* sorted_ids,
+                             const int32_t* ntpp, int capacity, void* a1, cudaStream_t stream) {
+  if (capacity == 0) return cudaSuccess;
+  const int blocks = capacity < 148 * 8 ? capacity : 148 * 8;
+  return launch_pdl(copy_rows_kernel, blocks, 256, 0, stream, static_cast<const uint8_t*>(xq), H, topk, nflat,
+                    sorted_ids, ntpp, static_cast<uint8_t*>(a1));
+}
+
 cudaError_t launch_prepare_x(const void* x, int T, int H, int topk, bool fp8, bool mx, const int32_t* pos_of_flat,
                              int capacity, const float* row_weight, void* xq, void* scales, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
