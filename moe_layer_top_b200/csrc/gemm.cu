@@ -1,6 +1,6 @@
 // Grouped expert GEMMs on the 5th-generation tensor cores (tcgen05, sm_100a).
 //
-// GEMM1 (gate/up):  h[r, :] = a1[r, :] . w13[e(r)]^T, followed in the epilogue
+// GEMM1 (gate/up):  h[r, :] = x(r) . w13[e(r)]^T, followed in the epilogue
 //   by a2 = bf16(bf16(silu(gate)) * up) and, on the FP8 path, the per-(row,128)
 //   power-of-two E4M3 re-quantisation (vLLM PR #64760 analysis, §1.2: the
 //   fused SiLU-mul-quant kernel, here fused into the GEMM epilogue so the bf16
@@ -18,7 +18,10 @@
 //            decode batches, where the token count cannot fill the MMA M.
 //
 // Kernel structure (one CTA per SM, persistent over tiles, 10 warps):
-//   warp 0     : TMA producer (one lane), multi-stage smem ring;
+//   warp 0     : TMA producer (one lane issues; for swap-AB GEMM1 the whole
+//                warp first stages the tile's token row ids, which the lane
+//                then gathers with tile::gather4 from x or its per-token FP8
+//                copy), multi-stage smem ring;
 //   warp 1     : TMEM allocator and MMA issuer (one lane);
 //   warps 2..9 : epilogue, two groups of four warps (each group covers the
 //                128 TMEM lanes; the groups split the accumulator columns).
@@ -26,7 +29,12 @@
 // tiles).  FP8: weights carry one fp32 scale per 128x128 block and activations
 // one power-of-two scale per (row, 128); every 128-deep K block accumulates
 // into its own TMEM buffer (double-buffered) and the epilogue promotes it into
-// fp32 registers with the product of the two scales.
+// fp32 registers with the product of the two scales.  MXFP8 (separate kernel
+// below): E8M0 scales per 32 elements applied inside block-scaled MMAs.
+// Launch chain: GEMM1 lets GEMM2 launch only after its own dependency wait,
+// so GEMM2 streams its first weight stages before waiting on GEMM1.  Swap-AB
+// problems with at most half as many tiles as SMs split K; a reduce kernel
+// adds the splits.
 #include <cudaTypedefs.h>
 
 #include "common.cuh"
