@@ -56,6 +56,8 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--persistent-decode", action="store_true",
+                    help="small bf16 batches: the whole layer in one persistent cooperative launch (opt-in)")
     return ap.parse_args()
 
 
@@ -202,7 +204,7 @@ def workload_config(args):
 
 
 class Workload:
-    def __init__(self, cfg, T, seed, weights):
+    def __init__(self, cfg, T, seed, weights, persistent_decode=False):
         from moe_layer_top_b200 import ops
         self.ops = ops
         self.cfg, self.T = cfg, T
@@ -210,7 +212,8 @@ class Workload:
         self.w13, self.w2, self.s13, self.s2 = weights
         self.x = inputs.make_tokens(cfg, T, seed, device=dev)
         self.routing = inputs.make_routing(cfg, T, seed, device=dev)
-        self.p = ops.problem(T, cfg.E, cfg.topk, cfg.H, cfg.I, fp8=cfg.fp8, mx=cfg.mx)
+        self.p = ops.problem(T, cfg.E, cfg.topk, cfg.H, cfg.I, fp8=cfg.fp8, mx=cfg.mx,
+                             persistent_decode=persistent_decode)
         self.q = ops.resolve_problem(self.p)
         self.ws = ops.alloc_workspace(self.p)
         self.out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
@@ -518,7 +521,7 @@ def run_ours(args, rank, world, local):
     results = {}
     with ClockSampler(local) as clocks:
         for T in sweep_T:
-            wl = Workload(cfg, T, args.seed, weights)
+            wl = Workload(cfg, T, args.seed, weights, args.persistent_decode)
             steps = args.steps if T == T_head else max(3, args.steps // 2)
             step_ms, per_stage, wall, n_kernels = time_steps(wl, steps, args.warmup, flush, world)
             total_ms = max_over_ranks(float(step_ms.sum()), world)
@@ -585,7 +588,8 @@ def run_ours(args, rank, world, local):
                    "weights": ("mxfp8 e4m3 + per-32 e8m0 scales" if cfg.mx else "fp8 e4m3 + 128x128 fp32 scales")
                    if cfg.fp8 else "bf16",
                    "routing": cfg.routing, "l2": "flushed (256 MiB write) before every step, outside the timing",
-                   "launch": "CUDA graph of moe_fused_forward (PDL between kernels)",
+                   "launch": ("CUDA graph of moe_fused_forward (persistent decode kernel where eligible)"
+                              if args.persistent_decode else "CUDA graph of moe_fused_forward (PDL between kernels)"),
                    "layer_bytes_per_step": alg["layer_bytes"], "hit_experts": alg["hit_experts"]},
         "roofline": roofline,
         "layer_hbm_frac": round(alg["layer_bytes"] / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4),

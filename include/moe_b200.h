@@ -126,7 +126,12 @@ typedef struct moe_problem {
    * SiLU(gate) * up (the clamp_limit that the PR analysis' sorted-A predicate
    * excludes).  0 = no clamp (default). */
   float swiglu_limit;
-  int32_t reserved[4];  /* must be zero */
+  /* moe_fused_forward of a small bf16 batch (T * topk <= 256, E <= 256, swap-AB
+   * block_m 16, weights on the output): 1 = the whole layer in one persistent
+   * cooperative launch, 0 = the kernel-per-stage pipeline (default: measured
+   * faster, the persistent kernel is opt-in). */
+  int32_t persistent_decode;
+  int32_t reserved[3];  /* must be zero */
 } moe_problem;
 
 /*

@@ -79,8 +79,10 @@ int validate_problem(const moe_problem* p) {
   if (p->mode < MOE_MODE_AUTO || p->mode > MOE_MODE_SWAP_AB) return fail(MOE_ERR_INVALID, "mode %d", p->mode);
   if (p->renormalize != 0 && p->renormalize != 1) return fail(MOE_ERR_INVALID, "renormalize must be 0 or 1");
   if (p->split_k != 0 && p->split_k != 1) return fail(MOE_ERR_INVALID, "split_k must be 0 or 1");
-  for (int i = 0; i < 4; ++i)
+  for (int i = 0; i < 3; ++i)
     if (p->reserved[i] != 0) return fail(MOE_ERR_INVALID, "reserved fields must be zero");
+  if (p->persistent_decode != 0 && p->persistent_decode != 1)
+    return fail(MOE_ERR_INVALID, "persistent_decode must be 0 or 1");
   if (p->router_weight_on_input != 0 && p->router_weight_on_input != 1)
     return fail(MOE_ERR_INVALID, "router_weight_on_input must be 0 or 1");
   if (p->router_weight_on_input == 1 && p->topk != 1)
@@ -267,6 +269,46 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
   const void* tok_src = L.a1 >= 0 ? at<void>(ws, L.a1) : x;
   bool aligned_already = false;
   cudaError_t e;
+
+  // the whole layer of a small bf16 batch in one persistent cooperative launch
+  if (stage_begin == 0 && stage_end == MOE_NUM_STAGES && p.persistent_decode == 1 && !plan.fp8 && swap &&
+      p.block_m == moe::kDecodeBlockM && p.router_weight_on_input == 0 &&
+      moe::decode_fused_fits(p.T, p.E, p.topk, p.H, p.I)) {
+    int* sync = at<int>(ws, L.partials);  // the split-K buffer is not used by this path
+    if ((e = cudaMemsetAsync(status, 0, sizeof(int), stream)) != cudaSuccess ||
+        (e = cudaMemsetAsync(sync, 0, moe::kDecodeSyncInts * sizeof(int), stream)) != cudaSuccess)
+      return cuda_fail(e, "clear sync words");
+    moe::DecodeProblem dp{};
+    dp.T = p.T;
+    dp.E = p.E;
+    dp.topk = p.topk;
+    dp.H = p.H;
+    dp.I = p.I;
+    dp.renormalize = p.renormalize;
+    dp.capacity = cap;
+    dp.swiglu_limit = p.swiglu_limit > 0.0f ? p.swiglu_limit : INFINITY;
+    dp.logits = logits;
+    dp.ids_in = logits ? nullptr : topk_ids;
+    dp.weights_in = logits ? nullptr : topk_weights;
+    dp.x = x;
+    dp.w13 = w13;
+    dp.w2 = w2;
+    dp.topk_ids = at<int32_t>(ws, L.topk_ids);
+    dp.topk_weights = at<float>(ws, L.topk_weights);
+    dp.sorted_ids = at<int32_t>(ws, L.sorted_token_ids);
+    dp.expert_ids = at<int32_t>(ws, L.expert_ids);
+    dp.ntpp = at<int32_t>(ws, L.num_tokens_post_padded);
+    dp.counts = at<int32_t>(ws, L.expert_counts);
+    dp.offsets = at<int32_t>(ws, L.expert_offsets);
+    dp.a2 = at<void>(ws, L.a2);
+    dp.y = at<void>(ws, L.y);
+    dp.out = out;
+    dp.sync = sync;
+    dp.status = status;
+    dp.num_sms = sms;
+    e = moe::launch_decode_fused(dp, stream);
+    return e == cudaSuccess ? MOE_OK : cuda_fail(e, "persistent decode");
+  }
 
   for (int s = stage_begin; s < stage_end; ++s) {
     switch (s) {

@@ -1700,6 +1700,11 @@ size_t smem_of() {
 
 }  // namespace
 
+bool make_tma_map_2d(CUtensorMap* map, const void* base, long long rows, long long cols, int elem_bytes,
+                     int box_rows) {
+  return make_map(map, base, rows, cols, elem_bytes, box_rows);
+}
+
 cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const void* a1_scale, const void* w13,
                          const void* w13_scale, void* a2, void* a2_scale, cudaStream_t stream) {
   Args args{};

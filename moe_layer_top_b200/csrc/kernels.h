@@ -1,6 +1,7 @@
 // Host-side launchers of the MoE kernels (internal to the library).
 #pragma once
 
+#include <cuda.h>
 #include <cuda_runtime.h>
 #include <stdint.h>
 #include <stddef.h>
@@ -116,6 +117,43 @@ cudaError_t launch_gemm1(const GemmProblem& p, const void* a1, const void* a1_sc
 // swap-AB split-K launches the reduce kernel after it, as for GEMM1
 cudaError_t launch_gemm2(const GemmProblem& p, const void* a2, const void* a2_scale, const void* w2,
                          const void* w2_scale, void* y, cudaStream_t stream);
+
+// 2-D K-major TMA tensor map: [rows, cols] elements of elem_bytes, box = 128
+// bytes x box_rows, 128-byte swizzle (box_rows = 1 for tile::gather4 maps)
+bool make_tma_map_2d(CUtensorMap* map, const void* base, long long rows, long long cols, int elem_bytes,
+                     int box_rows);
+
+// persistent decode kernel (route + align + GEMM1 + GEMM2 + combine in one
+// cooperative launch) for small bf16 batches; see decode_fused.cu
+struct DecodeProblem {
+  int T, E, topk, H, I, renormalize, capacity;
+  float swiglu_limit;  // +inf: none
+  const float* logits;             // [T, E] or NULL
+  const int32_t* ids_in;           // [T, topk] when logits == NULL
+  const float* weights_in;         // [T, topk] when logits == NULL
+  const void* x;                   // [T, H] bf16
+  const void* w13;                 // [E, 2I, H] bf16
+  const void* w2;                  // [E, H, I] bf16
+  int32_t* topk_ids;               // router output [T, topk]
+  float* topk_weights;             // router output [T, topk]
+  int32_t* sorted_ids;             // [capacity]
+  int32_t* expert_ids;             // [capacity / 16]
+  int32_t* ntpp;
+  int32_t* counts;                 // [E]
+  int32_t* offsets;                // [E + 1]
+  void* a2;                        // [capacity, I] bf16
+  void* y;                         // [T * topk, H] bf16
+  void* out;                       // [T, H] bf16
+  int* sync;                       // kDecodeSyncInts ints, zeroed before the launch
+  int* status;
+  int num_sms;
+};
+constexpr int kDecodeMaxAssignments = 256;   // T * topk
+constexpr int kDecodeMaxExperts = 256;
+constexpr int kDecodeBlockM = 16;
+constexpr int kDecodeSyncInts = 8 + kDecodeMaxAssignments + kDecodeMaxExperts;  // flags + ready[block]
+bool decode_fused_fits(int T, int E, int topk, int H, int I);
+cudaError_t launch_decode_fused(const DecodeProblem& p, cudaStream_t stream);
 
 // failure-detection self-test: one bounded wait that must time out
 cudaError_t launch_wait_selftest(int* status, unsigned long long timeout_ns, unsigned long long* waited_ns,

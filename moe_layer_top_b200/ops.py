@@ -54,7 +54,7 @@ class MoeProblem(ctypes.Structure):
         ("I", ctypes.c_int32), ("weight_dtype", ctypes.c_int32), ("mode", ctypes.c_int32),
         ("block_m", ctypes.c_int32), ("renormalize", ctypes.c_int32), ("split_k", ctypes.c_int32),
         ("router_weight_on_input", ctypes.c_int32), ("swiglu_limit", ctypes.c_float),
-        ("reserved", ctypes.c_int32 * 4),
+        ("persistent_decode", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3),
     ]
 
 
@@ -135,7 +135,7 @@ def _stream(stream=None):
 
 
 def problem(T, E, topk, H, I, fp8=False, mode=MODE_AUTO, block_m=0, renormalize=True, split_k=True,
-            mx=False, router_weight_on_input=False, swiglu_limit=0.0) -> MoeProblem:
+            mx=False, router_weight_on_input=False, swiglu_limit=0.0, persistent_decode=False) -> MoeProblem:
     """A moe_problem; ``fp8`` selects E4M3 weights with 128x128 fp32 block scales, ``mx`` MXFP8
     (E4M3 with per-32 E8M0 scales); ``router_weight_on_input`` (top-1 only) scales x by the router
     weight before GEMM1; ``swiglu_limit`` > 0 clamps gate and up before the activation."""
@@ -144,6 +144,7 @@ def problem(T, E, topk, H, I, fp8=False, mode=MODE_AUTO, block_m=0, renormalize=
     p.weight_dtype = DTYPE_MXFP8_E4M3 if mx else (DTYPE_FP8_E4M3 if fp8 else DTYPE_BF16)
     p.router_weight_on_input = 1 if router_weight_on_input else 0
     p.swiglu_limit = float(swiglu_limit)
+    p.persistent_decode = 1 if persistent_decode else 0
     p.mode, p.block_m, p.renormalize = int(mode), int(block_m), 1 if renormalize else 0
     p.split_k = 0 if split_k else 1
     return p

@@ -59,7 +59,8 @@ class Case:
     """One workload instance on the GPU plus its oracle evaluation."""
 
     def __init__(self, cfg: inputs.MoEConfig, T: int, seed: int = 0, mode=ops.MODE_AUTO, block_m=0,
-                 weights=None, split_k=True, router_weight_on_input=False, swiglu_limit=0.0, renormalize=True):
+                 weights=None, split_k=True, router_weight_on_input=False, swiglu_limit=0.0, renormalize=True,
+                 persistent_decode=False):
         self.cfg, self.T, self.seed = cfg, T, seed
         self.renormalize = renormalize
         self.router_weight_on_input, self.swiglu_limit = router_weight_on_input, swiglu_limit
@@ -80,7 +81,8 @@ class Case:
             self.w13_scale = self.w2_scale = None
         self.p = ops.problem(T, cfg.E, cfg.topk, cfg.H, cfg.I, fp8=cfg.fp8, mode=mode, block_m=block_m,
                              split_k=split_k, mx=cfg.mx, router_weight_on_input=router_weight_on_input,
-                             swiglu_limit=swiglu_limit, renormalize=renormalize)
+                             swiglu_limit=swiglu_limit, renormalize=renormalize,
+                             persistent_decode=persistent_decode)
         self.q = ops.resolve_problem(self.p)
         self.ws = ops.alloc_workspace(self.p)
         self.out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
