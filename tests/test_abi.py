@@ -200,3 +200,19 @@ def test_selftest_argument_errors(L):
     assert L.moe_selftest_wait_timeout(0, g, g, None) == ops.MOE_ERR_INVALID
     assert L.moe_selftest_wait_timeout(2_000_000, g, g, None) == ops.MOE_ERR_INVALID
     assert L.moe_selftest_wait_timeout(100, None, g, None) == ops.MOE_ERR_INVALID
+
+
+def test_sf_atom_reindex_matches_header_formula():
+    """ops.sf_atoms_to_rows is the inverse of the SF-atom layout the header documents."""
+    import torch
+    rows, cols, batches = 256, 384, 2
+    atoms = torch.empty(batches * rows * cols // 32, dtype=torch.long)
+    for b in range(batches):
+        for n in range(rows):
+            for k in range(0, cols, 32):
+                nn = b * rows + n
+                off = ((nn // 128) * (cols // 128) + k // 128) * 512 + (nn % 32) * 16 + ((nn % 128) // 32) * 4 \
+                    + (k % 128) // 32
+                atoms[off] = (b * rows + n) * (cols // 32) + k // 32
+    back = ops.sf_atoms_to_rows(atoms.reshape(batches, -1), rows, cols)
+    assert torch.equal(back.reshape(-1), torch.arange(batches * rows * cols // 32))
