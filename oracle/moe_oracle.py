@@ -58,6 +58,8 @@ __all__ = [
     "align",
     "expert_mlp",
     "moe_forward",
+    "expert_shards",
+    "moe_forward_expert_parallel",
 ]
 
 # bfloat16: 1 sign, 8 exponent, 7 stored mantissa bits (8 significant bits).
@@ -317,7 +319,7 @@ def align_capacity(T: int, topk: int, E: int, block_m: int) -> int:
     return -(-bound // block_m) * block_m
 
 
-def align(topk_ids, E: int, block_m: int):
+def align(topk_ids, E: int, block_m: int, first_expert: int = 0, num_global_experts=None):
     """Expert-sorted, block-padded permutation of the flat assignments.
 
     [PR] §1.1: ``sorted_token_ids`` (flat ids ``t*topk + j`` grouped by expert,
@@ -325,14 +327,23 @@ def align(topk_ids, E: int, block_m: int):
     ``num_tokens_post_padded`` and one expert per block.  Readings: stable
     order inside an expert, sentinel ``T*topk`` in padding, -1 past the last
     used block.
+
+    Expert parallelism ([PPLX] "MoE Dispatch - Combine", "Experten-Parallel":
+    the dispatch keeps the tokens routed to this rank's experts): the ids are
+    global, in ``[0, num_global_experts)``; only those in
+    ``[first_expert, first_expert + E)`` are kept, as local experts
+    ``id - first_expert``; the others are skipped.
     """
     ids = np.asarray(topk_ids).astype(np.int64)
     t, k = ids.shape
-    flat = ids.reshape(-1)
-    n = flat.size
-    if n and (flat.min() < 0 or flat.max() >= E):
+    n_global = E if num_global_experts is None else int(num_global_experts)
+    g = ids.reshape(-1)
+    n = g.size
+    if n and (g.min() < 0 or g.max() >= n_global):
         raise ValueError("expert id out of range")
-    counts = np.bincount(flat, minlength=E).astype(np.int64)
+    flat = g - first_expert                      # local id; outside [0, E) = another rank's expert
+    flat = np.where((flat >= 0) & (flat < E), flat, -1)
+    counts = np.bincount(flat[flat >= 0], minlength=E).astype(np.int64)
     padded = -(-counts // block_m) * block_m
     offsets = np.zeros(E + 1, dtype=np.int64)
     offsets[1:] = np.cumsum(padded)
@@ -399,7 +410,8 @@ def expert_mlp(x_hat, w13_hat, w2_hat, requant, return_intermediates: bool = Fal
 
 def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weights=None,
                 w13_scale=None, w2_scale=None, renormalize: bool = True, tokens=None,
-                return_y: bool = False, mx=None, router_weight_on_input: bool = False, swiglu_limit=None):
+                return_y: bool = False, mx=None, router_weight_on_input: bool = False, swiglu_limit=None,
+                expert_range=None):
     """The fused MoE layer: route -> experts -> top-k weighted combine.
 
     [AWS] "Warum MoE-Kernel so wichtig sind": one operation that routes each
@@ -422,6 +434,12 @@ def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weigh
     again; top-k > 1 is rejected (a non-linear expert cannot take the weight
     on its input without changing the layer).
     swiglu_limit: see :func:`expert_mlp`.
+    expert_range: ``(first, count)`` for expert parallelism ([PPLX]
+    "Experten-Parallel": each rank accumulates the contributions of its own
+    experts before an all-reduce).  ``w13``/``w2`` (and their scales) then
+    hold the experts ``[first, first + count)`` only, indexed from zero, the
+    routing is over all experts, and ``out`` is the bf16 rounding of the sum
+    over the token's assignments to those experts (zero when there are none).
 
     Returns a dict with ``out`` [len(tokens), H] (float64 holding bf16
     values), ``topk_ids``, ``topk_weights`` and, when asked, ``y``
@@ -455,11 +473,15 @@ def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weigh
         x_hat = xs
 
     ids = topk_ids[tokens]
+    base, count = (0, None) if expert_range is None else (int(expert_range[0]), int(expert_range[1]))
     wts = topk_weights[tokens].astype(np.float64)
     acc = np.zeros((tokens.size, h_dim), dtype=np.float64)
     y_all = np.zeros((tokens.size, topk, h_dim), dtype=np.float64) if return_y else None
-    for e in np.unique(ids):
-        rows, cols = np.nonzero(ids == e)                        # (token, slot) pairs on expert e
+    for g in np.unique(ids):
+        e = g - base                                             # index into the weights given
+        if count is not None and not 0 <= e < count:
+            continue                                             # another rank's expert
+        rows, cols = np.nonzero(ids == g)                        # (token, slot) pairs on expert g
         if mx:
             w13_e = dequantize_mx_group32(w13[e], w13_scale[e])
             w2_e = dequantize_mx_group32(w2[e], w2_scale[e])
@@ -482,3 +504,40 @@ def moe_forward(x, w13, w2, topk: int, *, logits=None, topk_ids=None, topk_weigh
     if return_y:
         result["y"] = y_all
     return result
+
+
+def expert_shards(E: int, world_size: int):
+    """Contiguous expert ranges ``(first, count)`` of ``world_size`` ranks.
+
+    [PPLX] "Hosting von Qwen auf Blackwell" shards 128 experts over EP=4/8/16
+    ranks without saying how.  Reading: rank r holds experts
+    ``[floor(r*E/N), floor((r+1)*E/N))`` -- contiguous, sizes differing by at
+    most one.
+    """
+    if world_size < 1 or world_size > E:
+        raise ValueError("need 1 <= world_size <= E")
+    bounds = [(r * E) // world_size for r in range(world_size + 1)]
+    return [(bounds[r], bounds[r + 1] - bounds[r]) for r in range(world_size)]
+
+
+def moe_forward_expert_parallel(x, w13, w2, topk: int, world_size: int, *, w13_scale=None, w2_scale=None,
+                                **kw):
+    """The layer under expert parallelism ([PPLX] "Experten-Parallel"): x and
+    the routing replicated on every rank, each rank's bf16 partial sum over its
+    own experts (:func:`moe_forward` with ``expert_range``), then an
+    all-reduce (sum) of the partials over the ranks.
+
+    Reading: the all-reduce is the exact sum of the bf16 partials, rounded once
+    to bf16 (a collective may round in another order; the difference is within
+    bf16 rounding of the summands).  Returns a dict with ``out`` and the list
+    ``partials``.
+    """
+    partials = []
+    for first, count in expert_shards(len(w13), world_size):
+        sl = slice(first, first + count)
+        r = moe_forward(x, w13[sl], w2[sl], topk, expert_range=(first, count),
+                        w13_scale=None if w13_scale is None else w13_scale[sl],
+                        w2_scale=None if w2_scale is None else w2_scale[sl], **kw)
+        partials.append(r["out"])
+    return {"out": round_bf16(np.sum(partials, axis=0)), "partials": partials}
+
