@@ -35,7 +35,8 @@
  *    moe_last_error_string() (per host thread) describes it.  Arguments are
  *    validated before anything is enqueued, so an error return means nothing
  *    was launched (MOE_ERR_CUDA excepted: a launch failed part way).
- *  - Bad device data (an expert id outside [0, E)) cannot be seen on the
+ *  - Bad device data (an expert id outside [0, E), or outside
+ *    [0, num_global_experts) under expert parallelism) cannot be seen on the
  *    host: the kernels record it in the workspace status word (see
  *    moe_read_status) and the outputs of that call are undefined.
  */
@@ -64,7 +65,7 @@ extern "C" {
 
 /* device status word codes (moe_read_status) */
 #define MOE_STATUS_OK 0
-#define MOE_STATUS_BAD_EXPERT_ID 1    /* an expert id outside [0, E) */
+#define MOE_STATUS_BAD_EXPERT_ID 1    /* an expert id outside [0, E) (num_global_experts under EP) */
 #define MOE_STATUS_WAIT_TIMEOUT 0x100 /* a bounded in-kernel wait ran out; low byte = where */
 
 /* weight types */
@@ -102,7 +103,8 @@ extern "C" {
  * Problem description.  T, E, topk, H, I and weight_dtype are required;
  * mode = MOE_MODE_AUTO and block_m = 0 let the library choose; both are
  * written back by moe_resolve_problem().
- * Constraints: T >= 0, 1 <= topk <= E <= 1024, H and I positive multiples of
+ * Constraints: T >= 0, 1 <= topk <= E <= 1024 (topk <= num_global_experts
+ * under expert parallelism, below), H and I positive multiples of
  * 128, T * topk < 2^31.  Normal tiles (and so MXFP8) cover 256 columns of H
  * per GEMM2 tile and need H % 256 == 0; MOE_MODE_AUTO picks swap-AB tiles
  * when H % 256 == 128.
@@ -131,7 +133,25 @@ typedef struct moe_problem {
    * cooperative launch, 0 = the kernel-per-stage pipeline (default: measured
    * faster, the persistent kernel is opt-in). */
   int32_t persistent_decode;
-  int32_t reserved[3];  /* must be zero */
+  /* Expert parallelism ("Hosting von Qwen auf Blackwell", section "MoE
+   * Dispatch - Combine", "Experten-Parallel": x and the routing are the same
+   * on every rank; each rank runs only the assignments to its own experts,
+   * sums them per token, and an all-reduce over the ranks completes the
+   * layer).  The router scores num_global_experts experts (router_logits is
+   * [T, num_global_experts]; topk_ids hold global ids in
+   * [0, num_global_experts)), while this call holds the weights of the E
+   * experts [first_expert, first_expert + E) only: w13 [E, 2I, H] and
+   * w2 [E, H, I] are those experts' weights, local expert e is global expert
+   * first_expert + e, and expert_counts / expert_offsets / expert_ids in the
+   * workspace are local.  Assignments to other experts are skipped (not an
+   * error), so out[t] is the sum over t's local assignments only, zero when
+   * it has none; the sum of out over a partition of the experts is the
+   * layer.  Constraints: E <= num_global_experts <= 1024, 0 <= first_expert
+   * <= num_global_experts - E, topk <= num_global_experts.  0 and 0 = every
+   * expert is local (num_global_experts = E). */
+  int32_t num_global_experts;
+  int32_t first_expert;
+  int32_t reserved[1];  /* must be zero */
 } moe_problem;
 
 /*
@@ -273,14 +293,15 @@ MOE_API int moe_get_workspace_layout(const moe_problem* p, moe_workspace_layout*
 /*
  * The fused MoE layer, all stages on `stream`.
  *   x             [T, H] bf16.
- *   router_logits [T, E] fp32, or NULL to use topk_ids / topk_weights
- *                 ([T, topk] int32 / fp32), which are then required.
+ *   router_logits [T, E] fp32 ([T, num_global_experts] under expert
+ *                 parallelism), or NULL to use topk_ids / topk_weights
+ *                 ([T, topk] int32 / fp32, global expert ids), which are then required.
  *   w13           [E, 2I, H]: bf16, or E4M3 codes with w13_scale [E, 2I/128, H/128] fp32
  *                 (MOE_DTYPE_FP8_E4M3), or E4M3 codes with w13_scale as E8M0 SF atoms
  *                 of [E, 2I, H] (MOE_DTYPE_MXFP8_E4M3; x and the intermediate are then
  *                 MX-quantised the same way, per row and 32 columns).
  *   w2            [E, H, I]:  likewise, w2_scale [E, H/128, I/128] fp32 or SF atoms of [E, H, I].
- *   out           [T, H] bf16.
+ *   out           [T, H] bf16 (under expert parallelism: this rank's partial sum).
  *   ws            device scratch of at least moe_workspace_size(p) bytes,
  *                 256-byte aligned; the call clears what must start at zero.
  *                 Two calls that overlap on the device must not share it.

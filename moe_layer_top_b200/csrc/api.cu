@@ -60,12 +60,23 @@ inline int64_t align256(int64_t v) { return (v + 255) & ~int64_t(255); }
 
 bool aligned(const void* p, uintptr_t a) { return (reinterpret_cast<uintptr_t>(p) & (a - 1)) == 0; }
 
+// Router width: every expert, of which this call holds [first_expert, first_expert + E).
+int global_experts(const moe_problem* p) { return p->num_global_experts == 0 ? p->E : p->num_global_experts; }
+
+bool expert_parallel(const moe_problem* p) { return global_experts(p) != p->E; }
+
 int validate_problem(const moe_problem* p) {
   if (p == nullptr) return fail(MOE_ERR_INVALID, "problem is NULL");
   if (p->T < 0) return fail(MOE_ERR_INVALID, "T = %d < 0", p->T);
   if (p->E < 1 || p->E > 1024) return fail(MOE_ERR_INVALID, "E = %d outside [1, 1024]", p->E);
-  if (p->topk < 1 || p->topk > p->E || p->topk > 32)
-    return fail(MOE_ERR_INVALID, "topk = %d outside [1, min(E, 32)]", p->topk);
+  if (p->num_global_experts != 0 && (p->num_global_experts < p->E || p->num_global_experts > 1024))
+    return fail(MOE_ERR_INVALID, "num_global_experts = %d outside [E, 1024] (E = %d; 0 = E)", p->num_global_experts,
+                p->E);
+  if (p->first_expert < 0 || p->first_expert > global_experts(p) - p->E)
+    return fail(MOE_ERR_INVALID, "first_expert = %d outside [0, num_global_experts - E] = [0, %d]", p->first_expert,
+                global_experts(p) - p->E);
+  if (p->topk < 1 || p->topk > global_experts(p) || p->topk > 32)
+    return fail(MOE_ERR_INVALID, "topk = %d outside [1, min(num_global_experts, 32)]", p->topk);
   if (p->H <= 0 || p->H % 128) return fail(MOE_ERR_INVALID, "H = %d is not a positive multiple of 128", p->H);
   if (p->I <= 0 || p->I % 128) return fail(MOE_ERR_INVALID, "I = %d is not a positive multiple of 128", p->I);
   if (static_cast<int64_t>(p->T) * p->topk >= (int64_t(1) << 31))
@@ -79,8 +90,7 @@ int validate_problem(const moe_problem* p) {
   if (p->mode < MOE_MODE_AUTO || p->mode > MOE_MODE_SWAP_AB) return fail(MOE_ERR_INVALID, "mode %d", p->mode);
   if (p->renormalize != 0 && p->renormalize != 1) return fail(MOE_ERR_INVALID, "renormalize must be 0 or 1");
   if (p->split_k != 0 && p->split_k != 1) return fail(MOE_ERR_INVALID, "split_k must be 0 or 1");
-  for (int i = 0; i < 3; ++i)
-    if (p->reserved[i] != 0) return fail(MOE_ERR_INVALID, "reserved fields must be zero");
+  if (p->reserved[0] != 0) return fail(MOE_ERR_INVALID, "reserved fields must be zero");
   if (p->persistent_decode != 0 && p->persistent_decode != 1)
     return fail(MOE_ERR_INVALID, "persistent_decode must be 0 or 1");
   if (p->router_weight_on_input != 0 && p->router_weight_on_input != 1)
@@ -120,7 +130,8 @@ void resolve(moe_problem* p) {
     p->block_m = 128;
     return;
   }
-  const int64_t n = static_cast<int64_t>(p->T) * p->topk;
+  // assignments expected on this call's experts (all of them without expert parallelism)
+  const int64_t n = static_cast<int64_t>(p->T) * p->topk * p->E / global_experts(p);
   const int64_t hit = n < p->E ? n : p->E;
   const double avg = hit > 0 ? static_cast<double>(n) / static_cast<double>(hit) : 1.0;
   if (p->mode == MOE_MODE_AUTO) {
@@ -155,6 +166,8 @@ struct Plan {
   bool pair;        // two-SM FP8 tiles
   bool tok_gather;  // swap-AB: GEMM1 gathers token rows (TMA gather4) from x or its per-token copy;
                     // normal tiles read a sorted copy a1 [capacity, H] (gather4 is too slow for 128-row tiles)
+  bool ep;          // expert parallelism: some assignments go to other ranks' experts
+  moe::ExpertRange er;
 };
 
 int make_plan(const moe_problem* in, Plan* plan) {
@@ -167,6 +180,8 @@ int make_plan(const moe_problem* in, Plan* plan) {
   plan->fp8 = p.weight_dtype == MOE_DTYPE_FP8_E4M3 || plan->mx;
   plan->pair = p.mode == MOE_MODE_NORMAL && p.block_m == 256;
   plan->tok_gather = p.mode == MOE_MODE_SWAP_AB;
+  plan->ep = expert_parallel(&p);
+  plan->er = moe::ExpertRange{p.first_expert, global_experts(&p)};
   plan->nflat = static_cast<int64_t>(p.T) * p.topk;
   const int64_t cap = capacity_of(p.T, p.topk, p.E, p.block_m);
   if (cap >= (int64_t(1) << 31)) return fail(MOE_ERR_INVALID, "padded row capacity overflows int32");
@@ -198,7 +213,8 @@ int make_plan(const moe_problem* in, Plan* plan) {
     L.a1 = take(static_cast<int64_t>(p.T) * p.H * elem);
   else
     L.a1 = -1;
-  L.pos_of_flat = (plan->fp8 && !plan->pair) ? take(plan->nflat * 4) : -1;
+  // the inverse permutation: FP8 scale scatter, and the combine's mask under expert parallelism
+  L.pos_of_flat = ((plan->fp8 && !plan->pair) || plan->ep) ? take(plan->nflat * 4) : -1;
   // FP8: fp32 [K/128, cap]; MXFP8: E8M0 SF atoms, (cap/128) * (K/128) * 512 bytes -- the same size
   L.a1_scale = plan->fp8 ? take(cap * (p.H / 128) * 4) : -1;
   L.a2 = take(cap * p.I * elem);
@@ -262,7 +278,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
   const float* wts = logits ? at<float>(ws, L.topk_weights) : topk_weights;
   const int nflat = static_cast<int>(plan.nflat);
   const int cap = L.capacity;
-  const bool small = moe::route_align_small_fits(plan.nflat, p.E);
+  const bool small = moe::route_align_small_fits(plan.nflat, plan.er.e_global);
   const bool swap = p.mode == MOE_MODE_SWAP_AB;
   int32_t* pos = L.pos_of_flat >= 0 ? at<int32_t>(ws, L.pos_of_flat) : nullptr;
   // GEMM1's token source: the sorted copy (normal tiles), the per-token copy, or x
@@ -271,7 +287,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
   cudaError_t e;
 
   // the whole layer of a small bf16 batch in one persistent cooperative launch
-  if (stage_begin == 0 && stage_end == MOE_NUM_STAGES && p.persistent_decode == 1 && !plan.fp8 && swap &&
+  if (stage_begin == 0 && stage_end == MOE_NUM_STAGES && p.persistent_decode == 1 && !plan.fp8 && swap && !plan.ep &&
       p.block_m == moe::kDecodeBlockM && p.router_weight_on_input == 0 &&
       moe::decode_fused_fits(p.T, p.E, p.topk, p.H, p.I)) {
     int* sync = at<int>(ws, L.partials);  // the split-K buffer is not used by this path
@@ -317,8 +333,9 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
           return cuda_fail(e, "clear status");
         if (small && stage_end > MOE_STAGE_ALIGN) {
           // small batch: routing and the alignment in one single-CTA kernel
-          e = moe::launch_route_align_small(logits, logits ? nullptr : topk_ids, p.T, p.E, p.topk, p.renormalize,
-                                            at<int32_t>(ws, L.topk_ids), at<float>(ws, L.topk_weights), p.block_m,
+          e = moe::launch_route_align_small(logits, logits ? nullptr : topk_ids, p.T, p.E, plan.er, p.topk,
+                                            p.renormalize, at<int32_t>(ws, L.topk_ids), at<float>(ws, L.topk_weights),
+                                            p.block_m,
                                             cap, at<int32_t>(ws, L.sorted_token_ids), at<int32_t>(ws, L.expert_ids),
                                             at<int32_t>(ws, L.num_tokens_post_padded),
                                             at<int32_t>(ws, L.expert_counts), at<int32_t>(ws, L.expert_offsets),
@@ -326,7 +343,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
           if (e != cudaSuccess) return cuda_fail(e, "route+align");
           aligned_already = true;
         } else if (logits) {
-          e = moe::launch_route(logits, p.T, p.E, p.topk, p.renormalize, at<int32_t>(ws, L.topk_ids),
+          e = moe::launch_route(logits, p.T, plan.er.e_global, p.topk, p.renormalize, at<int32_t>(ws, L.topk_ids),
                                 at<float>(ws, L.topk_weights), stream);
           if (e != cudaSuccess) return cuda_fail(e, "route");
         }
@@ -334,7 +351,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
       case MOE_STAGE_ALIGN:
         if (aligned_already) break;
         if (small) {
-          e = moe::launch_route_align_small(nullptr, ids, p.T, p.E, p.topk, p.renormalize, nullptr, nullptr,
+          e = moe::launch_route_align_small(nullptr, ids, p.T, p.E, plan.er, p.topk, p.renormalize, nullptr, nullptr,
                                             p.block_m, cap, at<int32_t>(ws, L.sorted_token_ids),
                                             at<int32_t>(ws, L.expert_ids), at<int32_t>(ws, L.num_tokens_post_padded),
                                             at<int32_t>(ws, L.expert_counts), at<int32_t>(ws, L.expert_offsets),
@@ -342,7 +359,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
           if (e != cudaSuccess) return cuda_fail(e, "align");
           break;
         }
-        e = moe::launch_align(ids, nflat, p.E, p.block_m, cap, at<int32_t>(ws, L.sorted_token_ids),
+        e = moe::launch_align(ids, nflat, p.E, plan.er, p.block_m, cap, at<int32_t>(ws, L.sorted_token_ids),
                               at<int32_t>(ws, L.expert_ids), at<int32_t>(ws, L.num_tokens_post_padded),
                               at<int32_t>(ws, L.expert_counts), at<int32_t>(ws, L.expert_offsets),
                               at<int32_t>(ws, L.align_scratch), nullptr, nullptr, status, pos, stream);
@@ -409,7 +426,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
         break;
       }
       case MOE_STAGE_COMBINE:
-        e = moe::launch_combine(at<void>(ws, L.y), p.T, p.topk, p.H, out, stream);
+        e = moe::launch_combine(at<void>(ws, L.y), p.T, p.topk, p.H, plan.ep ? pos : nullptr, out, stream);
         if (e != cudaSuccess) return cuda_fail(e, "combine");
         break;
       default:
@@ -506,13 +523,15 @@ int moe_align(const int32_t* topk_ids, int32_t T, int32_t topk, int32_t E, int32
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "align");
   }
   if (moe::route_align_small_fits(n, E)) {
-    e = moe::launch_route_align_small(nullptr, topk_ids, T, E, topk, 1, nullptr, nullptr, block_m,
+    e = moe::launch_route_align_small(nullptr, topk_ids, T, E, moe::ExpertRange{0, E}, topk, 1, nullptr, nullptr,
+                                      block_m,
                                       static_cast<int>(cap), sorted_token_ids, expert_ids, num_tokens_post_padded,
                                       expert_counts ? expert_counts : counts, expert_offsets ? expert_offsets : offs,
                                       status, nullptr, s);
     return e == cudaSuccess ? MOE_OK : cuda_fail(e, "align");
   }
-  e = moe::launch_align(topk_ids, static_cast<int>(n), E, block_m, static_cast<int>(cap), sorted_token_ids,
+  e = moe::launch_align(topk_ids, static_cast<int>(n), E, moe::ExpertRange{0, E}, block_m, static_cast<int>(cap),
+                        sorted_token_ids,
                         expert_ids, num_tokens_post_padded, counts, offs, scratch, expert_counts, expert_offsets,
                         status, nullptr, s);
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "align");

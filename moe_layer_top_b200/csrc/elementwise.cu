@@ -254,10 +254,14 @@ cudaError_t launch_prepare_x(const void* x, int T, int H, int topk, bool fp8, bo
 // ----------------------------------------------------------------------------
 // combine ("Hosting von Qwen auf Blackwell", "MoE Dispatch - Combine": the
 // weighted accumulation; the weights were applied in the GEMM2 epilogue):
-// out[t, :] = bf16(sum_j y[t*topk + j, :]) in fp32, j ascending.
+// out[t, :] = bf16(sum_j y[t*topk + j, :]) in fp32, j ascending.  kMasked
+// (expert parallelism, "Experten-Parallel": the local accumulation before the
+// all-reduce): only the assignments with a row on this rank, pos_of_flat >= 0;
+// a token without one gets zeros.
 // ----------------------------------------------------------------------------
+template <bool kMasked>
 __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* y, int T, int topk, int H,
-                                                      __nv_bfloat16* out) {
+                                                      const int32_t* pos_of_flat, __nv_bfloat16* out) {
   pdl_launch_dependents();
   pdl_wait();
   const int vecs = H / 8;
@@ -269,6 +273,7 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* y, in
     float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
     const uint4* src = reinterpret_cast<const uint4*>(y + static_cast<size_t>(t) * topk * H) + v;
     for (int j = 0; j < topk; ++j) {
+      if (kMasked && (*(pos_of_flat + static_cast<size_t>(t) * topk + j)) < 0) continue;  // never written
       float f[8];
       unpack8((*(src + static_cast<size_t>(j) * vecs)), f);
 #pragma unroll
@@ -278,13 +283,18 @@ __global__ void __launch_bounds__(256) combine_kernel(const __nv_bfloat16* y, in
   }
 }
 
-cudaError_t launch_combine(const void* y, int T, int topk, int H, void* out, cudaStream_t stream) {
+cudaError_t launch_combine(const void* y, int T, int topk, int H, const int32_t* pos_of_flat, void* out,
+                           cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
   const long long total = static_cast<long long>(T) * (H / 8);
   long long blocks = (total + 255) / 256;
   if (blocks > 148 * 16) blocks = 148 * 16;
-  return launch_pdl(combine_kernel, static_cast<int>(blocks), 256, 0, stream, static_cast<const __nv_bfloat16*>(y), T,
-                    topk, H, static_cast<__nv_bfloat16*>(out));
+  const auto* yb = static_cast<const __nv_bfloat16*>(y);
+  auto* ob = static_cast<__nv_bfloat16*>(out);
+  if (pos_of_flat)
+    return launch_pdl(combine_kernel<true>, static_cast<int>(blocks), 256, 0, stream, yb, T, topk, H, pos_of_flat,
+                      ob);
+  return launch_pdl(combine_kernel<false>, static_cast<int>(blocks), 256, 0, stream, yb, T, topk, H, pos_of_flat, ob);
 }
 
 // ----------------------------------------------------------------------------

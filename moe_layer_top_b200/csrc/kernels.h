@@ -35,22 +35,33 @@ cudaError_t launch_route(const float* logits, int T, int E, int topk, int renorm
 constexpr int kAlignChunk = 256;  // assignments per warp-chunk
 inline int align_chunks(long long n) { return static_cast<int>((n + kAlignChunk - 1) / kAlignChunk); }
 
-cudaError_t launch_align(const int32_t* topk_ids, int n, int E, int block_m, int capacity,
+// Expert ranges (both align paths): the ids are global, in [0, e_global);
+// local expert e is global expert first + e for e in [0, E).  Assignments to
+// other experts are skipped silently; ids outside [0, e_global) are reported.
+// Without expert parallelism first = 0 and e_global = E.
+struct ExpertRange {
+  int first;
+  int e_global;
+};
+
+cudaError_t launch_align(const int32_t* topk_ids, int n, int E, ExpertRange er, int block_m, int capacity,
                          int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp, int32_t* counts_ws,
                          int32_t* offsets_ws, int32_t* chunk_scratch, int32_t* user_counts,
                          int32_t* user_offsets, int* status, int32_t* pos_of_flat, cudaStream_t stream);
 
-// single-CTA route (optional) + align for small batches
+// single-CTA route (optional, over er.e_global experts) + align for small batches
 constexpr int kSmallAlignMaxN = 8192;  // assignments (T * topk)
-constexpr int kSmallAlignMaxE = 256;
-bool route_align_small_fits(long long n, int E);
-cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in, int T, int E, int topk,
-                                     int renormalize, int32_t* ids_out, float* weights_out, int block_m, int capacity,
-                                     int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp, int32_t* counts,
-                                     int32_t* offsets, int* status, int32_t* pos_of_flat, cudaStream_t stream);
+constexpr int kSmallAlignMaxE = 256;   // router width (e_global)
+bool route_align_small_fits(long long n, int e_global);
+cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in, int T, int E, ExpertRange er,
+                                     int topk, int renormalize, int32_t* ids_out, float* weights_out, int block_m,
+                                     int capacity, int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp,
+                                     int32_t* counts, int32_t* offsets, int* status, int32_t* pos_of_flat,
+                                     cudaStream_t stream);
 
 // pos_of_flat (optional, both align paths): sorted position of every flat
-// assignment, -1 for an invalid expert id (the inverse of sorted_token_ids)
+// assignment, -1 for an invalid or non-local expert id (the inverse of
+// sorted_token_ids)
 
 // gather x rows into sorted order: bf16 copy, FP8 per-(row,128) quantisation
 // (a1_scale: fp32 [H/128, capacity]) or MXFP8 per-(row,32) quantisation
@@ -72,8 +83,10 @@ cudaError_t launch_prepare_x(const void* x, int T, int H, int topk, bool fp8, bo
 cudaError_t launch_copy_rows(const void* xq, int H, int topk, int nflat, const int32_t* sorted_ids,
                              const int32_t* ntpp, int capacity, void* a1, cudaStream_t stream);
 
-// out[t] = sum_j y[t*topk + j]
-cudaError_t launch_combine(const void* y, int T, int topk, int H, void* out, cudaStream_t stream);
+// out[t] = sum_j y[t*topk + j]; with pos_of_flat, only the assignments that
+// have a row (pos_of_flat >= 0: local experts under expert parallelism)
+cudaError_t launch_combine(const void* y, int T, int topk, int H, const int32_t* pos_of_flat, void* out,
+                           cudaStream_t stream);
 
 // FP8 128x128 block weight quantisation
 cudaError_t launch_quantize_weights(const void* w, long long batches, int rows, int cols, uint8_t* codes,

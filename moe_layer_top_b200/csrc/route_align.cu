@@ -18,6 +18,12 @@
 //      ascending flat order inside every expert, whatever the scheduling.
 // Padding slots, the tail past num_tokens_post_padded and the per-block
 // expert ids are filled by the same third pass.
+//
+// Expert parallelism ("Hosting von Qwen auf Blackwell", "Experten-Parallel":
+// the dispatch picks the tokens routed to this rank's experts): the router
+// scores all experts and the ids stay global; the alignment keeps only the
+// assignments to the local range [first, first + E), which it renumbers from
+// zero, so every later stage sees an ordinary E-expert problem.
 #include <climits>
 
 #include "common.cuh"
@@ -65,7 +71,7 @@ cudaError_t launch_route(const float* logits, int T, int E, int topk, int renorm
 constexpr int kAlignWarps = 8;
 
 __global__ void __launch_bounds__(kAlignWarps * 32) align_count_kernel(const int32_t* ids, int n,
-                                                                       int E, int nchunks,
+                                                                       int E, ExpertRange er, int nchunks,
                                                                        int32_t* chunk_counts,
                                                                        int* status) {
   extern __shared__ int32_t hist_all[];
@@ -81,11 +87,12 @@ __global__ void __launch_bounds__(kAlignWarps * 32) align_count_kernel(const int
   for (int i = lane; i < kAlignChunk; i += 32) {
     const int f = base + i;
     if (f < n) {
-      const int e = (*(ids + f));
-      if (e >= 0 && e < E)
-        atomicAdd(&hist[e], 1);
-      else
+      const int g = (*(ids + f));
+      const int e = g - er.first;
+      if (g < 0 || g >= er.e_global)
         report_status(status, MOE_STATUS_BAD_EXPERT_ID);
+      else if (e >= 0 && e < E)
+        atomicAdd(&hist[e], 1);  // other ranks' experts are not counted here
     }
   }
   __syncwarp();
@@ -150,7 +157,7 @@ __device__ __forceinline__ int owner_expert(const int32_t* offs, int E, int p) {
 }
 
 __global__ void __launch_bounds__(kAlignWarps * 32) align_scatter_kernel(
-    const int32_t* ids, int n, int E, int block_m, int capacity, int nchunks,
+    const int32_t* ids, int n, int E, int first, int block_m, int capacity, int nchunks,
     const int32_t* chunk_base, const int32_t* counts_ws, int32_t* sorted_ids,
     int32_t* expert_ids, int32_t* ntpp_out, int32_t* offsets_ws,
     int32_t* user_offsets, int32_t* pos_of_flat) {
@@ -211,8 +218,8 @@ __global__ void __launch_bounds__(kAlignWarps * 32) align_scatter_kernel(
       const int f = base + i0 + lane;
       int e = -1;
       if (f < n) {
-        e = (*(ids + f));
-        if (e < 0 || e >= E) e = -1;  // reported by pass 1; never indexed
+        e = (*(ids + f)) - first;
+        if (e < 0 || e >= E) e = -1;  // invalid (reported by pass 1) or not local: never indexed
       }
       const uint32_t same = __match_any_sync(0xffffffffu, e);
       const uint32_t lower = same & ((1u << lane) - 1u);
@@ -246,7 +253,8 @@ __global__ void __launch_bounds__(kAlignWarps * 32) align_scatter_kernel(
   }
 }
 
-cudaError_t launch_align(const int32_t* topk_ids, int n, int E, int block_m, int capacity, int32_t* sorted_ids,
+cudaError_t launch_align(const int32_t* topk_ids, int n, int E, ExpertRange er, int block_m, int capacity,
+                         int32_t* sorted_ids,
                          int32_t* expert_ids, int32_t* ntpp, int32_t* counts_ws, int32_t* offsets_ws,
                          int32_t* chunk_scratch, int32_t* user_counts, int32_t* user_offsets, int* status,
                          int32_t* pos_of_flat, cudaStream_t stream) {
@@ -255,7 +263,7 @@ cudaError_t launch_align(const int32_t* topk_ids, int n, int E, int block_m, int
   const int threads = kAlignWarps * 32;
   const int blocks = (nchunks + kAlignWarps - 1) / kAlignWarps;
   const size_t smem1 = static_cast<size_t>(kAlignWarps) * E * sizeof(int32_t);
-  cudaError_t err = launch_pdl(align_count_kernel, blocks, threads, smem1, stream, topk_ids, n, E, nchunks,
+  cudaError_t err = launch_pdl(align_count_kernel, blocks, threads, smem1, stream, topk_ids, n, E, er, nchunks,
                                chunk_scratch, status);
   if (err != cudaSuccess) return err;
   err = launch_pdl(align_scan_kernel, E, 256, 0, stream, chunk_scratch, nchunks, E, counts_ws, user_counts);
@@ -265,7 +273,7 @@ cudaError_t launch_align(const int32_t* topk_ids, int n, int E, int block_m, int
   const int fill_blocks = (capacity + threads * 4 - 1) / (threads * 4);
   if (fill_blocks > blocks3) blocks3 = fill_blocks < 296 ? fill_blocks : 296;
   if (blocks3 < blocks) blocks3 = blocks;
-  return launch_pdl(align_scatter_kernel, blocks3, threads, smem3, stream, topk_ids, n, E, block_m, capacity,
+  return launch_pdl(align_scatter_kernel, blocks3, threads, smem3, stream, topk_ids, n, E, er.first, block_m, capacity,
                     nchunks, chunk_scratch, counts_ws, sorted_ids, expert_ids, ntpp, offsets_ws, user_offsets,
                     pos_of_flat);
 }
@@ -280,7 +288,7 @@ cudaError_t launch_align(const int32_t* topk_ids, int n, int E, int block_m, int
 // ----------------------------------------------------------------------------
 template <int VPL>
 __global__ void __launch_bounds__(1024) route_align_small_kernel(
-    const float* logits, const int32_t* ids_in, int T, int E, int topk, int renormalize,
+    const float* logits, const int32_t* ids_in, int T, int E, ExpertRange er, int topk, int renormalize,
     int32_t* ids_out, float* weights_out, int block_m, int capacity,
     int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp_out,
     int32_t* counts_out, int32_t* offsets_out, int* status, int32_t* pos_of_flat) {
@@ -299,7 +307,7 @@ __global__ void __launch_bounds__(1024) route_align_small_kernel(
     for (int t = warp; t < T; t += 32) {
       int id;
       float w;
-      route_token<VPL>(logits + static_cast<size_t>(t) * E, E, topk, renormalize, lane, id, w);
+      route_token<VPL>(logits + static_cast<size_t>(t) * er.e_global, er.e_global, topk, renormalize, lane, id, w);
       if (lane < topk) {
         ids_out[t * topk + lane] = id;
         weights_out[t * topk + lane] = w;
@@ -316,11 +324,12 @@ __global__ void __launch_bounds__(1024) route_align_small_kernel(
   const int begin = warp * chunk;
   const int end = min(begin + chunk, n);
   for (int i = begin + lane; i < end; i += 32) {
-    const int e = ids_s[i];
-    if (e >= 0 && e < E)
-      atomicAdd(&hist[warp * E + e], 1);
-    else
+    const int g = ids_s[i];
+    const int e = g - er.first;
+    if (g < 0 || g >= er.e_global)
       report_status(status, MOE_STATUS_BAD_EXPERT_ID);
+    else if (e >= 0 && e < E)
+      atomicAdd(&hist[warp * E + e], 1);
   }
   __syncthreads();
   for (int e = tid; e < E; e += 1024) {
@@ -359,8 +368,8 @@ __global__ void __launch_bounds__(1024) route_align_small_kernel(
     const int i = i0 + lane;
     int e = -1;
     if (i < end) {
-      e = ids_s[i];
-      if (e < 0 || e >= E) e = -1;
+      e = ids_s[i] - er.first;
+      if (e < 0 || e >= E) e = -1;  // invalid or not local
     }
     const uint32_t same = __match_any_sync(0xffffffffu, e);
     const uint32_t lower = same & ((1u << lane) - 1u);
@@ -393,12 +402,15 @@ __global__ void __launch_bounds__(1024) route_align_small_kernel(
   if (tid == 0) *ntpp_out = ntpp;
 }
 
-bool route_align_small_fits(long long n, int E) { return n > 0 && n <= kSmallAlignMaxN && E <= kSmallAlignMaxE; }
+bool route_align_small_fits(long long n, int e_global) {
+  return n > 0 && n <= kSmallAlignMaxN && e_global <= kSmallAlignMaxE;
+}
 
-cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in, int T, int E, int topk,
-                                     int renormalize, int32_t* ids_out, float* weights_out, int block_m, int capacity,
-                                     int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp, int32_t* counts,
-                                     int32_t* offsets, int* status, int32_t* pos_of_flat, cudaStream_t stream) {
+cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in, int T, int E, ExpertRange er,
+                                     int topk, int renormalize, int32_t* ids_out, float* weights_out, int block_m,
+                                     int capacity, int32_t* sorted_ids, int32_t* expert_ids, int32_t* ntpp,
+                                     int32_t* counts, int32_t* offsets, int* status, int32_t* pos_of_flat,
+                                     cudaStream_t stream) {
   const size_t smem = (static_cast<size_t>(T) * topk + 32 * static_cast<size_t>(E) + 2 * static_cast<size_t>(E) + 1) *
                       sizeof(int32_t);
   static bool attr_set[4] = {false, false, false, false};
@@ -408,10 +420,11 @@ cudaError_t launch_route_align_small(const float* logits, const int32_t* ids_in,
       if (e != cudaSuccess) return e;
       attr_set[idx] = true;
     }
-    return launch_pdl(kern, 1, 1024, smem, stream, logits, ids_in, T, E, topk, renormalize, ids_out, weights_out,
-                      block_m, capacity, sorted_ids, expert_ids, ntpp, counts, offsets, status, pos_of_flat);
+    return launch_pdl(kern, 1, 1024, smem, stream, logits, ids_in, T, E, er, topk, renormalize, ids_out,
+                      weights_out, block_m, capacity, sorted_ids, expert_ids, ntpp, counts, offsets, status,
+                      pos_of_flat);
   };
-  if (E <= 128) return pick(route_align_small_kernel<4>, 0);
+  if (er.e_global <= 128) return pick(route_align_small_kernel<4>, 0);
   return pick(route_align_small_kernel<8>, 1);
 }
 

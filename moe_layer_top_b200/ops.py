@@ -54,7 +54,8 @@ class MoeProblem(ctypes.Structure):
         ("I", ctypes.c_int32), ("weight_dtype", ctypes.c_int32), ("mode", ctypes.c_int32),
         ("block_m", ctypes.c_int32), ("renormalize", ctypes.c_int32), ("split_k", ctypes.c_int32),
         ("router_weight_on_input", ctypes.c_int32), ("swiglu_limit", ctypes.c_float),
-        ("persistent_decode", ctypes.c_int32), ("reserved", ctypes.c_int32 * 3),
+        ("persistent_decode", ctypes.c_int32), ("num_global_experts", ctypes.c_int32),
+        ("first_expert", ctypes.c_int32), ("reserved", ctypes.c_int32 * 1),
     ]
 
 
@@ -135,11 +136,15 @@ def _stream(stream=None):
 
 
 def problem(T, E, topk, H, I, fp8=False, mode=MODE_AUTO, block_m=0, renormalize=True, split_k=True,
-            mx=False, router_weight_on_input=False, swiglu_limit=0.0, persistent_decode=False) -> MoeProblem:
+            mx=False, router_weight_on_input=False, swiglu_limit=0.0, persistent_decode=False,
+            num_global_experts=0, first_expert=0) -> MoeProblem:
     """A moe_problem; ``fp8`` selects E4M3 weights with 128x128 fp32 block scales, ``mx`` MXFP8
     (E4M3 with per-32 E8M0 scales); ``router_weight_on_input`` (top-1 only) scales x by the router
-    weight before GEMM1; ``swiglu_limit`` > 0 clamps gate and up before the activation."""
+    weight before GEMM1; ``swiglu_limit`` > 0 clamps gate and up before the activation.
+    Expert parallelism: ``E`` experts held here, global experts ``[first_expert, first_expert + E)``
+    of ``num_global_experts`` that the router scores (0 = ``E``)."""
     p = MoeProblem()
+    p.num_global_experts, p.first_expert = int(num_global_experts), int(first_expert)
     p.T, p.E, p.topk, p.H, p.I = int(T), int(E), int(topk), int(H), int(I)
     p.weight_dtype = DTYPE_MXFP8_E4M3 if mx else (DTYPE_FP8_E4M3 if fp8 else DTYPE_BF16)
     p.router_weight_on_input = 1 if router_weight_on_input else 0

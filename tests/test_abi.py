@@ -216,3 +216,38 @@ def test_sf_atom_reindex_matches_header_formula():
                 atoms[off] = (b * rows + n) * (cols // 32) + k // 32
     back = ops.sf_atoms_to_rows(atoms.reshape(batches, -1), rows, cols)
     assert torch.equal(back.reshape(-1), torch.arange(batches * rows * cols // 32))
+
+
+def test_expert_parallel_problem_validation(L):
+    """Expert ranges: E local experts [first_expert, first_expert + E) of num_global_experts."""
+    size = lambda **kw: L.moe_workspace_size(ctypes.byref(ops.problem(64, kw.pop("E", 16), kw.pop("topk", 8), 4096,
+                                                                        1536, **kw)))
+    assert size(num_global_experts=128, first_expert=112) > 0
+    assert size(num_global_experts=128, first_expert=0) > 0
+    assert size(E=2, topk=8, num_global_experts=16, first_expert=14) > 0   # topk may exceed the local count
+    assert size(num_global_experts=128, first_expert=113) == 0                # range past the last expert
+    assert size(num_global_experts=128, first_expert=-1) == 0
+    assert size(num_global_experts=8) == 0                                    # fewer global than local
+    assert size(num_global_experts=2048) == 0
+    assert size(first_expert=1) == 0                                          # no range without num_global_experts
+    assert size(E=2, topk=8) == 0                                             # topk <= num_global_experts
+    p = ops.problem(64, 16, 8, 4096, 1536)
+    p.reserved[0] = 1
+    assert L.moe_workspace_size(ctypes.byref(p)) == 0
+
+
+def test_expert_parallel_plan(L):
+    """A rank's tiles are chosen from the tokens its experts expect (T*topk*E/num_global_experts), and
+    its workspace keeps the inverse permutation, which masks the combine."""
+    full = ops.resolve_problem(ops.problem(4096, 128, 8, 4096, 1536))
+    shard = ops.resolve_problem(ops.problem(4096, 16, 8, 4096, 1536, num_global_experts=128, first_expert=32))
+    assert full.mode == ops.MODE_NORMAL and shard.mode == ops.MODE_NORMAL
+    small = ops.resolve_problem(ops.problem(64, 16, 8, 4096, 1536, num_global_experts=128, first_expert=32))
+    assert small.mode == ops.MODE_SWAP_AB and small.block_m == 16               # 64*8/128 = 4 tokens per expert
+    assert small.num_global_experts == 128 and small.first_expert == 32
+    for fp8 in (False, True):
+        lay = ops.workspace_layout(ops.problem(64, 16, 8, 4096, 1536, fp8=fp8, num_global_experts=128,
+                                               first_expert=16))
+        assert lay.pos_of_flat >= 0
+        # capacity bounds the local rows: every assignment may land here
+        assert lay.capacity == ops.align_capacity(64, 8, 16, lay.block_m)
