@@ -10,9 +10,11 @@ from a second graph of the same stages with event nodes between them.  The defau
 Qwen3-235B-shaped decode layer (H=4096, E=128, top-8, I=1536); the headline
 batch is its largest sweep point (T=64) and every sweep point is reported.
 L2 is flushed (a 256 MiB write) before every timed step; the flush is outside
-the CUDA-event brackets.  Multi-GPU runs are independent replicas (the layer
-has no exchange step on one node): each rank runs the same workload and the
-time is the max over ranks.
+the CUDA-event brackets.  Multi-GPU runs are independent replicas by default
+(each rank runs the same workload; the time is the max over ranks).  With
+``--ep N`` the layer is expert-parallel instead: each of N ranks holds E/N
+experts, runs its share of the replicated batch and the output is all-reduced
+over NCCL; on one GPU ``--ep N`` times one rank's share alone.
 
 The ``--impl reference`` arm times the CPU oracle (the plain float64 numpy
 restatement of the layer) on the host cores, on bounded token samples of the
@@ -56,6 +58,10 @@ def parse_args():
     ap.add_argument("--no-cpu-baseline", action="store_true")
     ap.add_argument("--cpu-budget", type=float, default=15.0, help="seconds of oracle work for the CPU baseline")
     ap.add_argument("--seed", type=int, default=0)
+    ap.add_argument("--ep", type=int, default=0,
+                    help="expert parallelism over N ranks: each rank holds E/N experts, x is replicated and an "
+                         "all-reduce of the output completes the layer; on one GPU, time one rank's share")
+    ap.add_argument("--ep-rank", type=int, default=0, help="with --ep on one GPU: which rank's share to time")
     ap.add_argument("--persistent-decode", action="store_true",
                     help="small bf16 batches: the whole layer in one persistent cooperative launch (opt-in)")
     return ap.parse_args()
@@ -204,7 +210,12 @@ def workload_config(args):
 
 
 class Workload:
-    def __init__(self, cfg, T, seed, weights, persistent_decode=False):
+    """One batch of the layer on this GPU.  ``ep = (first, count, reduce)``: this
+    rank's share of an expert-parallel layer (experts [first, first + count) of
+    cfg.E; ``reduce``: all-reduce the output over the process group after the
+    share, which completes the layer on every rank)."""
+
+    def __init__(self, cfg, T, seed, weights, persistent_decode=False, ep=None):
         from moe_layer_top_b200 import ops
         self.ops = ops
         self.cfg, self.T = cfg, T
@@ -212,8 +223,10 @@ class Workload:
         self.w13, self.w2, self.s13, self.s2 = weights
         self.x = inputs.make_tokens(cfg, T, seed, device=dev)
         self.routing = inputs.make_routing(cfg, T, seed, device=dev)
-        self.p = ops.problem(T, cfg.E, cfg.topk, cfg.H, cfg.I, fp8=cfg.fp8, mx=cfg.mx,
-                             persistent_decode=persistent_decode)
+        self.ep = ep
+        first, count = (0, cfg.E) if ep is None else ep[:2]
+        self.p = ops.problem(T, count, cfg.topk, cfg.H, cfg.I, fp8=cfg.fp8, mx=cfg.mx,
+                             persistent_decode=persistent_decode, num_global_experts=cfg.E, first_expert=first)
         self.q = ops.resolve_problem(self.p)
         self.ws = ops.alloc_workspace(self.p)
         self.out = torch.empty((T, cfg.H), dtype=torch.bfloat16, device=dev)
@@ -228,6 +241,12 @@ class Workload:
 
     def forward(self):
         self.ops.fused_forward(self.p, self.x, self.w13, self.w2, **self.kw())
+
+    def collective(self):
+        """The step's exchange: the all-reduce of an expert-parallel share (nothing otherwise)."""
+        if self.ep is not None and self.ep[2]:
+            import torch.distributed as dist
+            dist.all_reduce(self.out, op=dist.ReduceOp.SUM)
 
     def algorithmic(self):
         """Algorithmic bytes / FLOPs of the layer and of each GEMM for this routing."""
@@ -244,12 +263,13 @@ class Workload:
             w13_e = 2 * cfg.I * cfg.H * elem + (2 * cfg.I // 128) * (cfg.H // 128) * 4 * cfg.fp8
             w2_e = cfg.H * cfg.I * elem + (cfg.H // 128) * (cfg.I // 128) * 4 * cfg.fp8
         nflat = self.T * cfg.topk
+        nlocal = int(counts.sum())       # assignments run here (all of them without expert parallelism)
         route_io = self.T * cfg.E * 4 if "logits" in self.routing else nflat * 8
         rows = ntpp
         gemm1 = hit * w13_e + rows * cfg.H * elem + rows * cfg.I * elem
-        gemm2 = hit * w2_e + rows * cfg.I * elem + nflat * cfg.H * 2
+        gemm2 = hit * w2_e + rows * cfg.I * elem + nlocal * cfg.H * 2
         layer = hit * (w13_e + w2_e) + self.T * cfg.H * 2 * 2 + route_io
-        flops = 2.0 * nflat * 3 * cfg.H * cfg.I
+        flops = 2.0 * nlocal * 3 * cfg.H * cfg.I
         return {"hit_experts": hit, "padded_rows": ntpp, "layer_bytes": layer, "gemm1_bytes": gemm1,
                 "gemm2_bytes": gemm2, "flops": flops, "w13_bytes_per_expert": w13_e, "w2_bytes_per_expert": w2_e}
 
@@ -283,9 +303,20 @@ def graph_kernel_count(g):
         return None
 
 
-def make_weights(cfg, seed):
+def make_weights(cfg, seed, ep=None):
+    """The layer's weights on the GPU (with ``ep = (first, count, ...)`` only
+    experts [first, first + count), drawn exactly as in the full layer)."""
     from moe_layer_top_b200 import ops
-    w13, w2 = inputs.make_weights(cfg, seed, device="cuda")
+    if ep is None:
+        w13, w2 = inputs.make_weights(cfg, seed, device="cuda")
+    else:
+        first, count = ep[:2]
+        w13 = torch.empty((count, 2 * cfg.I, cfg.H), dtype=torch.bfloat16, device="cuda")
+        w2 = torch.empty((count, cfg.H, cfg.I), dtype=torch.bfloat16, device="cuda")
+        for i in range(count):
+            a, b = inputs.make_expert_weights(cfg, first + i, seed, device="cuda")
+            w13[i].copy_(a)
+            w2[i].copy_(b)
     if cfg.fp8:
         quant = ops.quantize_weights_mxfp8 if cfg.mx else ops.quantize_weights_fp8
         q13, s13 = quant(w13)
@@ -382,6 +413,7 @@ def time_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor, world
     for _ in range(warmup):
         flush.zero_()
         g_fwd.replay()
+        wl.collective()
         flush.zero_()
         g_stg.replay()
     torch.cuda.synchronize()
@@ -393,6 +425,7 @@ def time_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor, world
         flush.zero_()
         ev[i][0].record(stream)
         g_fwd.replay()
+        wl.collective()     # outside the graph: no NCCL call is ever captured
         ev[i][1].record(stream)
     torch.cuda.synchronize()
     barrier(world)
@@ -425,6 +458,7 @@ def e2e_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor):
         ops.fused_forward(wl.p, x_d, wl.w13, wl.w2, logits=r_d.get("logits"), topk_ids=r_d.get("topk_ids"),
                           topk_weights=r_d.get("topk_weights"), w13_scale=wl.s13, w2_scale=wl.s2, out=wl.out,
                           ws=wl.ws)
+        wl.collective()
         out_h.copy_(wl.out, non_blocking=True)
 
     for _ in range(warmup):
@@ -517,11 +551,20 @@ def run_ours(args, rank, world, local):
     sweep_T = [T_head] if args.tokens else sorted(cfg.tokens)
     peaks = measured_peaks()
     flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    weights = make_weights(cfg, args.seed)
+    ep = None
+    if args.ep:
+        # expert parallelism: on N ranks each runs its share and the output is
+        # all-reduced; on one GPU the step is one rank's share alone
+        from moe_layer_top_b200.expert_parallel import expert_shard
+        if world not in (1, args.ep):
+            raise SystemExit(f"--ep {args.ep} runs on {args.ep} ranks, or on one GPU (one share)")
+        ep_rank = rank if world > 1 else args.ep_rank
+        ep = (*expert_shard(cfg.E, args.ep, ep_rank), world > 1)
+    weights = make_weights(cfg, args.seed, ep)
     results = {}
     with ClockSampler(local) as clocks:
         for T in sweep_T:
-            wl = Workload(cfg, T, args.seed, weights, args.persistent_decode)
+            wl = Workload(cfg, T, args.seed, weights, args.persistent_decode, ep)
             steps = args.steps if T == T_head else max(3, args.steps // 2)
             step_ms, per_stage, wall, n_kernels = time_steps(wl, steps, args.warmup, flush, world)
             total_ms = max_over_ranks(float(step_ms.sum()), world)
@@ -532,7 +575,9 @@ def run_ours(args, rank, world, local):
     wl = head["wl"]
     alg = wl.algorithmic()
     K = head["steps"]
-    value = world * T_head * K / (head["total_ms"] / 1e3)
+    # replicas: every rank runs its own batch; expert parallelism: the ranks share one batch
+    layer_copies = 1 if ep is not None else world
+    value = layer_copies * T_head * K / (head["total_ms"] / 1e3)
     ms_per_step = head["total_ms"] / K
     stage_ms = head["per_stage"].mean(axis=0)
     # dominant kernel: the stage with the largest share of the step
@@ -541,7 +586,7 @@ def run_ours(args, rank, world, local):
     dom_bytes = {"gemm1": alg["gemm1_bytes"], "gemm2": alg["gemm2_bytes"]}.get(dom_name)
     if dom_bytes is None:
         dom_bytes = alg["layer_bytes"]
-    traffic = traffic_record(dom_name, args.workload, T_head)
+    traffic = traffic_record(dom_name, args.workload, T_head) if ep is None else None
     # FLOPs of the dominant GEMM (GEMM1 = 2/3 of the layer, GEMM2 = 1/3)
     dom_flops = alg["flops"] * {"gemm1": 2.0 / 3.0, "gemm2": 1.0 / 3.0}.get(dom_name, 1.0)
     # tensor-core peak for the arithmetic dtype: measured bf16 (burst: the kernel
@@ -564,7 +609,7 @@ def run_ours(args, rank, world, local):
         a = r["wl"].algorithmic()
         ms = r["total_ms"] / r["steps"]
         sm = r["per_stage"].mean(axis=0)
-        sweep.append({"T": T, "tokens_per_s": round(world * T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
+        sweep.append({"T": T, "tokens_per_s": round(layer_copies * T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
                       "layer_hbm_frac": round(a["layer_bytes"] / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
                       "tflops": round(a["flops"] / (ms / 1e3) / 1e12, 2),
                       "layer_tc_frac": round(a["flops"] / (ms / 1e3) / 1e12 /
@@ -576,15 +621,24 @@ def run_ours(args, rank, world, local):
                       "block_m": r["wl"].q.block_m})
     e2e_ms, h2d, d2h = e2e_steps(wl, K, args.warmup, flush)
     e2e_ms = max_over_ranks(e2e_ms, world)
-    e2e = {"value": round(world * T_head * K / (e2e_ms / 1e3), 1), "unit": "tokens/s", "h2d_bytes_per_step": h2d,
-           "d2h_bytes_per_step": d2h}
+    e2e = {"value": round(layer_copies * T_head * K / (e2e_ms / 1e3), 1), "unit": "tokens/s",
+           "h2d_bytes_per_step": h2d, "d2h_bytes_per_step": d2h}
+    if ep is None:
+        parallelism, scaling, wl_name = f"replicas{world}", "weak", cfg.name
+    elif world > 1:
+        parallelism, scaling = f"ep{world} (experts [{ep[0]}, {ep[0] + ep[1]}) on rank 0; NCCL all-reduce)", "strong"
+        wl_name = cfg.name
+    else:
+        parallelism, scaling = (f"ep{args.ep} share of rank {args.ep_rank} (experts [{ep[0]}, {ep[0] + ep[1]})) "
+                                f"alone on one GPU: no all-reduce", "strong")
+        wl_name = f"{cfg.name} (one EP={args.ep} share)"
     line = {
         "metric": "fused-MoE tokens/s; % HBM roofline (decode), % FP8/BF16 TC peak (prefill)",
         "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": "weak", "vs_baseline": None,
+        "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": scaling, "vs_baseline": None,
         "dtype": ("mxfp8_e4m3" if cfg.mx else "fp8_e4m3") if cfg.fp8 else "bf16", "data": "synthetic",
-        "config": {"workload": f"{cfg.name}: H={cfg.H} E={cfg.E} topk={cfg.topk} I={cfg.I} T={T_head}",
-                   "global_batch": world * T_head, "tokens_per_gpu": T_head, "parallelism": f"replicas{world}",
+        "config": {"workload": f"{wl_name}: H={cfg.H} E={cfg.E} topk={cfg.topk} I={cfg.I} T={T_head}",
+                   "global_batch": layer_copies * T_head, "tokens_per_gpu": T_head, "parallelism": parallelism,
                    "weights": ("mxfp8 e4m3 + per-32 e8m0 scales" if cfg.mx else "fp8 e4m3 + 128x128 fp32 scales")
                    if cfg.fp8 else "bf16",
                    "routing": cfg.routing, "l2": "flushed (256 MiB write) before every step, outside the timing",
@@ -600,7 +654,7 @@ def run_ours(args, rank, world, local):
         "gpu_launches_source": "kernel nodes of the captured forward graph" if head["kernels"] else "formula",
         "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline:
+    if rank == 0 and world == 1 and not args.no_cpu_baseline and ep is None:
         line["cpu_baseline"] = cpu_baseline(cfg, T_head, args.seed, args.cpu_budget)
     return line
 
