@@ -17,7 +17,7 @@ Sources (web pages the method is taken from):
        (blog.secrett2633.cloud).
 [PPLX] "Hosting von Qwen auf Blackwell" (perplexity.ai).
 
-Readings where the pages are silent (each also listed in the design doc):
+Readings where the pages are silent:
 
 * route: experts are chosen on the raw logits (softmax is monotone), equal
   logits go to the lower expert index; weights are the softmax over all
