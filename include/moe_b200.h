@@ -166,10 +166,11 @@ typedef struct moe_workspace_layout {
   int64_t sorted_token_ids; /* int32 [capacity] */
   int64_t expert_ids;       /* int32 [capacity / block_m] */
   int64_t num_tokens_post_padded; /* int32 */
-  int64_t expert_counts;    /* int32 [E] */
+  int64_t expert_counts;    /* int32 [E] (local experts under expert parallelism) */
   int64_t expert_offsets;   /* int32 [E + 1] */
   int64_t align_scratch;    /* int32 [chunks * E] */
-  int64_t pos_of_flat;      /* int32 [T*topk]: sorted row of each assignment, -1 for a bad id (FP8 / MXFP8) */
+  int64_t pos_of_flat;      /* int32 [T*topk]: sorted row of each assignment, -1 for a bad id or another
+                               rank's expert (FP8 / MXFP8 except two-SM tiles, and every expert-parallel call) */
   int64_t a1;               /* GEMM1 token rows.  Normal tiles: x rows in sorted order [capacity, H], bf16 or
                                E4M3 (padding rows unspecified).  Swap-AB: one row per token [T, H] -- E4M3
                                codes (FP8) or bf16(x * w) (router weight on the input) -- gathered by TMA;
@@ -177,7 +178,8 @@ typedef struct moe_workspace_layout {
   int64_t a1_scale;         /* fp32 [H/128, capacity] (FP8, K-block major); E8M0 SF atoms of [capacity, H] (MXFP8) */
   int64_t a2;               /* bf16 or E4M3 [capacity, I] activation in sorted order (padding rows unspecified) */
   int64_t a2_scale;         /* fp32 [I/128, capacity] (FP8, K-block major); E8M0 SF atoms of [capacity, I] (MXFP8) */
-  int64_t y;                /* bf16 [T*topk, H] weighted expert outputs */
+  int64_t y;                /* bf16 [T*topk, H] weighted expert outputs (rows of other ranks' assignments
+                               unwritten under expert parallelism) */
   int64_t partials;         /* fp32 split-K partial sums of the swap-AB GEMMs (swap-AB only) */
   int64_t total_bytes;
   int32_t capacity;         /* rows of sorted_token_ids */
