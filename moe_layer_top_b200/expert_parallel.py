@@ -59,9 +59,27 @@ class ExpertParallelMoE:
             self.world_size, self.rank = 1, 0
         self.E, self.T = int(E), int(T)
         self.first_expert, self.num_local = expert_shard(self.E, self.world_size, self.rank)
-        self.problem = ops.problem(T, self.num_local, topk, H, I, num_global_experts=self.E,
-                                   first_expert=self.first_expert, **problem_kw)
-        self._ws = None
+        self._shape = (int(topk), int(H), int(I), dict(problem_kw))
+        self._problems, self._workspaces = {}, {}
+        self.problem = self.problem_for(self.T)
+
+    def problem_for(self, T: int):
+        """This rank's moe_problem for a batch of T tokens."""
+        if T not in self._problems:
+            topk, H, I, kw = self._shape
+            self._problems[T] = ops.problem(T, self.num_local, topk, H, I, num_global_experts=self.E,
+                                            first_expert=self.first_expert, **kw)
+        return self._problems[T]
+
+    def workspace_for(self, T: int, device) -> torch.Tensor:
+        """The workspace of this rank's T-token problem on ``device`` (allocated on first use)."""
+        dev = torch.device(device)
+        if dev.type == "cuda" and dev.index is None:
+            dev = torch.device("cuda", torch.cuda.current_device())
+        key = (T, str(dev))
+        if key not in self._workspaces:
+            self._workspaces[key] = ops.alloc_workspace(self.problem_for(T), dev)
+        return self._workspaces[key]
 
     def local_experts(self, w: torch.Tensor) -> torch.Tensor:
         """This rank's experts of a full per-expert tensor [E, ...] (weights or their scales)."""
@@ -70,19 +88,39 @@ class ExpertParallelMoE:
         return w[self.first_expert:self.first_expert + self.num_local]
 
     def local_forward(self, x, w13, w2, **kw) -> torch.Tensor:
-        """This rank's partial output: the sum over each token's assignments to local experts."""
-        if x.shape[0] != self.T:
-            raise ValueError(f"x has {x.shape[0]} tokens, the problem {self.T}")
-        if self._ws is None or self._ws.device != x.device:
-            self._ws = ops.alloc_workspace(self.problem, x.device)
-        return ops.fused_forward(self.problem, x, w13, w2, ws=self._ws, **kw)
+        """This rank's partial output for x [T', H] (any T'): the sum over each token's assignments
+        to local experts."""
+        T = x.shape[0]
+        return ops.fused_forward(self.problem_for(T), x, w13, w2, ws=self.workspace_for(T, x.device), **kw)
 
-    def forward(self, x, w13, w2, **kw) -> torch.Tensor:
-        out = self.local_forward(x, w13, w2, **kw)
-        if self.world_size > 1:
-            if not (dist.is_available() and dist.is_initialized()):
-                raise RuntimeError("forward of a rank of several needs the process group; use local_forward")
-            dist.all_reduce(out, op=dist.ReduceOp.SUM, group=self.group)
+    def forward(self, x, w13, w2, *, chunks: int = 1, **kw) -> torch.Tensor:
+        """The layer's output on every rank.  ``chunks`` > 1 splits the batch into that many
+        contiguous token ranges: the all-reduce of a range is issued asynchronously (NCCL runs it
+        on its own stream) while the next range computes, so the exchange overlaps the GEMMs
+        (every output row depends only on its own token, so the result is the same layer)."""
+        if self.world_size > 1 and not (dist.is_available() and dist.is_initialized()):
+            raise RuntimeError("forward of a rank of several needs the process group; use local_forward")
+        T = x.shape[0]
+        chunks = max(1, min(int(chunks), T))
+        if chunks == 1:
+            out = self.local_forward(x, w13, w2, **kw)
+            if self.world_size > 1:
+                dist.all_reduce(out, op=dist.ReduceOp.SUM, group=self.group)
+            return out
+        out = kw.pop("out", None)
+        if out is None:
+            out = torch.empty((T, x.shape[1]), dtype=torch.bfloat16, device=x.device)
+        per_token = ("logits", "topk_ids", "topk_weights")
+        bounds = [(c * T) // chunks for c in range(chunks + 1)]
+        pending = []
+        for c0, c1 in zip(bounds, bounds[1:]):
+            sub = {k: (v[c0:c1] if k in per_token and v is not None else v) for k, v in kw.items()}
+            self.local_forward(x[c0:c1], w13, w2, out=out[c0:c1], **sub)
+            if self.world_size > 1:
+                pending.append(dist.all_reduce(out[c0:c1], op=dist.ReduceOp.SUM, group=self.group,
+                                               async_op=True))
+        for work in pending:
+            work.wait()
         return out
 
     __call__ = forward

@@ -28,14 +28,19 @@ def _free_port():
 class _OracleLocal(ExpertParallelMoE):
     """The rank-local part from the oracle (CPU); everything else is the product class."""
 
-    def local_forward(self, x, w13, w2, **kw):
-        p = self.problem
-        assert w13.shape[0] == p.E == self.num_local and w2.shape[0] == p.E
+    def local_forward(self, x, w13, w2, out=None, **kw):
+        p = self.problem_for(x.shape[0])
+        assert p.T == x.shape[0] and w13.shape[0] == p.E == self.num_local and w2.shape[0] == p.E
         logits = kw.get("logits")
+        assert logits is None or logits.shape == (p.T, self.E)
         r = O.moe_forward(x.double().numpy(), w13.double().numpy(), w2.double().numpy(), p.topk,
                           logits=None if logits is None else logits.numpy(),
                           expert_range=(p.first_expert, p.E))
-        return torch.from_numpy(r["out"]).to(torch.bfloat16)
+        res = torch.from_numpy(r["out"]).to(torch.bfloat16)
+        if out is None:
+            return res
+        out.copy_(res)
+        return out
 
 
 def _worker(rank, world, port, T, out_dir):
@@ -49,7 +54,9 @@ def _worker(rank, world, port, T, out_dir):
         logits = inputs.make_routing(cfg, T, 11)["logits"]
         layer = _OracleLocal(T, cfg.E, cfg.topk, cfg.H, cfg.I)
         out = layer.forward(x, layer.local_experts(w13), layer.local_experts(w2), logits=logits)
-        torch.save({"out": out, "first": layer.first_expert, "count": layer.num_local,
+        # the chunked form: three token ranges, each all-reduced asynchronously
+        chunked = layer.forward(x, layer.local_experts(w13), layer.local_experts(w2), logits=logits, chunks=3)
+        torch.save({"out": out, "chunked": chunked, "first": layer.first_expert, "count": layer.num_local,
                     "problem": (layer.problem.E, layer.problem.num_global_experts, layer.problem.first_expert)},
                    os.path.join(out_dir, f"rank{rank}.pt"))
     finally:
@@ -73,6 +80,7 @@ def test_expert_parallel_ranks_complete_the_layer(tmp_path, world):
     full = O.moe_forward(x, w13.double().numpy(), w2.double().numpy(), cfg.topk, logits=logits)["out"]
     for r in res:
         torch.testing.assert_close(r["out"], res[0]["out"], rtol=0, atol=0)
+        torch.testing.assert_close(r["chunked"], r["out"], rtol=0, atol=0)
     got = res[0]["out"].double().numpy()
     assert np.abs(got).max() > 0
     # partials rounded to bf16, summed in bf16 by the collective: a few bf16 ulps of the layer

@@ -88,7 +88,7 @@ class Sharded:
 
 
 def _check_routing_and_alignment(s, m, ref_ids):
-    v = ops.workspace_views(m.problem, m._ws)
+    v = ops.workspace_views(m.problem, m.workspace_for(s.T, "cuda"))
     q = v["problem"]
     if "logits" in s.routing:
         np.testing.assert_array_equal(v["topk_ids"].cpu().numpy(), ref_ids)
@@ -104,7 +104,7 @@ def _check_routing_and_alignment(s, m, ref_ids):
     assert np.all(pos[~local] == -1)
     st = v["sorted_token_ids"].cpu().numpy()
     np.testing.assert_array_equal(st[pos[local]], np.nonzero(local)[0])
-    assert ops.read_status(m.problem, m._ws) == ops.MOE_STATUS_OK
+    assert ops.read_status(m.problem, m.workspace_for(s.T, "cuda")) == ops.MOE_STATUS_OK
 
 
 CASES = [
@@ -152,7 +152,7 @@ def test_rank_without_tokens_writes_zeros():
     s = Sharded(cfg, 20, 2, seed=1, routing={"topk_ids": ids, "topk_weights": w})
     parts = s.run()
     assert torch.count_nonzero(parts[1]).item() == 0
-    assert ops.read_status(s.ranks[1].problem, s.ranks[1]._ws) == ops.MOE_STATUS_OK
+    assert ops.read_status(s.ranks[1].problem, s.ranks[1].workspace_for(s.T, "cuda")) == ops.MOE_STATUS_OK
     assert_close(parts[0].float().cpu().numpy(), s.oracle()["out"], False)
 
 
@@ -166,8 +166,8 @@ def test_invalid_global_id_is_reported_and_skipped():
     s = Sharded(cfg, 12, 2, seed=2, routing={"topk_ids": ids, "topk_weights": w})
     s.run()
     for m in s.ranks:
-        assert ops.read_status(m.problem, m._ws) == ops.MOE_STATUS_BAD_EXPERT_ID
-        pos = ops.workspace_views(m.problem, m._ws)["pos_of_flat"].cpu().numpy()
+        assert ops.read_status(m.problem, m.workspace_for(s.T, "cuda")) == ops.MOE_STATUS_BAD_EXPERT_ID
+        pos = ops.workspace_views(m.problem, m.workspace_for(s.T, "cuda"))["pos_of_flat"].cpu().numpy()
         assert pos[3 * 2 + 1] == -1
 
 
@@ -197,3 +197,31 @@ def test_one_share_is_the_plain_layer_bit_for_bit():
     plain = ops.fused_forward(p, s.x, s.w13, s.w2, logits=s.routing["logits"])
     torch.cuda.synchronize()
     assert torch.equal(part, plain)
+
+
+def test_chunked_forward_is_the_layer():
+    """forward(chunks=3) on one rank: three token ranges, each its own problem and workspace."""
+    cfg = inputs.make_custom_config("ep_chunks", E=16, topk=4, H=512, I=256, fp8=True, routing="logits",
+                                    tokens=(50,))
+    s = Sharded(cfg, 50, 1, seed=8)
+    m = s.ranks[0]
+    kw = dict(logits=s.routing["logits"], w13_scale=s.s13, w2_scale=s.s2)
+    whole = m.forward(s.x, s.w13, s.w2, **kw).clone()
+    chunked = m.forward(s.x, s.w13, s.w2, chunks=3, **kw)
+    torch.cuda.synchronize()
+    ref = s.oracle()["out"]
+    assert_close(chunked.float().cpu().numpy(), ref, True)
+    assert_close(whole.float().cpu().numpy(), ref, True)
+    assert sorted(m._problems) == [16, 17, 50]
+
+
+def test_share_of_a_token_range_is_those_rows():
+    cfg = inputs.make_custom_config("ep_rows", E=12, topk=3, H=256, I=128, routing="logits", tokens=(40,))
+    s = Sharded(cfg, 40, 3, seed=9)
+    s.run()
+    m = s.ranks[1]
+    sub = m.local_forward(s.x[8:29], m.local_experts(s.w13), m.local_experts(s.w2),
+                          logits=s.routing["logits"][8:29])
+    torch.cuda.synchronize()
+    ref = s.oracle(expert_range=(m.first_expert, m.num_local), tokens=np.arange(8, 29))["out"]
+    assert_close(sub.float().cpu().numpy(), ref, False)
