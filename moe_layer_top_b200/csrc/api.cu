@@ -446,7 +446,7 @@ extern "C" {
 
 const char* moe_last_error_string(void) { return g_last_error.c_str(); }
 
-int32_t moe_version(void) { return 100; }
+int32_t moe_version(void) { return 200; }
 
 int moe_selftest_wait_timeout(uint32_t timeout_us, int32_t* status, uint64_t* waited_ns, void* stream) {
   if (timeout_us < 1 || timeout_us > 1000000)

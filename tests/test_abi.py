@@ -37,7 +37,7 @@ def test_header_declares_the_boundary():
 def test_library_exports_every_declared_symbol(L):
     for name in _declared():
         assert hasattr(L, name), name
-    assert L.moe_version() == 100
+    assert L.moe_version() == 200
 
 
 def test_struct_sizes_match_header():
