@@ -340,6 +340,71 @@ MOE_API int moe_read_status(const moe_problem* p, void* ws, int32_t clear, int32
  */
 MOE_API int moe_selftest_wait_timeout(uint32_t timeout_us, int32_t* status, uint64_t* waited_ns, void* stream);
 
+/*
+ * Fused combine + all-reduce of an expert-parallel layer ("Hosting von Qwen
+ * auf Blackwell", section "MoE Dispatch - Combine", "Experten-Parallel": the
+ * local accumulation, then an all-reduce over the ranks; section
+ * "All-Reduce": the reduction split over the ranks, each reducing a part and
+ * sending it to the others).  It replaces the combine stage of every rank's
+ * moe_forward_stages(..., MOE_STAGE_ROUTE, MOE_STAGE_COMBINE, ...) call and
+ * the all-reduce after it: one kernel per rank, over peer memory, in which
+ * every token chunk is first summed locally (partial), then reduced by the
+ * rank that owns the chunk (chunk c: rank c % world) from every rank's partial
+ * in rank order (fp32, one bf16 rounding) and stored into every rank's out.
+ *
+ * moe_allreduce_rank: one rank's buffers, as mapped in the calling process
+ * (peers' through CUDA peer mappings; all ranks on one NVLink domain).
+ *   y, pos_of_flat  that rank's workspace regions "y" and "pos_of_flat"
+ *                   (moe_get_workspace_layout of its expert-parallel problem);
+ *                   read by that rank only.
+ *   partial, out    bf16 [T, H] each, 16-byte aligned; partial is read and out
+ *                   written by every rank.
+ *   flags           int32 [moe_combine_allreduce_flag_count(T, world)], zeroed
+ *                   once by the caller before the first call; the same flags
+ *                   serve every later call of the same T and world.
+ *   status          int32 status word of the rank (e.g. its workspace's).
+ * epoch: 1 for the first call on a set of flags, then one more per call (the
+ * flags remember the last epoch; nothing is reset between calls).  Every rank
+ * passes the same epoch, T, topk, H and world.
+ * timeout_us (1 .. 10 000 000): every wait on another rank is bounded; one
+ * that runs out records MOE_STATUS_WAIT_TIMEOUT | 0x31 (chunk ready) or 0x32
+ * (chunk done) in the rank's status word, the rank's later waits of that call
+ * give up at once, and the kernel returns (out is then incomplete).
+ * Buffers of rows [0, T) only; T = 0 is a no-op.
+ */
+#define MOE_MAX_RANKS 16
+
+typedef struct moe_allreduce_rank {
+  const void* y;
+  const int32_t* pos_of_flat;
+  void* partial;
+  void* out;
+  int32_t* flags;
+  int32_t* status;
+} moe_allreduce_rank;
+
+/* int32 entries of each rank's flags array for T tokens over world ranks (0 on bad arguments). */
+MOE_API int32_t moe_combine_allreduce_flag_count(int32_t T, int32_t world);
+
+/*
+ * This rank's kernel (ranks[0 .. world) as mapped here, `rank` = the caller's
+ * index).  Every rank must launch it for the same epoch; each returns when
+ * its own out is complete.  The y, pos_of_flat and status of the other ranks
+ * are not read and may be NULL.
+ */
+MOE_API int moe_combine_allreduce(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t rank,
+                                  const moe_allreduce_rank* ranks, uint32_t epoch, uint32_t timeout_us,
+                                  void* stream);
+
+/*
+ * Every rank's kernel as one cooperative launch on the current device, with
+ * all ranks' buffers in this device's memory: the same device code and the
+ * same flag protocol, for testing the exchange on one GPU.
+ */
+MOE_API int moe_combine_allreduce_emulated(int32_t T, int32_t topk, int32_t H, int32_t world,
+                                           const moe_allreduce_rank* ranks, uint32_t epoch, uint32_t timeout_us,
+                                           void* stream);
+
 /* Library version: major * 10000 + minor * 100 + patch. */
 MOE_API int32_t moe_version(void);
 

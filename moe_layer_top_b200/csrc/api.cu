@@ -7,6 +7,7 @@
 #include <cstring>
 #include <string>
 
+#include "allreduce.h"
 #include "kernels.h"
 #include "moe_b200.h"
 
@@ -563,6 +564,58 @@ int moe_quantize_weights_mxfp8(const void* w, int64_t batches, int32_t rows, int
   if (rc != MOE_OK) return rc;
   cudaError_t e = moe::launch_quantize_weights_mx(w, batches, rows, cols, codes, sf, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "quantize");
+}
+
+int32_t moe_combine_allreduce_flag_count(int32_t T, int32_t world) {
+  if (T < 0 || world < 1 || world > MOE_MAX_RANKS) return 0;
+  return 2 * moe::allreduce_chunks(T, world).nchunks + 1;
+}
+
+namespace {
+
+int combine_allreduce(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t rank, const moe_allreduce_rank* ranks,
+                      uint32_t epoch, uint32_t timeout_us, void* stream, bool emulated) {
+  if (world < 1 || world > MOE_MAX_RANKS) return fail(MOE_ERR_INVALID, "allreduce: world %d outside [1, %d]", world,
+                                                      MOE_MAX_RANKS);
+  if (!emulated && (rank < 0 || rank >= world)) return fail(MOE_ERR_INVALID, "allreduce: rank %d outside [0, %d)", rank,
+                                                            world);
+  if (T < 0 || topk < 1 || topk > 32 || H <= 0 || H % 128)
+    return fail(MOE_ERR_INVALID, "allreduce: T=%d topk=%d H=%d (H a positive multiple of 128)", T, topk, H);
+  if (static_cast<int64_t>(T) * topk >= (int64_t(1) << 31)) return fail(MOE_ERR_INVALID, "allreduce: T * topk overflows");
+  if (epoch < 1 || epoch > 0x7FFFFFFFu) return fail(MOE_ERR_INVALID, "allreduce: epoch %u outside [1, 2^31)", epoch);
+  if (timeout_us < 1 || timeout_us > 10000000u)
+    return fail(MOE_ERR_INVALID, "allreduce: timeout_us %u outside [1, 10000000]", timeout_us);
+  if (T == 0) return MOE_OK;
+  if (!ranks) return fail(MOE_ERR_INVALID, "allreduce: ranks is NULL");
+  moe::AllreduceRank r[moe::kMaxRanks] = {};
+  for (int p = 0; p < world; ++p) {
+    const moe_allreduce_rank& q = ranks[p];
+    const bool own = emulated || p == rank;  // buffers this rank's kernel reads besides partial / out / flags
+    if (!q.partial || !q.out || !q.flags || (own && (!q.y || !q.pos_of_flat || !q.status)))
+      return fail(MOE_ERR_INVALID, "allreduce: NULL buffer of rank %d", p);
+    if (!aligned(q.partial, 16) || !aligned(q.out, 16) || !aligned(q.flags, 4) || (own && !aligned(q.y, 16)) ||
+        (own && !aligned(q.pos_of_flat, 4)) || (own && !aligned(q.status, 4)))
+      return fail(MOE_ERR_INVALID, "allreduce: misaligned buffer of rank %d", p);
+    r[p] = moe::AllreduceRank{q.y, q.pos_of_flat, q.partial, q.out, q.flags, q.status};
+  }
+  int sms = 0;
+  int rc = device_check(&sms);
+  if (rc != MOE_OK) return rc;
+  cudaError_t e = moe::launch_combine_allreduce(r, world, emulated ? -1 : rank, T, topk, H, epoch,
+                                                1000ull * timeout_us, sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "allreduce");
+}
+
+}  // namespace
+
+int moe_combine_allreduce(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t rank,
+                          const moe_allreduce_rank* ranks, uint32_t epoch, uint32_t timeout_us, void* stream) {
+  return combine_allreduce(T, topk, H, world, rank, ranks, epoch, timeout_us, stream, false);
+}
+
+int moe_combine_allreduce_emulated(int32_t T, int32_t topk, int32_t H, int32_t world, const moe_allreduce_rank* ranks,
+                                   uint32_t epoch, uint32_t timeout_us, void* stream) {
+  return combine_allreduce(T, topk, H, world, 0, ranks, epoch, timeout_us, stream, true);
 }
 
 int moe_resolve_problem(moe_problem* p) {

@@ -44,8 +44,11 @@ EXPORTED = (
     "moe_last_error_string", "moe_route", "moe_align_capacity", "moe_align_workspace_size", "moe_align",
     "moe_quantize_weights_fp8", "moe_resolve_problem", "moe_workspace_size", "moe_get_workspace_layout",
     "moe_fused_forward", "moe_forward_stages", "moe_read_status", "moe_version", "moe_align_noalloc",
-    "moe_selftest_wait_timeout", "moe_quantize_weights_mxfp8",
+    "moe_selftest_wait_timeout", "moe_quantize_weights_mxfp8", "moe_combine_allreduce_flag_count",
+    "moe_combine_allreduce", "moe_combine_allreduce_emulated",
 )
+
+MAX_RANKS = 16
 
 
 class MoeProblem(ctypes.Structure):
@@ -57,6 +60,11 @@ class MoeProblem(ctypes.Structure):
         ("persistent_decode", ctypes.c_int32), ("num_global_experts", ctypes.c_int32),
         ("first_expert", ctypes.c_int32), ("reserved", ctypes.c_int32 * 1),
     ]
+
+
+class MoeAllreduceRank(ctypes.Structure):
+    _fields_ = [("y", ctypes.c_void_p), ("pos_of_flat", ctypes.c_void_p), ("partial", ctypes.c_void_p),
+                ("out", ctypes.c_void_p), ("flags", ctypes.c_void_p), ("status", ctypes.c_void_p)]
 
 
 class MoeWorkspaceLayout(ctypes.Structure):
@@ -106,6 +114,11 @@ def lib():
             "moe_forward_stages": (ctypes.c_int, [P, vp, vp, vp, vp, vp, vp, vp, vp, vp, vp, sz, i32, i32, vp]),
             "moe_read_status": (ctypes.c_int, [P, vp, i32, ctypes.POINTER(i32), vp]),
             "moe_selftest_wait_timeout": (ctypes.c_int, [ctypes.c_uint32, vp, vp, vp]),
+            "moe_combine_allreduce_flag_count": (i32, [i32, i32]),
+            "moe_combine_allreduce": (ctypes.c_int, [i32, i32, i32, i32, i32, ctypes.POINTER(MoeAllreduceRank),
+                                                     ctypes.c_uint32, ctypes.c_uint32, vp]),
+            "moe_combine_allreduce_emulated": (ctypes.c_int, [i32, i32, i32, i32, ctypes.POINTER(MoeAllreduceRank),
+                                                              ctypes.c_uint32, ctypes.c_uint32, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -320,3 +333,35 @@ def selftest_wait_timeout(timeout_us: int, stream=None):
     _check(lib().moe_selftest_wait_timeout(int(timeout_us), _ptr(st), _ptr(waited), _stream(stream)))
     torch.cuda.synchronize()
     return int(st.item()), int(waited.item())
+
+
+# ----------------------------------------------------------------------------- fused combine + all-reduce
+def combine_allreduce_flag_count(T: int, world: int) -> int:
+    """int32 entries of each rank's flags array (zero them once before the first call)."""
+    return int(lib().moe_combine_allreduce_flag_count(int(T), int(world)))
+
+
+def _ranks_array(ranks):
+    arr = (MoeAllreduceRank * len(ranks))()
+    for i, r in enumerate(ranks):
+        for name in ("y", "pos_of_flat", "partial", "out", "flags", "status"):
+            v = r.get(name)
+            setattr(arr[i], name, None if v is None else (v if isinstance(v, int) else v.data_ptr()))
+    return arr
+
+
+def combine_allreduce(T, topk, H, rank, ranks, epoch, timeout_us=2_000_000, stream=None):
+    """This rank's fused combine + all-reduce.  ``ranks``: one dict per rank with ``y``,
+    ``pos_of_flat``, ``partial``, ``out``, ``flags``, ``status`` -- tensors, or device addresses
+    (ints) of peers' buffers as mapped in this process."""
+    arr = _ranks_array(ranks)
+    _check(lib().moe_combine_allreduce(int(T), int(topk), int(H), len(ranks), int(rank), arr, int(epoch),
+                                       int(timeout_us), _stream(stream)))
+
+
+def combine_allreduce_emulated(T, topk, H, ranks, epoch, timeout_us=2_000_000, stream=None):
+    """Every rank's fused combine + all-reduce in one cooperative launch on this GPU (all buffers local)."""
+    arr = _ranks_array(ranks)
+    _check(lib().moe_combine_allreduce_emulated(int(T), int(topk), int(H), len(ranks), arr, int(epoch),
+                                                int(timeout_us), _stream(stream)))
+

@@ -251,3 +251,33 @@ def test_expert_parallel_plan(L):
         assert lay.pos_of_flat >= 0
         # capacity bounds the local rows: every assignment may land here
         assert lay.capacity == ops.align_capacity(64, 8, 16, lay.block_m)
+
+
+def test_combine_allreduce_chunking_and_argument_errors(L):
+    """Flag counts follow the chunking rule (at most 64 chunks per rank, at most 1024, whole tokens);
+    every argument error is caught before a launch."""
+    assert ops.combine_allreduce_flag_count(64, 8) == 2 * 64 + 1        # one token per chunk
+    assert ops.combine_allreduce_flag_count(16384, 4) == 2 * 256 + 1    # 64 tokens per chunk
+    assert ops.combine_allreduce_flag_count(100000, 16) == 2 * 1021 + 1  # 98 tokens, ceil(100000 / 98) chunks
+    assert ops.combine_allreduce_flag_count(0, 2) == 1
+    assert ops.combine_allreduce_flag_count(8, 0) == 0 and ops.combine_allreduce_flag_count(8, 17) == 0
+    g = 1 << 20
+    good = [dict(y=g, pos_of_flat=g, partial=g, out=g, flags=g, status=g) for _ in range(2)]
+
+    def rc(T=8, topk=2, H=256, rank=0, ranks=good, epoch=1, timeout=1000, emulated=False):
+        arr = ops._ranks_array(ranks) if ranks is not None else None
+        if emulated:
+            return L.moe_combine_allreduce_emulated(T, topk, H, len(ranks or []), arr, epoch, timeout, None)
+        return L.moe_combine_allreduce(T, topk, H, len(ranks or []), rank, arr, epoch, timeout, None)
+
+    inv = ops.MOE_ERR_INVALID
+    assert rc(rank=2) == inv and rc(rank=-1) == inv
+    assert rc(H=100) == inv and rc(topk=0) == inv and rc(T=-1) == inv
+    assert rc(epoch=0) == inv and rc(timeout=0) == inv and rc(timeout=20_000_000) == inv
+    assert rc(ranks=[dict(good[0])] * 17) == inv
+    assert rc(ranks=[good[0], dict(good[1], partial=None)]) == inv
+    assert rc(ranks=[good[0], dict(good[1], out=g + 8)]) == inv                # out must be 16-byte aligned
+    assert rc(ranks=[dict(good[0], y=None), good[1]]) == inv                   # own y is read
+    assert rc(ranks=[good[0], dict(good[1], y=None, pos_of_flat=None, status=None)]) != inv  # a peer's are not
+    assert rc(ranks=[good[0], dict(good[1], y=None)], emulated=True) == inv     # emulated: every rank's are read
+    assert rc(T=0) == ops.MOE_OK                                                # nothing to do
