@@ -356,7 +356,9 @@ MOE_API int moe_selftest_wait_timeout(uint32_t timeout_us, int32_t* status, uint
  * (peers' through CUDA peer mappings; all ranks on one NVLink domain).
  *   y, pos_of_flat  that rank's workspace regions "y" and "pos_of_flat"
  *                   (moe_get_workspace_layout of its expert-parallel problem);
- *                   read by that rank only.
+ *                   read by that rank only.  pos_of_flat may be NULL when
+ *                   every assignment has a row on the rank (a problem without
+ *                   expert parallelism, whose layout may have no such region).
  *   partial, out    bf16 [T, H] each, 16-byte aligned; partial is read and out
  *                   written by every rank.
  *   flags           int32 [moe_combine_allreduce_flag_count(T, world)], zeroed

@@ -135,7 +135,7 @@ __global__ void __launch_bounds__(kThreadsAr) combine_allreduce_kernel(const ArP
       float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
       for (int j = 0; j < P.topk; ++j) {
         const long long f = t * P.topk + j;
-        if (R.pos_of_flat[f] < 0) continue;  // another rank's expert: no row here
+        if (R.pos_of_flat && R.pos_of_flat[f] < 0) continue;  // another rank's expert: no row here
         float g[8];
         unpack8(y[f * vecs + v], g);
 #pragma unroll

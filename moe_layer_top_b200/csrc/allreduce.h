@@ -14,7 +14,7 @@ constexpr int kMaxArChunks = 1024;  // token chunks per call (flags: 2 ints per 
 // peer mapping).  All bf16 arrays are row-major with rows of H elements.
 struct AllreduceRank {
   const void* y;               // bf16 [T*topk, H]: the rank's GEMM2 rows (read by that rank only)
-  const int32_t* pos_of_flat;  // int32 [T*topk]: -1 = the assignment has no row on that rank
+  const int32_t* pos_of_flat;  // int32 [T*topk]: -1 = the assignment has no row on that rank (NULL: all have)
   void* partial;               // bf16 [T, H]: the rank's local sums (read by every rank)
   void* out;                   // bf16 [T, H]: the layer (written by every rank)
   int* flags;                  // int32 [2 * chunks + 1]: chunk ready / chunk done epochs, abort epoch

@@ -591,7 +591,7 @@ int combine_allreduce(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t
   for (int p = 0; p < world; ++p) {
     const moe_allreduce_rank& q = ranks[p];
     const bool own = emulated || p == rank;  // buffers this rank's kernel reads besides partial / out / flags
-    if (!q.partial || !q.out || !q.flags || (own && (!q.y || !q.pos_of_flat || !q.status)))
+    if (!q.partial || !q.out || !q.flags || (own && (!q.y || !q.status)))
       return fail(MOE_ERR_INVALID, "allreduce: NULL buffer of rank %d", p);
     if (!aligned(q.partial, 16) || !aligned(q.out, 16) || !aligned(q.flags, 4) || (own && !aligned(q.y, 16)) ||
         (own && !aligned(q.pos_of_flat, 4)) || (own && !aligned(q.status, 4)))

@@ -10,11 +10,16 @@ Here the rank-local part is one ``moe_fused_forward`` call whose problem names
 the rank's expert range (``num_global_experts`` / ``first_expert``): the
 library routes over all experts, its alignment keeps the local assignments and
 its combine sums only their rows.  The reduction is a ``torch.distributed``
-all-reduce (NCCL over NVLink between GPUs).  Each rank holds the weights of its
-experts only: ``E / world_size`` of them, contiguous.
+all-reduce (NCCL over NVLink between GPUs), or, with ``fused_allreduce``, the
+library's own kernel that does the combine and the all-reduce together over
+peer memory (symmetric buffers from ``torch.distributed._symmetric_memory``).
+Each rank holds the weights of its experts only: ``E / world_size`` of them,
+contiguous.
 """
 
 from __future__ import annotations
+
+import os
 
 import torch
 import torch.distributed as dist
@@ -46,7 +51,7 @@ class ExpertParallelMoE:
     """
 
     def __init__(self, T: int, E: int, topk: int, H: int, I: int, *, group=None, rank=None, world_size=None,
-                 **problem_kw):
+                 fused_allreduce: bool = False, **problem_kw):
         self.group = group
         if (rank is None) != (world_size is None):
             raise ValueError("give both rank and world_size, or neither")
@@ -62,6 +67,8 @@ class ExpertParallelMoE:
         self._shape = (int(topk), int(H), int(I), dict(problem_kw))
         self._problems, self._workspaces = {}, {}
         self.problem = self.problem_for(self.T)
+        self.fused_allreduce = bool(fused_allreduce)
+        self._exchange = {}
 
     def problem_for(self, T: int):
         """This rank's moe_problem for a batch of T tokens."""
@@ -93,13 +100,70 @@ class ExpertParallelMoE:
         T = x.shape[0]
         return ops.fused_forward(self.problem_for(T), x, w13, w2, ws=self.workspace_for(T, x.device), **kw)
 
+    def _exchange_for(self, T: int, device):
+        """Symmetric buffers (partial, out, flags) of the fused combine + all-reduce for T tokens,
+        their peer addresses, and the call counter (collective on first use for a T)."""
+        if T in self._exchange:
+            return self._exchange[T]
+        # the kernel uses plain peer loads and stores only: no multicast object is bound to these buffers
+        os.environ.setdefault("TORCH_SYMM_MEM_DISABLE_MULTICAST", "1")
+        import torch.distributed._symmetric_memory as symm_mem
+        group = self.group if self.group is not None else dist.group.WORLD
+        if not symm_mem.is_symm_mem_enabled_for_group(group.group_name):
+            symm_mem.enable_symm_mem_for_group(group.group_name)
+        H = self._shape[1]
+        partial = symm_mem.empty((T, H), dtype=torch.bfloat16, device=device)
+        out = symm_mem.empty((T, H), dtype=torch.bfloat16, device=device)
+        flags = symm_mem.empty((ops.combine_allreduce_flag_count(T, self.world_size),), dtype=torch.int32,
+                               device=device)
+        flags.zero_()
+        handles = [symm_mem.rendezvous(t, group) for t in (partial, out, flags)]
+        torch.cuda.synchronize(device)
+        dist.barrier(group)      # every rank's flags are zero before any rank signals
+        p = self.problem_for(T)
+        ws = self.workspace_for(T, device)
+        lay = ops.workspace_layout(p)
+        base = ws.data_ptr()
+        ranks = []
+        for r in range(self.world_size):
+            d = {"partial": handles[0].buffer_ptrs[r], "out": handles[1].buffer_ptrs[r],
+                 "flags": handles[2].buffer_ptrs[r]}
+            if r == self.rank:
+                d.update(y=base + lay.y, status=base + lay.status,
+                         pos_of_flat=base + lay.pos_of_flat if lay.pos_of_flat >= 0 else None)
+            ranks.append(d)
+        ex = {"partial": partial, "out": out, "flags": flags, "handles": handles, "ranks": ranks, "epoch": 0}
+        self._exchange[T] = ex
+        return ex
+
+    def _fused_forward(self, x, w13, w2, **kw) -> torch.Tensor:
+        T = x.shape[0]
+        user_out = kw.pop("out", None)
+        ex = self._exchange_for(T, x.device)
+        p = self.problem_for(T)
+        ops.forward_stages(p, x, w13, w2, ops.STAGE_ROUTE, ops.STAGE_COMBINE, out=ex["out"],
+                           ws=self.workspace_for(T, x.device), **kw)
+        ex["epoch"] += 1
+        topk, H = self._shape[0], self._shape[1]
+        ops.combine_allreduce(T, topk, H, self.rank, ex["ranks"], ex["epoch"])
+        if user_out is None:
+            return ex["out"]
+        user_out.copy_(ex["out"])
+        return user_out
+
     def forward(self, x, w13, w2, *, chunks: int = 1, **kw) -> torch.Tensor:
         """The layer's output on every rank.  ``chunks`` > 1 splits the batch into that many
         contiguous token ranges: the all-reduce of a range is issued asynchronously (NCCL runs it
         on its own stream) while the next range computes, so the exchange overlaps the GEMMs
-        (every output row depends only on its own token, so the result is the same layer)."""
+        (every output row depends only on its own token, so the result is the same layer).
+        With ``fused_allreduce`` the stages up to GEMM2 run, then one kernel per rank sums the
+        local rows and all-reduces them over peer memory (``chunks`` is not used); the result is
+        then a symmetric buffer that the next call of the same T overwrites, unless ``out`` is
+        given."""
         if self.world_size > 1 and not (dist.is_available() and dist.is_initialized()):
             raise RuntimeError("forward of a rank of several needs the process group; use local_forward")
+        if self.fused_allreduce:
+            return self._fused_forward(x, w13, w2, **kw)
         T = x.shape[0]
         chunks = max(1, min(int(chunks), T))
         if chunks == 1:

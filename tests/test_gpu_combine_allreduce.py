@@ -116,3 +116,54 @@ def test_rank_whose_peer_never_runs_gives_up():
     again = s.run()
     for a, b in zip(again, plain):
         assert torch.equal(a, b)
+
+
+_SYMMETRIC_CHILD = r"""
+import os, sys
+import torch
+import torch.distributed as dist
+sys.path.insert(0, os.environ["MOE_TEST_ROOT"])
+from moe_layer_top_b200 import inputs, ops
+from moe_layer_top_b200.expert_parallel import ExpertParallelMoE
+
+torch.cuda.set_device(0)
+dist.init_process_group("nccl", rank=0, world_size=1, init_method="tcp://127.0.0.1:" + os.environ["MOE_TEST_PORT"],
+                        device_id=torch.device("cuda:0"))
+cfg = inputs.make_custom_config("ar_symm", E=16, topk=4, H=512, I=256, routing="logits", tokens=(40,))
+T, dev = 40, torch.device("cuda:0")
+w13, w2 = inputs.make_weights(cfg, 6, device=dev)
+x = inputs.make_tokens(cfg, T, 6, device=dev)
+logits = inputs.make_routing(cfg, T, 6, device=dev)["logits"]
+plain = ops.fused_forward(ops.problem(T, cfg.E, cfg.topk, cfg.H, cfg.I), x, w13, w2, logits=logits)
+m = ExpertParallelMoE(T, cfg.E, cfg.topk, cfg.H, cfg.I, fused_allreduce=True)
+a = m.forward(x, w13, w2, logits=logits).clone()
+b = m.forward(x, w13, w2, logits=logits, out=torch.empty_like(plain))
+torch.cuda.synchronize()
+assert torch.equal(a, plain) and torch.equal(b, plain), "fused path differs from the plain layer"
+flags = m._exchange[T]["flags"]
+assert int(flags[:-1].min()) == 2 and int(flags[:-1].max()) == 2 and int(flags[-1]) == 0, flags
+assert ops.read_status(m.problem, m.workspace_for(T, dev)) == ops.MOE_STATUS_OK
+del m, a, b
+torch.cuda.synchronize()
+dist.destroy_process_group()
+print("SYMMETRIC-OK")
+"""
+
+
+def test_fused_allreduce_through_symmetric_memory_one_rank():
+    """The production wiring (symmetric buffers, rendezvous, peer addresses, epochs) on a one-rank
+    NCCL group: the fused kernel then reduces one partial, so the result is the plain layer bit for
+    bit.  Run in a child process so its process group ends with it."""
+    import os
+    import socket
+    import subprocess
+    import sys
+    with socket.socket() as sk:
+        sk.bind(("127.0.0.1", 0))
+        port = sk.getsockname()[1]
+    root = os.path.dirname(os.path.dirname(os.path.abspath(__file__)))
+    env = dict(os.environ, MOE_TEST_ROOT=root, MOE_TEST_PORT=str(port), MASTER_ADDR="127.0.0.1",
+               TORCH_SYMM_MEM_DISABLE_MULTICAST="1", NCCL_NVLS_ENABLE="0")
+    res = subprocess.run([sys.executable, "-c", _SYMMETRIC_CHILD], env=env, capture_output=True, text=True,
+                         timeout=240)
+    assert res.returncode == 0 and "SYMMETRIC-OK" in res.stdout, (res.stdout[-2000:], res.stderr[-3000:])
