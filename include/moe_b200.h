@@ -407,6 +407,28 @@ MOE_API int moe_combine_allreduce_emulated(int32_t T, int32_t topk, int32_t H, i
                                            const moe_allreduce_rank* ranks, uint32_t epoch, uint32_t timeout_us,
                                            void* stream);
 
+/*
+ * Reduce-scatter form, for data parallelism combined with expert parallelism
+ * (the page's decoders: each rank serves its own requests while the experts
+ * are sharded).  Every rank brings T tokens; the ranks' x and routing inputs
+ * are gathered (rank r's tokens are rows [r*T, (r+1)*T) of the gathered
+ * batch), every rank runs its expert share on the whole gathered batch of
+ * world * T tokens, and this kernel then leaves in each rank's out [T, H] the
+ * layer for that rank's own tokens: partial is [world * T, H], y and
+ * pos_of_flat are those of the share's world*T-token problem, out is [T, H],
+ * flags has moe_combine_reduce_scatter_flag_count(T, world) entries.  Rank r
+ * reduces its own rows from every rank's partial (rank order, fp32, one bf16
+ * rounding) and stores only into its own out.  Epochs, time limits, status
+ * codes and the emulated form are as for the all-reduce above.
+ */
+MOE_API int32_t moe_combine_reduce_scatter_flag_count(int32_t T, int32_t world);
+MOE_API int moe_combine_reduce_scatter(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t rank,
+                                       const moe_allreduce_rank* ranks, uint32_t epoch, uint32_t timeout_us,
+                                       void* stream);
+MOE_API int moe_combine_reduce_scatter_emulated(int32_t T, int32_t topk, int32_t H, int32_t world,
+                                                const moe_allreduce_rank* ranks, uint32_t epoch,
+                                                uint32_t timeout_us, void* stream);
+
 /* Library version: major * 10000 + minor * 100 + patch. */
 MOE_API int32_t moe_version(void);
 

@@ -19,6 +19,13 @@
 //      rank's out and releases flags[chunks + c] = epoch on every rank;
 //   3. the kernel returns once every chunk of this rank's out is done.
 //
+// Reduce-scatter form (data parallel + expert parallel: every rank brings its
+// own T tokens, the layer runs on the ranks' gathered batch of world * T
+// tokens, and each rank keeps the rows of its own tokens): the partial covers
+// the whole gathered batch, the chunks of rank r's rows belong to rank r, and
+// the owner stores the sum into its own out [T, H] only.  The done flags
+// still go to every rank: they tell a rank that its partial has been read.
+//
 // Flags hold the epoch of the last call that passed them (the caller counts
 // calls from 1 and zeroes the flags once), so nothing is reset between
 // calls.  A rank cannot start call e+1 before its call e returned, i.e. before
@@ -44,10 +51,24 @@ constexpr int kWhereArReady = 0x31, kWhereArDone = 0x32;
 
 struct ArParams {
   AllreduceRank r[kMaxRanks];
-  int world, rank, T, topk, H, chunk_tokens, nchunks, ctas_per_rank;
+  int world, rank, topk, H, chunk_tokens, ctas_per_rank;
+  int scatter;        // 0: all-reduce of [rows, H]; 1: reduce-scatter of [world * rows, H]
+  int rows;           // rows of out (per rank)
+  int nchunks_rows;   // chunks of `rows` rows
+  int nchunks;        // all chunks: nchunks_rows, or world * nchunks_rows when scattering
   uint32_t epoch;
   unsigned long long timeout_ns;
 };
+
+// token rows [t0, t1) of chunk c in the partial buffers
+__device__ __forceinline__ void chunk_rows(const ArParams& P, int c, long long& t0, long long& t1) {
+  const int region = P.scatter ? c / P.nchunks_rows : 0;
+  const int local = P.scatter ? c - region * P.nchunks_rows : c;
+  const long long base = static_cast<long long>(region) * P.rows;
+  t0 = base + static_cast<long long>(local) * P.chunk_tokens;
+  t1 = t0 + P.chunk_tokens;
+  if (t1 > base + P.rows) t1 = base + P.rows;
+}
 
 struct alignas(16) bf16x8 {
   __nv_bfloat162 h[4];
@@ -126,9 +147,9 @@ __global__ void __launch_bounds__(kThreadsAr) combine_allreduce_kernel(const ArP
 
   // 1. local accumulation of this CTA's chunks, each published when written
   for (int c = cta; c < P.nchunks; c += P.ctas_per_rank) {
-    const int t0 = c * P.chunk_tokens;
-    const int t1 = min(P.T, t0 + P.chunk_tokens);
-    const long long n = static_cast<long long>(t1 - t0) * vecs;
+    long long t0, t1;
+    chunk_rows(P, c, t0, t1);
+    const long long n = (t1 - t0) * vecs;
     for (long long i = threadIdx.x; i < n; i += kThreadsAr) {
       const long long t = t0 + i / vecs;
       const int v = static_cast<int>(i % vecs);
@@ -150,9 +171,14 @@ __global__ void __launch_bounds__(kThreadsAr) combine_allreduce_kernel(const ArP
     }
   }
 
-  // 2. this rank's chunks: every rank's partial -> sum -> every rank's out
+  // 2. this rank's chunks: every rank's partial -> sum -> every rank's out (all-reduce) or this
+  //    rank's out (reduce-scatter)
+  const int c_first = P.scatter ? me * P.nchunks_rows : me;
+  const int c_end = P.scatter ? (me + 1) * P.nchunks_rows : P.nchunks;
+  const int c_step = P.scatter ? 1 : P.world;
+  const long long out_base = P.scatter ? static_cast<long long>(me) * P.rows * vecs : 0;
   int k = 0;
-  for (int c = me; c < P.nchunks; c += P.world, ++k) {
+  for (int c = c_first; c < c_end; c += c_step, ++k) {
     if (k % P.ctas_per_rank != cta) continue;
     if (threadIdx.x == 0) {
       bool good = true;
@@ -162,11 +188,11 @@ __global__ void __launch_bounds__(kThreadsAr) combine_allreduce_kernel(const ArP
     }
     __syncthreads();
     if (ok) {
-      const int t0 = c * P.chunk_tokens;
-      const int t1 = min(P.T, t0 + P.chunk_tokens);
-      const long long n = static_cast<long long>(t1 - t0) * vecs;
+      long long t0, t1;
+      chunk_rows(P, c, t0, t1);
+      const long long n = (t1 - t0) * vecs;
       for (long long i = threadIdx.x; i < n; i += kThreadsAr) {
-        const long long e = static_cast<long long>(t0) * vecs + i;
+        const long long e = t0 * vecs + i;
         float acc[8] = {0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f, 0.f};
         for (int p = 0; p < P.world; ++p) {
           float g[8];
@@ -175,7 +201,10 @@ __global__ void __launch_bounds__(kThreadsAr) combine_allreduce_kernel(const ArP
           for (int q = 0; q < 8; ++q) acc[q] += g[q];
         }
         const uint4 o = pack8(acc);
-        for (int p = 0; p < P.world; ++p) static_cast<uint4*>(P.r[p].out)[e] = o;
+        if (P.scatter)
+          static_cast<uint4*>(R.out)[e - out_base] = o;
+        else
+          for (int p = 0; p < P.world; ++p) static_cast<uint4*>(P.r[p].out)[e] = o;
       }
     }
     __syncthreads();
@@ -186,7 +215,8 @@ __global__ void __launch_bounds__(kThreadsAr) combine_allreduce_kernel(const ArP
     __syncthreads();  // ok is rewritten for the next chunk
   }
 
-  // 3. return once every chunk of this rank's out is complete
+  // 3. return once every chunk has been reduced: this rank's out is complete and no owner still
+  //    reads its partial
   if (threadIdx.x == 0) {
     for (int c = cta; c < P.nchunks; c += P.ctas_per_rank)
       if (!wait_epoch(R.flags + P.nchunks + c, P.epoch, abort_word, R.status, P.timeout_ns, kWhereArDone)) break;
@@ -195,7 +225,16 @@ __global__ void __launch_bounds__(kThreadsAr) combine_allreduce_kernel(const ArP
 
 }  // namespace
 
-AllreduceChunks allreduce_chunks(int T, int world) {
+AllreduceChunks allreduce_chunks(int T, int world, bool scatter) {
+  if (scatter) {
+    // chunks of each rank's rows; the world regions together stay within kMaxArChunks
+    if (T <= 0) return {1, 0};
+    long long target = 64;
+    if (target * world > kMaxArChunks) target = kMaxArChunks / world;
+    if (target > T) target = T;
+    const int ct = static_cast<int>((T + target - 1) / target);
+    return {ct, world * ((T + ct - 1) / ct)};
+  }
   if (T <= 0) return {1, 0};
   long long target = 64LL * world;  // a few chunks per CTA of every rank at decode sizes
   if (target > kMaxArChunks) target = kMaxArChunks;
@@ -205,9 +244,9 @@ AllreduceChunks allreduce_chunks(int T, int world) {
 }
 
 cudaError_t launch_combine_allreduce(const AllreduceRank* ranks, int world, int rank, int T, int topk, int H,
-                                     uint32_t epoch, unsigned long long timeout_ns, int num_sms,
+                                     bool scatter, uint32_t epoch, unsigned long long timeout_ns, int num_sms,
                                      cudaStream_t stream) {
-  const AllreduceChunks ch = allreduce_chunks(T, world);
+  const AllreduceChunks ch = allreduce_chunks(T, world, scatter);
   if (ch.nchunks == 0) return cudaSuccess;
   int per_sm = 0;
   cudaError_t e = cudaOccupancyMaxActiveBlocksPerMultiprocessor(&per_sm, combine_allreduce_kernel, kThreadsAr, 0);
@@ -222,11 +261,13 @@ cudaError_t launch_combine_allreduce(const AllreduceRank* ranks, int world, int 
   for (int p = 0; p < world; ++p) P.r[p] = ranks[p];
   P.world = world;
   P.rank = rank;
-  P.T = T;
   P.topk = topk;
   P.H = H;
   P.chunk_tokens = ch.chunk_tokens;
+  P.scatter = scatter ? 1 : 0;
+  P.rows = T;
   P.nchunks = ch.nchunks;
+  P.nchunks_rows = scatter ? ch.nchunks / world : ch.nchunks;
   P.ctas_per_rank = ctas;
   P.epoch = epoch;
   P.timeout_ns = timeout_ns;

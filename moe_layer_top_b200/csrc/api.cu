@@ -568,20 +568,26 @@ int moe_quantize_weights_mxfp8(const void* w, int64_t batches, int32_t rows, int
 
 int32_t moe_combine_allreduce_flag_count(int32_t T, int32_t world) {
   if (T < 0 || world < 1 || world > MOE_MAX_RANKS) return 0;
-  return 2 * moe::allreduce_chunks(T, world).nchunks + 1;
+  return 2 * moe::allreduce_chunks(T, world, false).nchunks + 1;
+}
+
+int32_t moe_combine_reduce_scatter_flag_count(int32_t T, int32_t world) {
+  if (T < 0 || world < 1 || world > MOE_MAX_RANKS) return 0;
+  return 2 * moe::allreduce_chunks(T, world, true).nchunks + 1;
 }
 
 namespace {
 
 int combine_allreduce(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t rank, const moe_allreduce_rank* ranks,
-                      uint32_t epoch, uint32_t timeout_us, void* stream, bool emulated) {
+                      uint32_t epoch, uint32_t timeout_us, void* stream, bool emulated, bool scatter) {
   if (world < 1 || world > MOE_MAX_RANKS) return fail(MOE_ERR_INVALID, "allreduce: world %d outside [1, %d]", world,
                                                       MOE_MAX_RANKS);
   if (!emulated && (rank < 0 || rank >= world)) return fail(MOE_ERR_INVALID, "allreduce: rank %d outside [0, %d)", rank,
                                                             world);
   if (T < 0 || topk < 1 || topk > 32 || H <= 0 || H % 128)
     return fail(MOE_ERR_INVALID, "allreduce: T=%d topk=%d H=%d (H a positive multiple of 128)", T, topk, H);
-  if (static_cast<int64_t>(T) * topk >= (int64_t(1) << 31)) return fail(MOE_ERR_INVALID, "allreduce: T * topk overflows");
+  if (static_cast<int64_t>(T) * topk * (scatter ? world : 1) >= (int64_t(1) << 31))
+    return fail(MOE_ERR_INVALID, "allreduce: rows * topk overflows int32");
   if (epoch < 1 || epoch > 0x7FFFFFFFu) return fail(MOE_ERR_INVALID, "allreduce: epoch %u outside [1, 2^31)", epoch);
   if (timeout_us < 1 || timeout_us > 10000000u)
     return fail(MOE_ERR_INVALID, "allreduce: timeout_us %u outside [1, 10000000]", timeout_us);
@@ -601,7 +607,7 @@ int combine_allreduce(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t
   int sms = 0;
   int rc = device_check(&sms);
   if (rc != MOE_OK) return rc;
-  cudaError_t e = moe::launch_combine_allreduce(r, world, emulated ? -1 : rank, T, topk, H, epoch,
+  cudaError_t e = moe::launch_combine_allreduce(r, world, emulated ? -1 : rank, T, topk, H, scatter, epoch,
                                                 1000ull * timeout_us, sms, static_cast<cudaStream_t>(stream));
   return e == cudaSuccess ? MOE_OK : cuda_fail(e, "allreduce");
 }
@@ -610,12 +616,23 @@ int combine_allreduce(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t
 
 int moe_combine_allreduce(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t rank,
                           const moe_allreduce_rank* ranks, uint32_t epoch, uint32_t timeout_us, void* stream) {
-  return combine_allreduce(T, topk, H, world, rank, ranks, epoch, timeout_us, stream, false);
+  return combine_allreduce(T, topk, H, world, rank, ranks, epoch, timeout_us, stream, false, false);
 }
 
 int moe_combine_allreduce_emulated(int32_t T, int32_t topk, int32_t H, int32_t world, const moe_allreduce_rank* ranks,
                                    uint32_t epoch, uint32_t timeout_us, void* stream) {
-  return combine_allreduce(T, topk, H, world, 0, ranks, epoch, timeout_us, stream, true);
+  return combine_allreduce(T, topk, H, world, 0, ranks, epoch, timeout_us, stream, true, false);
+}
+
+int moe_combine_reduce_scatter(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t rank,
+                               const moe_allreduce_rank* ranks, uint32_t epoch, uint32_t timeout_us, void* stream) {
+  return combine_allreduce(T, topk, H, world, rank, ranks, epoch, timeout_us, stream, false, true);
+}
+
+int moe_combine_reduce_scatter_emulated(int32_t T, int32_t topk, int32_t H, int32_t world,
+                                        const moe_allreduce_rank* ranks, uint32_t epoch, uint32_t timeout_us,
+                                        void* stream) {
+  return combine_allreduce(T, topk, H, world, 0, ranks, epoch, timeout_us, stream, true, true);
 }
 
 int moe_resolve_problem(moe_problem* p) {

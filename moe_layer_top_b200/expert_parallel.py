@@ -48,10 +48,18 @@ class ExpertParallelMoE:
     returns the whole layer's output on every rank.  ``rank`` / ``world_size``
     default to the process group's (one rank without one); given explicitly
     they select a share without a group, for :meth:`local_forward` alone.
+
+    ``data_parallel``: every rank brings its OWN batch of T tokens (the page's
+    decoders: data parallel and expert parallel together).  The ranks' x and
+    routing inputs are gathered, each rank runs its share on the gathered batch
+    of world * T tokens, and a reduce-scatter leaves each rank the layer for its
+    own tokens.  (The page's decoders exchange only the chosen (token, expert)
+    rows with a sparse all-to-all; the gather sends every token to every rank,
+    which costs the same bytes when a token's k experts span most ranks.)
     """
 
     def __init__(self, T: int, E: int, topk: int, H: int, I: int, *, group=None, rank=None, world_size=None,
-                 fused_allreduce: bool = False, **problem_kw):
+                 fused_allreduce: bool = False, data_parallel: bool = False, **problem_kw):
         self.group = group
         if (rank is None) != (world_size is None):
             raise ValueError("give both rank and world_size, or neither")
@@ -66,7 +74,8 @@ class ExpertParallelMoE:
         self.first_expert, self.num_local = expert_shard(self.E, self.world_size, self.rank)
         self._shape = (int(topk), int(H), int(I), dict(problem_kw))
         self._problems, self._workspaces = {}, {}
-        self.problem = self.problem_for(self.T)
+        self.data_parallel = bool(data_parallel)
+        self.problem = self.problem_for(self.T * (self.world_size if self.data_parallel else 1))
         self.fused_allreduce = bool(fused_allreduce)
         self._exchange = {}
 
@@ -101,8 +110,9 @@ class ExpertParallelMoE:
         return ops.fused_forward(self.problem_for(T), x, w13, w2, ws=self.workspace_for(T, x.device), **kw)
 
     def _exchange_for(self, T: int, device):
-        """Symmetric buffers (partial, out, flags) of the fused combine + all-reduce for T tokens,
-        their peer addresses, and the call counter (collective on first use for a T)."""
+        """Symmetric buffers (partial, out, flags) of the fused combine + all-reduce for T tokens
+        (per rank, with ``data_parallel``), their peer addresses, and the call counter (collective
+        on first use for a T)."""
         if T in self._exchange:
             return self._exchange[T]
         # the kernel uses plain peer loads and stores only: no multicast object is bound to these buffers
@@ -112,16 +122,17 @@ class ExpertParallelMoE:
         if not symm_mem.is_symm_mem_enabled_for_group(group.group_name):
             symm_mem.enable_symm_mem_for_group(group.group_name)
         H = self._shape[1]
-        partial = symm_mem.empty((T, H), dtype=torch.bfloat16, device=device)
+        rows = T * self.world_size if self.data_parallel else T     # the batch the share runs on
+        count = (ops.combine_reduce_scatter_flag_count if self.data_parallel else ops.combine_allreduce_flag_count)
+        partial = symm_mem.empty((rows, H), dtype=torch.bfloat16, device=device)
         out = symm_mem.empty((T, H), dtype=torch.bfloat16, device=device)
-        flags = symm_mem.empty((ops.combine_allreduce_flag_count(T, self.world_size),), dtype=torch.int32,
-                               device=device)
+        flags = symm_mem.empty((count(T, self.world_size),), dtype=torch.int32, device=device)
         flags.zero_()
         handles = [symm_mem.rendezvous(t, group) for t in (partial, out, flags)]
         torch.cuda.synchronize(device)
         dist.barrier(group)      # every rank's flags are zero before any rank signals
-        p = self.problem_for(T)
-        ws = self.workspace_for(T, device)
+        p = self.problem_for(rows)
+        ws = self.workspace_for(rows, device)
         lay = ops.workspace_layout(p)
         base = ws.data_ptr()
         ranks = []
@@ -136,20 +147,52 @@ class ExpertParallelMoE:
         self._exchange[T] = ex
         return ex
 
-    def _fused_forward(self, x, w13, w2, **kw) -> torch.Tensor:
-        T = x.shape[0]
+    def _fused_forward(self, T, x, w13, w2, **kw) -> torch.Tensor:
+        """x: the batch the share runs on (the gathered one with ``data_parallel``); T: tokens of
+        this rank's output."""
+        rows = x.shape[0]
         user_out = kw.pop("out", None)
         ex = self._exchange_for(T, x.device)
-        p = self.problem_for(T)
+        p = self.problem_for(rows)
         ops.forward_stages(p, x, w13, w2, ops.STAGE_ROUTE, ops.STAGE_COMBINE, out=ex["out"],
-                           ws=self.workspace_for(T, x.device), **kw)
+                           ws=self.workspace_for(rows, x.device), **kw)
         ex["epoch"] += 1
         topk, H = self._shape[0], self._shape[1]
-        ops.combine_allreduce(T, topk, H, self.rank, ex["ranks"], ex["epoch"])
+        exchange = ops.combine_reduce_scatter if self.data_parallel else ops.combine_allreduce
+        exchange(T, topk, H, self.rank, ex["ranks"], ex["epoch"])
         if user_out is None:
             return ex["out"]
         user_out.copy_(ex["out"])
         return user_out
+
+    def _gather(self, x, kw):
+        """The ranks' batches and per-token routing inputs, concatenated in rank order."""
+        if self.world_size == 1:
+            return x, dict(kw)
+
+        def gather(t):
+            full = torch.empty((t.shape[0] * self.world_size,) + tuple(t.shape[1:]), dtype=t.dtype, device=t.device)
+            dist.all_gather_into_tensor(full, t.contiguous(), group=self.group)
+            return full
+        kw = dict(kw)
+        for key in ("logits", "topk_ids", "topk_weights"):
+            if kw.get(key) is not None:
+                kw[key] = gather(kw[key])
+        return gather(x), kw
+
+    def _data_parallel_forward(self, x, w13, w2, **kw) -> torch.Tensor:
+        T = x.shape[0]
+        xg, kw = self._gather(x, kw)
+        if self.fused_allreduce:
+            return self._fused_forward(T, xg, w13, w2, **kw)
+        user_out = kw.pop("out", None)
+        full = self.local_forward(xg, w13, w2, **kw)      # this rank's partial for every rank's tokens
+        out = user_out if user_out is not None else torch.empty((T, x.shape[1]), dtype=full.dtype,
+                                                                device=full.device)
+        if self.world_size == 1:
+            return out.copy_(full) if user_out is not None else full
+        dist.reduce_scatter_tensor(out, full, op=dist.ReduceOp.SUM, group=self.group)
+        return out
 
     def forward(self, x, w13, w2, *, chunks: int = 1, **kw) -> torch.Tensor:
         """The layer's output on every rank.  ``chunks`` > 1 splits the batch into that many
@@ -157,13 +200,15 @@ class ExpertParallelMoE:
         on its own stream) while the next range computes, so the exchange overlaps the GEMMs
         (every output row depends only on its own token, so the result is the same layer).
         With ``fused_allreduce`` the stages up to GEMM2 run, then one kernel per rank sums the
-        local rows and all-reduces them over peer memory (``chunks`` is not used); the result is
-        then a symmetric buffer that the next call of the same T overwrites, unless ``out`` is
-        given."""
+        local rows and all-reduces (with ``data_parallel``: reduce-scatters) them over peer
+        memory; the result is then a symmetric buffer that the next call of the same T
+        overwrites, unless ``out`` is given.  ``chunks`` applies to the NCCL all-reduce only."""
         if self.world_size > 1 and not (dist.is_available() and dist.is_initialized()):
             raise RuntimeError("forward of a rank of several needs the process group; use local_forward")
+        if self.data_parallel:
+            return self._data_parallel_forward(x, w13, w2, **kw)
         if self.fused_allreduce:
-            return self._fused_forward(x, w13, w2, **kw)
+            return self._fused_forward(x.shape[0], x, w13, w2, **kw)
         T = x.shape[0]
         chunks = max(1, min(int(chunks), T))
         if chunks == 1:

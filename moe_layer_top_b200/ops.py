@@ -45,7 +45,8 @@ EXPORTED = (
     "moe_quantize_weights_fp8", "moe_resolve_problem", "moe_workspace_size", "moe_get_workspace_layout",
     "moe_fused_forward", "moe_forward_stages", "moe_read_status", "moe_version", "moe_align_noalloc",
     "moe_selftest_wait_timeout", "moe_quantize_weights_mxfp8", "moe_combine_allreduce_flag_count",
-    "moe_combine_allreduce", "moe_combine_allreduce_emulated",
+    "moe_combine_allreduce", "moe_combine_allreduce_emulated", "moe_combine_reduce_scatter_flag_count",
+    "moe_combine_reduce_scatter", "moe_combine_reduce_scatter_emulated",
 )
 
 MAX_RANKS = 16
@@ -119,6 +120,13 @@ def lib():
                                                      ctypes.c_uint32, ctypes.c_uint32, vp]),
             "moe_combine_allreduce_emulated": (ctypes.c_int, [i32, i32, i32, i32, ctypes.POINTER(MoeAllreduceRank),
                                                               ctypes.c_uint32, ctypes.c_uint32, vp]),
+            "moe_combine_reduce_scatter_flag_count": (i32, [i32, i32]),
+            "moe_combine_reduce_scatter": (ctypes.c_int, [i32, i32, i32, i32, i32,
+                                                          ctypes.POINTER(MoeAllreduceRank), ctypes.c_uint32,
+                                                          ctypes.c_uint32, vp]),
+            "moe_combine_reduce_scatter_emulated": (ctypes.c_int, [i32, i32, i32, i32,
+                                                                   ctypes.POINTER(MoeAllreduceRank),
+                                                                   ctypes.c_uint32, ctypes.c_uint32, vp]),
         }
         for name, (res, args) in sig.items():
             fn = getattr(L, name)
@@ -364,4 +372,23 @@ def combine_allreduce_emulated(T, topk, H, ranks, epoch, timeout_us=2_000_000, s
     arr = _ranks_array(ranks)
     _check(lib().moe_combine_allreduce_emulated(int(T), int(topk), int(H), len(ranks), arr, int(epoch),
                                                 int(timeout_us), _stream(stream)))
+
+
+def combine_reduce_scatter_flag_count(T: int, world: int) -> int:
+    """int32 entries of each rank's flags array for the reduce-scatter form (T tokens per rank)."""
+    return int(lib().moe_combine_reduce_scatter_flag_count(int(T), int(world)))
+
+
+def combine_reduce_scatter(T, topk, H, rank, ranks, epoch, timeout_us=2_000_000, stream=None):
+    """This rank's fused combine + reduce-scatter (T tokens per rank; partial [world*T, H], out [T, H])."""
+    arr = _ranks_array(ranks)
+    _check(lib().moe_combine_reduce_scatter(int(T), int(topk), int(H), len(ranks), int(rank), arr, int(epoch),
+                                            int(timeout_us), _stream(stream)))
+
+
+def combine_reduce_scatter_emulated(T, topk, H, ranks, epoch, timeout_us=2_000_000, stream=None):
+    """Every rank's fused combine + reduce-scatter in one cooperative launch on this GPU."""
+    arr = _ranks_array(ranks)
+    _check(lib().moe_combine_reduce_scatter_emulated(int(T), int(topk), int(H), len(ranks), arr, int(epoch),
+                                                     int(timeout_us), _stream(stream)))
 

@@ -94,3 +94,37 @@ def test_expert_shard_matches_the_oracle_reading():
         expert_shard(4, 5, 0)
     with pytest.raises(ValueError):
         expert_shard(8, 2, 2)
+
+
+def _dp_worker(rank, world, port, T, out_dir):
+    """Data parallel + expert parallel: rank r brings tokens [r*T, (r+1)*T) of one global batch."""
+    os.environ.update(MASTER_ADDR="127.0.0.1", MASTER_PORT=str(port))
+    dist.init_process_group("gloo", rank=rank, world_size=world,
+                            timeout=__import__("datetime").timedelta(seconds=60))
+    try:
+        cfg = inputs.make_custom_config("ep_tiny", E=7, topk=3, H=256, I=128)
+        w13, w2 = inputs.make_weights(cfg, 12)
+        x = inputs.make_tokens(cfg, world * T, 12)[rank * T:(rank + 1) * T]
+        logits = inputs.make_routing(cfg, world * T, 12)["logits"][rank * T:(rank + 1) * T]
+        layer = _OracleLocal(T, cfg.E, cfg.topk, cfg.H, cfg.I, data_parallel=True)
+        assert layer.problem.T == world * T                    # the share runs on the gathered batch
+        out = layer.forward(x, layer.local_experts(w13), layer.local_experts(w2), logits=logits)
+        torch.save({"out": out}, os.path.join(out_dir, f"dp{rank}.pt"))
+    finally:
+        dist.destroy_process_group()
+
+
+@pytest.mark.parametrize("world", [2, 3])
+def test_data_parallel_ranks_get_their_own_tokens(tmp_path, world):
+    T = 5
+    mp.spawn(_dp_worker, args=(world, _free_port(), T, str(tmp_path)), nprocs=world, join=True)
+    cfg = inputs.make_custom_config("ep_tiny", E=7, topk=3, H=256, I=128)
+    w13, w2 = inputs.make_weights(cfg, 12)
+    x = inputs.make_tokens(cfg, world * T, 12).double().numpy()
+    logits = inputs.make_routing(cfg, world * T, 12)["logits"].numpy()
+    full = O.moe_forward(x, w13.double().numpy(), w2.double().numpy(), cfg.topk, logits=logits)["out"]
+    for r in range(world):
+        got = torch.load(os.path.join(tmp_path, f"dp{r}.pt"))["out"].double().numpy()
+        ref = full[r * T:(r + 1) * T]
+        assert got.shape == ref.shape and np.abs(ref).max() > 0
+        assert np.linalg.norm(got - ref) <= 8e-3 * np.linalg.norm(ref)

@@ -23,10 +23,13 @@ from test_gpu_expert_parallel import Sharded
 pytestmark = pytest.mark.gpu
 
 
-def _run_shares(s):
+def _run_shares(s, scatter=False):
     """Stages route .. GEMM2 of every rank's share, the share's own combine (for reference),
-    and the per-rank buffers of the fused exchange."""
+    and the per-rank buffers of the fused exchange (reduce-scatter: s.T is the gathered batch,
+    out holds s.T / world rows)."""
     T, H = s.T, s.cfg.H
+    T_out = T // s.world if scatter else T
+    count = ops.combine_reduce_scatter_flag_count if scatter else ops.combine_allreduce_flag_count
     dev = torch.device("cuda")
     ranks, plain, probs = [], [], []
     for m in s.ranks:
@@ -39,16 +42,15 @@ def _run_shares(s):
         v = ops.workspace_views(p, ws)
         ranks.append(dict(y=v["y"], pos_of_flat=v["pos_of_flat"], status=v["status"],
                           partial=torch.full((T, H), float("nan"), dtype=torch.bfloat16, device=dev),
-                          out=torch.full((T, H), float("nan"), dtype=torch.bfloat16, device=dev),
-                          flags=torch.zeros(ops.combine_allreduce_flag_count(T, s.world), dtype=torch.int32,
-                                            device=dev)))
+                          out=torch.full((T_out, H), float("nan"), dtype=torch.bfloat16, device=dev),
+                          flags=torch.zeros(count(T_out, s.world), dtype=torch.int32, device=dev)))
         plain.append(ref)
         probs.append(p)
     torch.cuda.synchronize()
     return ranks, plain, probs
 
 
-def _check(s, ranks, plain, probs, epoch):
+def _check(s, ranks, plain, probs, epoch, scatter=False):
     torch.cuda.synchronize()
     for r, p, m in zip(ranks, probs, s.ranks):
         assert ops.read_status(p, m.workspace_for(s.T, "cuda")) == ops.MOE_STATUS_OK
@@ -60,8 +62,9 @@ def _check(s, ranks, plain, probs, epoch):
     for r in ranks:
         total += r["partial"].float()                         # rank order, fp32, one rounding
     expect = total.to(torch.bfloat16)
-    for r in ranks:
-        assert torch.equal(r["out"], expect)
+    rows = s.T // s.world
+    for i, r in enumerate(ranks):
+        assert torch.equal(r["out"], expect[i * rows:(i + 1) * rows] if scatter else expect)
 
 
 CASES = [
@@ -118,6 +121,37 @@ def test_rank_whose_peer_never_runs_gives_up():
         assert torch.equal(a, b)
 
 
+RS_CASES = [
+    ("decode_bf16", inputs.CONFIGS["decode_bf16"], 4, 4, {}),
+    ("fp8_normal", inputs.make_custom_config("rs_fp8", E=16, topk=4, H=512, I=256, fp8=True, routing="logits",
+                                             tokens=(300,)), 150, 2, dict(mode=ops.MODE_NORMAL)),
+    ("wide_router_8_ranks", inputs.make_custom_config("rs_wide", E=512, topk=8, H=256, I=128, routing="logits",
+                                                      tokens=(64,)), 8, 8, {}),
+    ("uneven_shards", inputs.make_custom_config("rs_uneven", E=10, topk=3, H=256, I=128, routing="logits",
+                                                tokens=(36,)), 9, 4, {}),
+    ("many_chunks", inputs.make_custom_config("rs_chunks", E=8, topk=2, H=256, I=128, routing="logits",
+                                              tokens=(3000,)), 1500, 2, {}),
+]
+
+
+@pytest.mark.parametrize("name,cfg,T,world,kw", RS_CASES, ids=[c[0] for c in RS_CASES])
+def test_fused_combine_reduce_scatter_emulated(name, cfg, T, world, kw):
+    """Data parallel + expert parallel: T tokens per rank, every share runs on the gathered batch of
+    world * T tokens, each rank keeps the layer of its own rows."""
+    s = Sharded(cfg, world * T, world, seed=7, **kw)
+    ranks, plain, probs = _run_shares(s, scatter=True)
+    ops.combine_reduce_scatter_emulated(T, cfg.topk, cfg.H, ranks, epoch=1)
+    _check(s, ranks, plain, probs, 1, scatter=True)
+    rows = np.arange(T) if T <= 64 else np.sort(np.random.default_rng(1).choice(T, 32, replace=False))
+    for r in (0, world - 1):
+        ref = s.oracle(tokens=r * T + rows)["out"]
+        assert_close(ranks[r]["out"].float().cpu().numpy()[rows], ref, cfg.fp8)
+    for r in ranks:
+        r["out"].fill_(float("nan"))
+    ops.combine_reduce_scatter_emulated(T, cfg.topk, cfg.H, ranks, epoch=2)
+    _check(s, ranks, plain, probs, 2, scatter=True)
+
+
 _SYMMETRIC_CHILD = r"""
 import os, sys
 import torch
@@ -143,7 +177,14 @@ assert torch.equal(a, plain) and torch.equal(b, plain), "fused path differs from
 flags = m._exchange[T]["flags"]
 assert int(flags[:-1].min()) == 2 and int(flags[:-1].max()) == 2 and int(flags[-1]) == 0, flags
 assert ops.read_status(m.problem, m.workspace_for(T, dev)) == ops.MOE_STATUS_OK
-del m, a, b
+# data parallel + expert parallel, fused reduce-scatter and the NCCL form
+m2 = ExpertParallelMoE(T, cfg.E, cfg.topk, cfg.H, cfg.I, fused_allreduce=True, data_parallel=True)
+c = m2.forward(x, w13, w2, logits=logits).clone()
+m3 = ExpertParallelMoE(T, cfg.E, cfg.topk, cfg.H, cfg.I, data_parallel=True)
+d = m3.forward(x, w13, w2, logits=logits)
+torch.cuda.synchronize()
+assert torch.equal(c, plain) and torch.equal(d, plain), "data-parallel paths differ from the plain layer"
+del m, m2, m3, a, b, c, d
 torch.cuda.synchronize()
 dist.destroy_process_group()
 print("SYMMETRIC-OK")
