@@ -33,6 +33,10 @@ Readings where the pages are silent:
   once to bf16; duplicate expert ids in a row are independent assignments.
 * MXFP8: one E8M0 scale per 32 consecutive elements of a row, chosen by the
   same power-of-two rule as the per-(row,128) activation scale.
+* expert parallelism: rank r of N holds the contiguous experts
+  [floor(r*E/N), floor((r+1)*E/N)); each rank's output is the bf16 rounding of
+  its own assignments' sum; the all-reduce is the exact sum of those bf16
+  partials, rounded once.
 
 Parity pins for every function live in ``tests/test_oracle_*.py``.
 """
