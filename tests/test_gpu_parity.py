@@ -382,3 +382,27 @@ def test_swiglu_clamp_mx_and_two_sm():
         out = c.run()
         assert c.status() == ops.MOE_STATUS_OK
         assert_close(out.float().cpu().numpy(), c.oracle()["out"], fp8=True)
+
+
+PR_TEST_SHAPE = inputs.make_custom_config("pr_test_shape", E=256, topk=8, H=4096, I=256, fp8=True,
+                                          routing="uniform_ids", tokens=(1024,))
+
+
+def test_pr_analysis_test_shape():
+    """The shape of the PR analysis' own parity test (m = 1024 tokens, E = 256, H = 4096, I = 256,
+    top-8, FP8 weights with 128x128 blocks, uniform random ids, softmax weights; our generator, not
+    its seed): oracle parity on sampled tokens, and the analysis' point that a change of layout must
+    not change the numbers -- swap-AB tiles with 32 and 64 token rows per block are bitwise equal, the
+    normal orientation is within the FP8 tolerance."""
+    w = inputs.make_weights(PR_TEST_SHAPE, 123, device="cuda")
+    a = Case(PR_TEST_SHAPE, 1024, seed=123, weights=w, mode=ops.MODE_SWAP_AB, block_m=32, split_k=False)
+    out32 = a.run().clone()
+    assert a.status() == ops.MOE_STATUS_OK
+    out64 = Case(PR_TEST_SHAPE, 1024, seed=123, weights=w, mode=ops.MODE_SWAP_AB, block_m=64, split_k=False).run()
+    assert torch.equal(out32, out64)
+    tok = _sample(1024, 10, 123)
+    ref = a.oracle(tokens=tok)
+    assert_close(out32[torch.from_numpy(tok).cuda()].float().cpu().numpy(), ref["out"], fp8=True)
+    normal = Case(PR_TEST_SHAPE, 1024, seed=123, weights=w, mode=ops.MODE_NORMAL, block_m=128).run()
+    nr, mr = errors(normal.float().cpu().numpy(), out32.float().cpu().numpy())
+    assert nr <= 2e-2 and mr <= 0.05
