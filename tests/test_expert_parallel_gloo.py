@@ -128,3 +128,27 @@ def test_data_parallel_ranks_get_their_own_tokens(tmp_path, world):
         ref = full[r * T:(r + 1) * T]
         assert got.shape == ref.shape and np.abs(ref).max() > 0
         assert np.linalg.norm(got - ref) <= 8e-3 * np.linalg.norm(ref)
+
+
+def test_share_construction_without_a_group():
+    """Shares chosen explicitly (no process group): ranges, per-share problems, weight slicing and
+    the errors a caller can make."""
+    w = torch.zeros((10, 4, 2))
+    shares = [ExpertParallelMoE(6, 10, 3, 256, 128, rank=r, world_size=4) for r in range(4)]
+    assert [(m.first_expert, m.num_local) for m in shares] == [(0, 2), (2, 3), (5, 2), (7, 3)]
+    for m in shares:
+        p = m.problem
+        assert (p.T, p.E, p.num_global_experts, p.first_expert, p.topk) == (6, m.num_local, 10, m.first_expert, 3)
+        assert m.local_experts(w).shape[0] == m.num_local
+        assert m.local_experts(torch.arange(10))[0].item() == m.first_expert
+        assert m.problem_for(17).T == 17 and m.problem_for(17) is m.problem_for(17)
+    dp = ExpertParallelMoE(6, 10, 3, 256, 128, rank=1, world_size=4, data_parallel=True)
+    assert dp.problem.T == 24                             # the share runs on the gathered batch
+    with pytest.raises(ValueError):
+        shares[0].local_experts(torch.zeros((9, 4)))
+    with pytest.raises(ValueError):
+        ExpertParallelMoE(6, 10, 3, 256, 128, rank=1)     # rank without world_size
+    with pytest.raises(ValueError):
+        ExpertParallelMoE(6, 3, 1, 256, 128, rank=0, world_size=4)   # more ranks than experts
+    with pytest.raises(RuntimeError):
+        shares[1].forward(torch.zeros((6, 256), dtype=torch.bfloat16), None, None)   # no process group
