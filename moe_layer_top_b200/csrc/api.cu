@@ -437,6 +437,41 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
   return MOE_OK;
 }
 
+int combine_allreduce(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t rank, const moe_allreduce_rank* ranks,
+                      uint32_t epoch, uint32_t timeout_us, void* stream, bool emulated, bool scatter) {
+  if (world < 1 || world > MOE_MAX_RANKS) return fail(MOE_ERR_INVALID, "allreduce: world %d outside [1, %d]", world,
+                                                      MOE_MAX_RANKS);
+  if (!emulated && (rank < 0 || rank >= world)) return fail(MOE_ERR_INVALID, "allreduce: rank %d outside [0, %d)", rank,
+                                                            world);
+  if (T < 0 || topk < 1 || topk > 32 || H <= 0 || H % 128)
+    return fail(MOE_ERR_INVALID, "allreduce: T=%d topk=%d H=%d (H a positive multiple of 128)", T, topk, H);
+  if (static_cast<int64_t>(T) * topk * (scatter ? world : 1) >= (int64_t(1) << 31))
+    return fail(MOE_ERR_INVALID, "allreduce: rows * topk overflows int32");
+  if (epoch < 1 || epoch > 0x7FFFFFFFu) return fail(MOE_ERR_INVALID, "allreduce: epoch %u outside [1, 2^31)", epoch);
+  if (timeout_us < 1 || timeout_us > 10000000u)
+    return fail(MOE_ERR_INVALID, "allreduce: timeout_us %u outside [1, 10000000]", timeout_us);
+  if (T == 0) return MOE_OK;
+  if (!ranks) return fail(MOE_ERR_INVALID, "allreduce: ranks is NULL");
+  moe::AllreduceRank r[moe::kMaxRanks] = {};
+  for (int p = 0; p < world; ++p) {
+    const moe_allreduce_rank& q = ranks[p];
+    const bool own = emulated || p == rank;  // buffers this rank's kernel reads besides partial / out / flags
+    if (!q.partial || !q.out || !q.flags || (own && (!q.y || !q.status)))
+      return fail(MOE_ERR_INVALID, "allreduce: NULL buffer of rank %d", p);
+    if (!aligned(q.partial, 16) || !aligned(q.out, 16) || !aligned(q.flags, 4) || (own && !aligned(q.y, 16)) ||
+        (own && !aligned(q.pos_of_flat, 4)) || (own && !aligned(q.status, 4)))
+      return fail(MOE_ERR_INVALID, "allreduce: misaligned buffer of rank %d", p);
+    r[p] = moe::AllreduceRank{q.y, q.pos_of_flat, q.partial, q.out, q.flags, q.status};
+  }
+  int sms = 0;
+  int rc = device_check(&sms);
+  if (rc != MOE_OK) return rc;
+  cudaError_t e = moe::launch_combine_allreduce(r, world, emulated ? -1 : rank, T, topk, H, scatter, epoch,
+                                                1000ull * timeout_us, sms, static_cast<cudaStream_t>(stream));
+  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "allreduce");
+}
+
+
 }  // namespace
 
 namespace moe {
@@ -576,43 +611,6 @@ int32_t moe_combine_reduce_scatter_flag_count(int32_t T, int32_t world) {
   return 2 * moe::allreduce_chunks(T, world, true).nchunks + 1;
 }
 
-namespace {
-
-int combine_allreduce(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t rank, const moe_allreduce_rank* ranks,
-                      uint32_t epoch, uint32_t timeout_us, void* stream, bool emulated, bool scatter) {
-  if (world < 1 || world > MOE_MAX_RANKS) return fail(MOE_ERR_INVALID, "allreduce: world %d outside [1, %d]", world,
-                                                      MOE_MAX_RANKS);
-  if (!emulated && (rank < 0 || rank >= world)) return fail(MOE_ERR_INVALID, "allreduce: rank %d outside [0, %d)", rank,
-                                                            world);
-  if (T < 0 || topk < 1 || topk > 32 || H <= 0 || H % 128)
-    return fail(MOE_ERR_INVALID, "allreduce: T=%d topk=%d H=%d (H a positive multiple of 128)", T, topk, H);
-  if (static_cast<int64_t>(T) * topk * (scatter ? world : 1) >= (int64_t(1) << 31))
-    return fail(MOE_ERR_INVALID, "allreduce: rows * topk overflows int32");
-  if (epoch < 1 || epoch > 0x7FFFFFFFu) return fail(MOE_ERR_INVALID, "allreduce: epoch %u outside [1, 2^31)", epoch);
-  if (timeout_us < 1 || timeout_us > 10000000u)
-    return fail(MOE_ERR_INVALID, "allreduce: timeout_us %u outside [1, 10000000]", timeout_us);
-  if (T == 0) return MOE_OK;
-  if (!ranks) return fail(MOE_ERR_INVALID, "allreduce: ranks is NULL");
-  moe::AllreduceRank r[moe::kMaxRanks] = {};
-  for (int p = 0; p < world; ++p) {
-    const moe_allreduce_rank& q = ranks[p];
-    const bool own = emulated || p == rank;  // buffers this rank's kernel reads besides partial / out / flags
-    if (!q.partial || !q.out || !q.flags || (own && (!q.y || !q.status)))
-      return fail(MOE_ERR_INVALID, "allreduce: NULL buffer of rank %d", p);
-    if (!aligned(q.partial, 16) || !aligned(q.out, 16) || !aligned(q.flags, 4) || (own && !aligned(q.y, 16)) ||
-        (own && !aligned(q.pos_of_flat, 4)) || (own && !aligned(q.status, 4)))
-      return fail(MOE_ERR_INVALID, "allreduce: misaligned buffer of rank %d", p);
-    r[p] = moe::AllreduceRank{q.y, q.pos_of_flat, q.partial, q.out, q.flags, q.status};
-  }
-  int sms = 0;
-  int rc = device_check(&sms);
-  if (rc != MOE_OK) return rc;
-  cudaError_t e = moe::launch_combine_allreduce(r, world, emulated ? -1 : rank, T, topk, H, scatter, epoch,
-                                                1000ull * timeout_us, sms, static_cast<cudaStream_t>(stream));
-  return e == cudaSuccess ? MOE_OK : cuda_fail(e, "allreduce");
-}
-
-}  // namespace
 
 int moe_combine_allreduce(int32_t T, int32_t topk, int32_t H, int32_t world, int32_t rank,
                           const moe_allreduce_rank* ranks, uint32_t epoch, uint32_t timeout_us, void* stream) {
