@@ -247,7 +247,10 @@ MOE_API int moe_align(const int32_t* topk_ids, int32_t T, int32_t topk, int32_t 
  *    before anything is enqueued.
  *  - The first call on each device looks up the array's device address
  *    (cudaGetSymbolAddress, with that device current); make that first call
- *    before any stream capture.
+ *    before any stream capture.  The address is kept for the life of the
+ *    process: after cudaDeviceReset on a device, do not call this entry point
+ *    on that device again.  A failed lookup returns MOE_ERR_CUDA with the CUDA
+ *    error's name and text in moe_last_error_string().
  *  - All calls on a device share the array, and it keeps the previous
  *    call's contents; each call clears or rewrites every entry it reads.
  *    Calls whose executions overlap on the GPU (unordered streams) race.

@@ -13,9 +13,12 @@
 // The array is MOE_ALIGN_NOALLOC_SCRATCH_BYTES long and lives on every GPU
 // that loads the library until the process exits.  Its device address is
 // looked up once per device (cudaGetSymbolAddress, with that device current)
-// on the first call made on that device.  Every call on a device shares the
-// array: calls that overlap on the GPU (different streams without ordering)
-// race on it.
+// on the first call made on that device and cached for the life of the
+// process; after a cudaDeviceReset of that device the cached address is
+// stale, so the entry point must not be called on it again.  Every call on a
+// device shares the array: calls that overlap on the GPU (different streams
+// without ordering) race on it.
+#include <cstdio>
 #include <mutex>
 
 #include "kernels.h"
@@ -67,7 +70,12 @@ extern "C" MOE_API int moe_align_noalloc(const int32_t* topk_ids, int32_t T, int
                              "MOE_ALIGN_NOALLOC_SCRATCH_BYTES array holds; use moe_align with a workspace");
   void* scratch = nullptr;
   const cudaError_t e = scratch_address(&scratch);
-  if (e != cudaSuccess) return moe::record_error(MOE_ERR_CUDA, "align_noalloc: cudaGetSymbolAddress failed");
+  if (e != cudaSuccess) {
+    char msg[192];
+    snprintf(msg, sizeof msg, "align_noalloc: no device address for the static scratch (%s: %s)",
+             cudaGetErrorName(e), cudaGetErrorString(e));
+    return moe::record_error(MOE_ERR_CUDA, msg);
+  }
   // moe_align clears the status word it owns and writes every other scratch
   // entry it reads, so no stale contents of the previous call are used
   return moe_align(topk_ids, T, topk, E, block_m, sorted_token_ids, expert_ids, num_tokens_post_padded,

@@ -27,6 +27,24 @@ import torch.distributed as dist
 from . import ops
 
 
+NO_MULTICAST_ENV = "TORCH_SYMM_MEM_DISABLE_MULTICAST"
+
+
+def force_no_multicast() -> None:
+    """Make torch's symmetric memory bind no NVLink multicast object to its buffers.
+
+    The fused exchange reads and writes peers with plain loads and stores only, and a rank
+    that ends while its memory is bound to a multicast object can fault the other GPUs.  A
+    caller who set the switch to anything but "1" gets an error instead of a silent override
+    (torch may already have read the value)."""
+    v = os.environ.get(NO_MULTICAST_ENV)
+    if v is not None and v != "1":
+        raise RuntimeError(f"{NO_MULTICAST_ENV}={v!r}: the fused combine + all-reduce needs symmetric "
+                           f"buffers without multicast; unset it or set it to 1")
+    os.environ[NO_MULTICAST_ENV] = "1"
+    assert os.environ[NO_MULTICAST_ENV] == "1"
+
+
 def expert_shard(E: int, world_size: int, rank: int) -> tuple:
     """Experts ``(first, count)`` of ``rank``: ``[floor(rank*E/N), floor((rank+1)*E/N))``,
     contiguous, sizes differing by at most one."""
@@ -115,8 +133,7 @@ class ExpertParallelMoE:
         on first use for a T)."""
         if T in self._exchange:
             return self._exchange[T]
-        # the kernel uses plain peer loads and stores only: no multicast object is bound to these buffers
-        os.environ.setdefault("TORCH_SYMM_MEM_DISABLE_MULTICAST", "1")
+        force_no_multicast()
         import torch.distributed._symmetric_memory as symm_mem
         group = self.group if self.group is not None else dist.group.WORLD
         if not symm_mem.is_symm_mem_enabled_for_group(group.group_name):
@@ -124,6 +141,7 @@ class ExpertParallelMoE:
         H = self._shape[1]
         rows = T * self.world_size if self.data_parallel else T     # the batch the share runs on
         count = (ops.combine_reduce_scatter_flag_count if self.data_parallel else ops.combine_allreduce_flag_count)
+        assert os.environ.get(NO_MULTICAST_ENV) == "1", "symmetric buffers must not be multicast-bound"
         partial = symm_mem.empty((rows, H), dtype=torch.bfloat16, device=device)
         out = symm_mem.empty((T, H), dtype=torch.bfloat16, device=device)
         flags = symm_mem.empty((count(T, self.world_size),), dtype=torch.int32, device=device)

@@ -152,3 +152,17 @@ def test_share_construction_without_a_group():
         ExpertParallelMoE(6, 3, 1, 256, 128, rank=0, world_size=4)   # more ranks than experts
     with pytest.raises(RuntimeError):
         shares[1].forward(torch.zeros((6, 256), dtype=torch.bfloat16), None, None)   # no process group
+
+
+def test_multicast_switch_is_forced(monkeypatch):
+    """The fused exchange's symmetric buffers are never bound to a multicast object: the switch is
+    set to 1 when unset, and a caller's other value is an error, not silently kept."""
+    from moe_layer_top_b200.expert_parallel import NO_MULTICAST_ENV, force_no_multicast
+    monkeypatch.delenv(NO_MULTICAST_ENV, raising=False)
+    force_no_multicast()
+    assert os.environ[NO_MULTICAST_ENV] == "1"
+    force_no_multicast()                                  # idempotent
+    monkeypatch.setenv(NO_MULTICAST_ENV, "0")
+    with pytest.raises(RuntimeError):
+        force_no_multicast()
+    assert os.environ[NO_MULTICAST_ENV] == "0"

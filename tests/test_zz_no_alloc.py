@@ -2,8 +2,11 @@
 memory (its scratch is a static device array inside the library).
 
 Checked through the C ABI against moe_align (which takes a caller-provided
-workspace) on two calls in a row, the second smaller than the first so that
-stale contents of the shared array would show.  Alignment results are
+workspace) on four calls in a row, so that stale contents of the shared
+array would show: a large call on the three-pass path (count, scan, scatter
+over per-chunk histograms; more than 8192 assignments), a small one on the
+single-CTA path, then two more three-pass calls, each smaller than the first
+and with another expert count and block size.  Alignment results are
 integers, so the comparison is exact, as for moe_align against the oracle.
 
 This file is collected last on purpose: if it fails, every other test has
@@ -50,6 +53,8 @@ def test_noalloc_align_matches_workspace_align_on_consecutive_calls():
     cases = [
         (4096, 128, 8, 128, rng.integers(0, 128, (4096, 8))),                         # larger first
         (37, 256, 8, 16, np.minimum(rng.zipf(1.3, (37, 8)) - 1, 255)),                # then smaller, skewed
+        (1500, 256, 8, 64, np.minimum(rng.zipf(1.2, (1500, 8)) - 1, 255)),            # three-pass path again,
+        (1100, 64, 8, 128, rng.integers(0, 64, (1100, 8))),                           # smaller, other E and BM
     ]
     for T, E, k, bm, ids_np in cases:
         ids = torch.from_numpy(ids_np.astype(np.int32)).cuda()
