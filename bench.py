@@ -5,10 +5,17 @@
 One step = one pass of the whole layer (route -> align -> gather -> GEMM1
 (+SiLU*up) -> GEMM2 (+routed weight) -> combine) over one batch of seeded
 synthetic input resident in HBM, replayed from a CUDA graph of one
-moe_fused_forward call (the way a decode loop runs it).  Per-kernel times come
-from a second graph of the same stages with event nodes between them.  The default workload is the bf16
-Qwen3-235B-shaped decode layer (H=4096, E=128, top-8, I=1536); the headline
-batch is its largest sweep point (T=64) and every sweep point is reported.
+moe_fused_forward call (the way a serving loop runs it).  Per-kernel times
+come from a second graph of the same stages with event nodes between them.
+
+The default run's headline is the largest single-GPU configuration: the
+skewed-routing FP8 layer (H=7168, E=256, top-8, I=2048, 128x128 block
+scales, Zipf(1.2) expert choice), headline batch T=8192, every sweep point
+(T = 1, 32, 512, 8192) reported.  Two sub-records ride along, each with its
+own roofline and CPU baseline: the compute-bound FP8 prefill layer
+(H=4096, E=128, top-8, I=1536, T=16384) and the bf16 decode layer of the
+same shape (T = 1 ... 64).  ``--workload NAME`` times one workload alone.
+
 L2 is flushed (a 256 MiB write) before every timed step; the flush is outside
 the CUDA-event brackets.  Multi-GPU runs are independent replicas by default
 (each rank runs the same workload; the time is the max over ranks).  With
@@ -16,9 +23,9 @@ the CUDA-event brackets.  Multi-GPU runs are independent replicas by default
 experts, runs its share of the replicated batch and the output is all-reduced
 over NCCL; on one GPU ``--ep N`` times one rank's share alone.
 
-The ``--impl reference`` arm times the CPU oracle (the plain float64 numpy
-restatement of the layer) on the host cores, on bounded token samples of the
-same workload.
+The ``--impl reference`` arm times the CPU oracle (the plain C++
+double-precision restatement of the layer, OpenMP over rows) on the host
+cores, on bounded token samples of the same workload.
 """
 
 from __future__ import annotations
@@ -49,7 +56,10 @@ def parse_args():
     ap.add_argument("--gpus", type=int, default=1)
     ap.add_argument("--steps", type=int, default=20)
     ap.add_argument("--warmup", type=int, default=5)
-    ap.add_argument("--workload", default="decode_bf16", choices=sorted(inputs.CONFIGS))
+    ap.add_argument("--workload", default=None, choices=sorted(inputs.CONFIGS),
+                    help="one workload only (default: the largest single-GPU configuration, skewed_fp8, with the "
+                         "prefill_fp8 and decode_bf16 layers as sub-records)")
+    ap.add_argument("--no-sub-records", action="store_true", help="default workload without the sub-records")
     ap.add_argument("--tokens", type=int, default=0,
                     help="run only this batch size (default: the workload's sweep, headline = its largest)")
     ap.add_argument("--experts", type=int, default=0,
@@ -203,7 +213,7 @@ def traffic_record(kernel: str, workload: str, T: int):
 # ----------------------------------------------------------------------------- our arm
 def workload_config(args):
     import dataclasses
-    cfg = inputs.CONFIGS[args.workload]
+    cfg = inputs.CONFIGS[args.workload or DEFAULT_WORKLOAD]
     if args.experts:
         cfg = dataclasses.replace(cfg, name=f"{cfg.name}[E={args.experts}]", E=args.experts)
     return cfg
@@ -479,12 +489,25 @@ def e2e_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor):
     return float(np.sum(times)), h2d, d2h
 
 
-def cpu_baseline(cfg, T, seed, budget_s):
-    """The oracle, as it stands, timed on a bounded token sample of the workload.
+def _cpu_model() -> str:
+    try:
+        with open("/proc/cpuinfo") as f:
+            for line in f:
+                if line.startswith("model name"):
+                    return line.split(":", 1)[1].strip()
+    except OSError:
+        pass
+    return "unknown"
+
+
+def cpu_baseline(cfg, T, seed, budget_s, single_thread=True):
+    """The oracle, as it stands (C++, double precision), timed on bounded token
+    samples of the workload: with OpenMP over the rows on every host core
+    (``value``), and on one thread (``single_thread``).
 
     The generator's inputs for the sampled tokens (and the oracle's own FP8
-    block quantisation of the weights they touch) are prepared untimed; the
-    timed region is the oracle's forward on those tokens."""
+    quantisation of the weights they touch) are prepared untimed; the timed
+    region is the oracle's forward on those tokens."""
     from oracle import moe_oracle as O
     dev = "cuda" if torch.cuda.is_available() else "cpu"
     x = inputs.make_tokens(cfg, T, seed, device=dev).float().cpu().double().numpy()
@@ -497,13 +520,15 @@ def cpu_baseline(cfg, T, seed, budget_s):
         rkw = {"topk_ids": routing["topk_ids"], "topk_weights": routing["topk_weights"]}
     host = {}
 
+    def bits(w):
+        return w.contiguous().view(torch.int16).cpu().numpy().view(np.uint16)
+
     def prepare(tokens):
         for e in np.unique(ids_all[tokens]):
             e = int(e)
             if e not in host:
                 a, b = inputs.make_expert_weights(cfg, e, seed, device=dev)
-                a = a.float().cpu().double().numpy()
-                b = b.float().cpu().double().numpy()
+                a, b = bits(a), bits(b)
                 if cfg.mx:
                     host[e] = (*O.quantize_mx_group32(a), *O.quantize_mx_group32(b))
                 elif cfg.fp8:
@@ -518,59 +543,50 @@ def cpu_baseline(cfg, T, seed, budget_s):
         def __getitem__(self, e):
             return host[int(e)][self.i]
 
-    order = np.random.default_rng(seed).permutation(T)
-    done, t_spent, n = 0, 0.0, 1
-    while done < T and (done == 0 or t_spent < budget_s):
-        tok = order[done:done + n]
-        prepare(tok)
-        t0 = time.perf_counter()
-        if cfg.fp8:
-            O.moe_forward(x, View(0), View(2), cfg.topk, w13_scale=View(1), w2_scale=View(3), tokens=tok,
-                          mx=cfg.mx, **rkw)
-        else:
-            O.moe_forward(x, View(0), View(2), cfg.topk, tokens=tok, **rkw)
-        t_spent += time.perf_counter() - t0
-        done += len(tok)
-        n = min(2 * n, T - done) if done < T else n
-    try:
-        from threadpoolctl import threadpool_info
-        cores = max([int(i.get("num_threads", 1)) for i in threadpool_info()] or [1])
-    except Exception:  # noqa: BLE001
-        cores = 1
-    return {"value": done / t_spent, "unit": "tokens/s", "cores": cores, "kind": "oracle",
-            "sample": f"{done} of {T} tokens of {cfg.name} (T={T}); float64 numpy oracle forward, inputs "
-                      f"prepared untimed; {t_spent:.2f} s timed"}
+    def timed(threads, budget):
+        order = np.random.default_rng(seed).permutation(T)
+        done, t_spent, n = 0, 0.0, 1
+        while done < T and (done == 0 or t_spent < budget):
+            tok = order[done:done + n]
+            prepare(tok)
+            t0 = time.perf_counter()
+            if cfg.fp8:
+                O.moe_forward(x, View(0), View(2), cfg.topk, w13_scale=View(1), w2_scale=View(3), tokens=tok,
+                              mx=cfg.mx, threads=threads, **rkw)
+            else:
+                O.moe_forward(x, View(0), View(2), cfg.topk, tokens=tok, threads=threads, **rkw)
+            t_spent += time.perf_counter() - t0
+            done += len(tok)
+            n = min(2 * n, T - done) if done < T else n
+        return done, t_spent
+
+    cores = O.max_threads()
+    done, t_spent = timed(0, budget_s)
+    rec = {"value": round(done / t_spent, 3), "unit": "tokens/s", "cores": cores, "kind": "oracle",
+           "sample": f"{done} of {T} tokens of {cfg.name} (T={T}); C++ double-precision oracle forward, OpenMP "
+                     f"over rows on {cores} threads, inputs prepared untimed; {t_spent:.2f} s timed",
+           "cpu": _cpu_model()}
+    if single_thread:
+        d1, t1 = timed(1, budget_s / 2)
+        rec["single_thread"] = {"value": round(d1 / t1, 3), "unit": "tokens/s", "cores": 1,
+                                "sample": f"{d1} of {T} tokens, one thread; {t1:.2f} s timed"}
+    return rec
 
 
-def run_ours(args, rank, world, local):
-    from moe_layer_top_b200 import build, ops
-    build.build()
-    ops.lib()
-    cfg = workload_config(args)
-    T_head = args.tokens or max(cfg.tokens)
-    sweep_T = [T_head] if args.tokens else sorted(cfg.tokens)
-    peaks = measured_peaks()
-    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
-    ep = None
-    if args.ep:
-        # expert parallelism: on N ranks each runs its share and the output is
-        # all-reduced; on one GPU the step is one rank's share alone
-        from moe_layer_top_b200.expert_parallel import expert_shard
-        if world not in (1, args.ep):
-            raise SystemExit(f"--ep {args.ep} runs on {args.ep} ranks, or on one GPU (one share)")
-        ep_rank = rank if world > 1 else args.ep_rank
-        ep = (*expert_shard(cfg.E, args.ep, ep_rank), world > 1)
+def measure(cfg, args, world, flush, peaks, ep=None, T_only=0):
+    """Time one workload (its sweep, headline = the largest batch) and return its record."""
+    from moe_layer_top_b200 import ops
+    T_head = T_only or max(cfg.tokens)
+    sweep_T = [T_head] if T_only else sorted(cfg.tokens)
     weights = make_weights(cfg, args.seed, ep)
     results = {}
-    with ClockSampler(local) as clocks:
-        for T in sweep_T:
-            wl = Workload(cfg, T, args.seed, weights, args.persistent_decode, ep)
-            steps = args.steps if T == T_head else max(3, args.steps // 2)
-            step_ms, per_stage, wall, n_kernels = time_steps(wl, steps, args.warmup, flush, world)
-            total_ms = max_over_ranks(float(step_ms.sum()), world)
-            results[T] = {"wl": wl, "per_stage": per_stage, "total_ms": total_ms, "steps": steps, "wall_s": wall,
-                          "kernels": n_kernels}
-    clk = clocks.summary()
+    for T in sweep_T:
+        wl = Workload(cfg, T, args.seed, weights, args.persistent_decode, ep)
+        steps = args.steps if T == T_head else max(3, args.steps // 2)
+        step_ms, per_stage, wall, n_kernels = time_steps(wl, steps, args.warmup, flush, world)
+        total_ms = max_over_ranks(float(step_ms.sum()), world)
+        results[T] = {"wl": wl, "per_stage": per_stage, "total_ms": total_ms, "steps": steps, "wall_s": wall,
+                      "kernels": n_kernels}
     head = results[T_head]
     wl = head["wl"]
     alg = wl.algorithmic()
@@ -580,18 +596,19 @@ def run_ours(args, rank, world, local):
     value = layer_copies * T_head * K / (head["total_ms"] / 1e3)
     ms_per_step = head["total_ms"] / K
     stage_ms = head["per_stage"].mean(axis=0)
+    fp8_ratio = 2.0 if cfg.fp8 else 1.0
+    tc_peak = peaks["bf16_tflops"] * fp8_ratio
     # dominant kernel: the stage with the largest share of the step
     dom = int(np.argmax(stage_ms))
     dom_name = ops.STAGE_NAMES[dom]
     dom_bytes = {"gemm1": alg["gemm1_bytes"], "gemm2": alg["gemm2_bytes"]}.get(dom_name)
     if dom_bytes is None:
         dom_bytes = alg["layer_bytes"]
-    traffic = traffic_record(dom_name, args.workload, T_head) if ep is None else None
+    traffic = traffic_record(dom_name, cfg.name, T_head) if ep is None else None
     # FLOPs of the dominant GEMM (GEMM1 = 2/3 of the layer, GEMM2 = 1/3)
     dom_flops = alg["flops"] * {"gemm1": 2.0 / 3.0, "gemm2": 1.0 / 3.0}.get(dom_name, 1.0)
     # tensor-core peak for the arithmetic dtype: measured bf16 (burst: the kernel
     # is timed on its own inside a short step); FP8 = 2x that, the nominal ratio
-    tc_peak = peaks["bf16_tflops"] * (2.0 if cfg.fp8 else 1.0)
     tc_source = f"{peaks['source']} bf16 burst" + (" x 2 (nominal FP8/bf16 ratio)" if cfg.fp8 else "")
     if dom_flops / (tc_peak * 1e12) > dom_bytes / (peaks["hbm_gbs"] * 1e9):
         achieved = dom_flops / (stage_ms[dom] / 1e3) / 1e12
@@ -612,8 +629,7 @@ def run_ours(args, rank, world, local):
         sweep.append({"T": T, "tokens_per_s": round(layer_copies * T / (ms / 1e3), 1), "ms_per_step": round(ms, 4),
                       "layer_hbm_frac": round(a["layer_bytes"] / (ms / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
                       "tflops": round(a["flops"] / (ms / 1e3) / 1e12, 2),
-                      "layer_tc_frac": round(a["flops"] / (ms / 1e3) / 1e12 /
-                                             (peaks["bf16_tflops"] * (2.0 if cfg.fp8 else 1.0)), 4),
+                      "layer_tc_frac": round(a["flops"] / (ms / 1e3) / 1e12 / tc_peak, 4),
                       "hit_experts": a["hit_experts"],
                       "stage_us": {ops.STAGE_NAMES[s]: round(float(sm[s]) * 1e3, 1) for s in range(ops.NUM_STAGES)},
                       "mode": "swap_ab" if r["wl"].q.mode == ops.MODE_SWAP_AB else "normal",
@@ -632,11 +648,10 @@ def run_ours(args, rank, world, local):
         parallelism, scaling = (f"ep{args.ep} share of rank {args.ep_rank} (experts [{ep[0]}, {ep[0] + ep[1]})) "
                                 f"alone on one GPU: no all-reduce", "strong")
         wl_name = f"{cfg.name} (one EP={args.ep} share)"
-    line = {
-        "metric": "fused-MoE tokens/s; % HBM roofline (decode), % FP8/BF16 TC peak (prefill)",
-        "value": round(value, 1), "unit": "tokens/s", "n_gpus": world, "steps": K, "warmup": args.warmup,
-        "ms_per_step": round(ms_per_step, 4), "higher_is_better": True, "scaling": scaling, "vs_baseline": None,
-        "dtype": ("mxfp8_e4m3" if cfg.mx else "fp8_e4m3") if cfg.fp8 else "bf16", "data": "synthetic",
+    rec = {
+        "value": round(value, 1), "unit": "tokens/s", "steps": K, "ms_per_step": round(ms_per_step, 4),
+        "scaling": scaling,
+        "dtype": ("mxfp8_e4m3" if cfg.mx else "fp8_e4m3") if cfg.fp8 else "bf16",
         "config": {"workload": f"{wl_name}: H={cfg.H} E={cfg.E} topk={cfg.topk} I={cfg.I} T={T_head}",
                    "global_batch": layer_copies * T_head, "tokens_per_gpu": T_head, "parallelism": parallelism,
                    "weights": ("mxfp8 e4m3 + per-32 e8m0 scales" if cfg.mx else "fp8 e4m3 + 128x128 fp32 scales")
@@ -644,18 +659,67 @@ def run_ours(args, rank, world, local):
                    "routing": cfg.routing, "l2": "flushed (256 MiB write) before every step, outside the timing",
                    "launch": ("CUDA graph of moe_fused_forward (persistent decode kernel where eligible)"
                               if args.persistent_decode else "CUDA graph of moe_fused_forward (PDL between kernels)"),
-                   "layer_bytes_per_step": alg["layer_bytes"], "hit_experts": alg["hit_experts"]},
+                   "layer_bytes_per_step": alg["layer_bytes"], "layer_flops_per_step": alg["flops"],
+                   "hit_experts": alg["hit_experts"]},
         "roofline": roofline,
         "layer_hbm_frac": round(alg["layer_bytes"] / (ms_per_step / 1e3) / 1e9 / peaks["hbm_gbs"], 4),
+        "layer_tc_frac": round(alg["flops"] / (ms_per_step / 1e3) / 1e12 / tc_peak, 4),
         "stage_us": {ops.STAGE_NAMES[s]: round(float(stage_ms[s]) * 1e3, 1) for s in range(ops.NUM_STAGES)},
         "sweep": sweep,
         "e2e": e2e,
         "gpu_launches": K * (head["kernels"] or kernels_per_forward(cfg, T_head, "logits" in wl.routing)),
         "gpu_launches_source": "kernel nodes of the captured forward graph" if head["kernels"] else "formula",
-        "clocks": clk,
     }
-    if rank == 0 and world == 1 and not args.no_cpu_baseline and ep is None:
+    del results, wl, weights
+    torch.cuda.empty_cache()
+    return rec, T_head
+
+
+# the default run: the largest single-GPU configuration is the headline; the
+# compute-bound prefill layer and the bf16 decode layer ride along as sub-records
+DEFAULT_WORKLOAD = "skewed_fp8"
+DEFAULT_SUB_RECORDS = ("prefill_fp8", "decode_bf16")
+
+
+def run_ours(args, rank, world, local):
+    from moe_layer_top_b200 import build, ops
+    build.build()
+    ops.lib()
+    cfg = workload_config(args)
+    peaks = measured_peaks()
+    flush = torch.empty(L2_FLUSH_BYTES // 4, dtype=torch.float32, device="cuda")
+    ep = None
+    if args.ep:
+        # expert parallelism: on N ranks each runs its share and the output is
+        # all-reduced; on one GPU the step is one rank's share alone
+        from moe_layer_top_b200.expert_parallel import expert_shard
+        if world not in (1, args.ep):
+            raise SystemExit(f"--ep {args.ep} runs on {args.ep} ranks, or on one GPU (one share)")
+        ep_rank = rank if world > 1 else args.ep_rank
+        ep = (*expert_shard(cfg.E, args.ep, ep_rank), world > 1)
+    subs = []
+    if args.workload is None and not (args.tokens or args.experts or args.ep or args.no_sub_records):
+        subs = list(DEFAULT_SUB_RECORDS)
+    with ClockSampler(local) as clocks:
+        head, T_head = measure(cfg, args, world, flush, peaks, ep, args.tokens)
+        sub_recs = {name: measure(inputs.CONFIGS[name], args, world, flush, peaks) for name in subs}
+    clk = clocks.summary()
+    line = {"metric": "fused-MoE tokens/s; % HBM roofline (decode), % FP8/BF16 TC peak (prefill)",
+            "value": head["value"], "unit": "tokens/s", "n_gpus": world, "steps": head["steps"],
+            "warmup": args.warmup, "ms_per_step": head["ms_per_step"], "higher_is_better": True,
+            "scaling": head["scaling"], "vs_baseline": None, "dtype": head["dtype"], "data": "synthetic"}
+    line.update({k: v for k, v in head.items() if k not in line})
+    line["clocks"] = clk
+    cpu = rank == 0 and world == 1 and not args.no_cpu_baseline and ep is None
+    if cpu:
         line["cpu_baseline"] = cpu_baseline(cfg, T_head, args.seed, args.cpu_budget)
+    if sub_recs:
+        line["sub_records"] = {}
+        for name, (rec, T) in sub_recs.items():
+            if cpu:
+                rec["cpu_baseline"] = cpu_baseline(inputs.CONFIGS[name], T, args.seed, args.cpu_budget / 2,
+                                                   single_thread=False)
+            line["sub_records"][name] = rec
     return line
 
 
@@ -666,12 +730,12 @@ def run_reference(args, rank, world):
     if rank != 0:
         return None
     for _ in range(args.warmup):
-        cpu_baseline(cfg, T, args.seed, budget_s=0.0)
+        cpu_baseline(cfg, T, args.seed, budget_s=0.0, single_thread=False)
     vals = []
     base = None
     per_step_budget = max(1.0, args.cpu_budget / max(1, args.steps))
     for _ in range(args.steps):
-        base = cpu_baseline(cfg, T, args.seed, budget_s=per_step_budget)
+        base = cpu_baseline(cfg, T, args.seed, budget_s=per_step_budget, single_thread=False)
         vals.append(base["value"])
     value = float(np.mean(vals))
     base["value"] = round(value, 3)

@@ -17,8 +17,9 @@ TOL_MAX_REL = 0.05
 
 
 class LazyExperts:
-    """Per-expert host copies of the generator's bf16 weights, and the
-    oracle's own FP8 (block-128 or MX) quantisation of them, made on first access."""
+    """Per-expert host copies of the generator's bf16 weights (bit patterns),
+    and the oracle's own FP8 (block-128 or MX) quantisation of them, made on
+    first access."""
 
     def __init__(self, w_dev: torch.Tensor, fp8: bool, mx: bool = False):
         self.w_dev = w_dev
@@ -29,7 +30,7 @@ class LazyExperts:
     def _get(self, e):
         e = int(e)
         if e not in self._cache:
-            w = self.w_dev[e].float().cpu().double().numpy()
+            w = self.w_dev[e].view(torch.int16).cpu().numpy().view(np.uint16)     # bf16 bit patterns
             if self.mx:
                 self._cache[e] = O.quantize_mx_group32(w)
             else:
@@ -100,23 +101,34 @@ class Case:
     def status(self):
         return ops.read_status(self.p, self.ws)
 
+    def _oracle_inputs(self):
+        """Host copies of x and the routing input, and the oracle's lazily quantised experts
+        (made once per case)."""
+        if not hasattr(self, "_host"):
+            kw = {}
+            if "logits" in self.routing:
+                kw["logits"] = self.routing["logits"].cpu().numpy()
+            else:
+                kw["topk_ids"] = self.routing["topk_ids"].cpu().numpy()
+                kw["topk_weights"] = self.routing["topk_weights"].cpu().numpy()
+            kw["router_weight_on_input"] = self.router_weight_on_input
+            kw["renormalize"] = self.renormalize
+            kw["swiglu_limit"] = self.swiglu_limit if self.swiglu_limit > 0 else None
+            l13 = LazyExperts(self.w13_bf16, self.cfg.fp8, self.cfg.mx)
+            l2 = LazyExperts(self.w2_bf16, self.cfg.fp8, self.cfg.mx)
+            if self.cfg.fp8:
+                kw.update(w13_scale=l13.scales, w2_scale=l2.scales, mx=self.cfg.mx)
+            self._host = (self.x.float().cpu().double().numpy(), l13.codes, l2.codes, kw)
+        return self._host
+
     def oracle(self, tokens=None, return_y=False):
-        x = self.x.float().cpu().double().numpy()
-        kw = {}
-        if "logits" in self.routing:
-            kw["logits"] = self.routing["logits"].cpu().numpy()
-        else:
-            kw["topk_ids"] = self.routing["topk_ids"].cpu().numpy()
-            kw["topk_weights"] = self.routing["topk_weights"].cpu().numpy()
-        kw["router_weight_on_input"] = self.router_weight_on_input
-        kw["renormalize"] = self.renormalize
-        kw["swiglu_limit"] = self.swiglu_limit if self.swiglu_limit > 0 else None
-        l13 = LazyExperts(self.w13_bf16, self.cfg.fp8, self.cfg.mx)
-        l2 = LazyExperts(self.w2_bf16, self.cfg.fp8, self.cfg.mx)
-        if self.cfg.fp8:
-            return O.moe_forward(x, l13.codes, l2.codes, self.cfg.topk, w13_scale=l13.scales, w2_scale=l2.scales,
-                                 tokens=tokens, return_y=return_y, mx=self.cfg.mx, **kw)
-        return O.moe_forward(x, l13.codes, l2.codes, self.cfg.topk, tokens=tokens, return_y=return_y, **kw)
+        x, w13, w2, kw = self._oracle_inputs()
+        return O.moe_forward(x, w13, w2, self.cfg.topk, tokens=tokens, return_y=return_y, **kw)
+
+    def oracle_assignments(self, flat):
+        """The oracle's unweighted expert outputs of the flat assignments t * topk + j."""
+        x, w13, w2, kw = self._oracle_inputs()
+        return O.assignment_outputs(x, w13, w2, self.cfg.topk, flat, **kw)
 
 
 def errors(got, ref):

@@ -184,6 +184,43 @@ def test_gather_quantises_x_bit_exact(mode, bm):
     np.testing.assert_array_equal(v["a1_scale_t"][:, :ntpp].cpu().numpy().T[rows], rs[tok])
 
 
+@pytest.mark.parametrize("mode,bm", [(ops.MODE_NORMAL, 128), (ops.MODE_SWAP_AB, 32)])
+def test_fp8_gemm1_intermediate_matches_oracle(mode, bm):
+    """The block-FP8 GEMM1 output a2 (E4M3 codes + per-(row,128) power-of-two scales) of every
+    real row against the oracle's requantisation of its own bf16 intermediate, for both GEMM1
+    epilogues.  The fast exponential of the SiLU and the fp32 accumulation order may move a bf16
+    value by one ulp, so codes are compared by value within one E4M3 step, and nearly all codes
+    and scales must be equal."""
+    c = Case(MID_FP8, 45, seed=8, mode=mode, block_m=bm, split_k=False)
+    c.run()
+    v = c.views()
+    k = MID_FP8.topk
+    ntpp = int(v["num_tokens_post_padded"].item())
+    sorted_ids = v["sorted_token_ids"][:ntpp].cpu().numpy()
+    expert_of_row = np.repeat(v["expert_ids"].cpu().numpy()[:ntpp // bm], bm)
+    rows = np.nonzero(sorted_ids < 45 * k)[0]
+    x = c.x.float().cpu().double().numpy()
+    a2 = v["a2"][:ntpp].cpu().numpy()
+    a2_s = v["a2_scale_t"][:, :ntpp].cpu().numpy().T
+    got_vals, ref_vals, same_codes, same_scales = [], [], 0, 0
+    for e in np.unique(expert_of_row[rows]):
+        rr = rows[expert_of_row[rows] == e]
+        xq, xs = O.quantize_act_group128(x[sorted_ids[rr] // k])
+        w13c, w13s = O.quantize_weight_block128(c.w13_bf16[e].float().cpu().double().numpy())
+        w2c, w2s = O.quantize_weight_block128(c.w2_bf16[e].float().cpu().double().numpy())
+        _, inter = O.expert_mlp(O.dequantize_act_group128(xq, xs), O.dequantize_weight_block128(w13c, w13s),
+                                O.dequantize_weight_block128(w2c, w2s), requant=True, return_intermediates=True)
+        got_vals.append(O.dequantize_act_group128(a2[rr], a2_s[rr]))
+        ref_vals.append(O.dequantize_act_group128(inter["a2_codes"], inter["a2_scales"]))
+        same_codes += int((a2[rr] == inter["a2_codes"]).sum())
+        same_scales += int((a2_s[rr] == inter["a2_scales"]).sum())
+    got, ref = np.concatenate(got_vals), np.concatenate(ref_vals)
+    assert same_codes >= 0.99 * got.size
+    assert same_scales >= 0.99 * (got.size // 128)
+    step = np.abs(ref) * 2.0 ** -3 + 1e-30
+    assert np.all(np.abs(got - ref) <= np.maximum(step, 2.0 ** -9 * np.abs(ref).max()))
+
+
 # ----------------------------------------------------------------------------- layer output
 @pytest.mark.parametrize("mode,bm", [(ops.MODE_AUTO, 0)] + MODES)
 def test_tiny_layer_all_modes(mode, bm):
@@ -228,21 +265,6 @@ def test_decode_bf16_full_size(T):
 def _sample(T, n, seed):
     rng = np.random.default_rng(seed)
     return np.unique(np.concatenate([[0, T - 1], rng.choice(T, size=min(n, T), replace=False)]))
-
-
-@pytest.mark.parametrize("name,T,n", [("fp8_uniform", 256, 6), ("fp8_uniform", 1024, 4), ("prefill_fp8", 16384, 4),
-                                      ("skewed_fp8", 1, 1), ("skewed_fp8", 32, 4), ("skewed_fp8", 512, 3)])
-def test_fp8_full_size_sampled(name, T, n):
-    cfg = inputs.CONFIGS[name]
-    c = Case(cfg, T, seed=0)
-    out = c.run()
-    assert c.status() == ops.MOE_STATUS_OK
-    tok = _sample(T, n, T)
-    ref = c.oracle(tokens=tok)
-    assert_close(out[torch.from_numpy(tok).cuda()].float().cpu().numpy(), ref["out"], fp8=True)
-    if "logits" in c.routing:   # the routing of every token is checked in full
-        ids, _ = O.route(c.routing["logits"].cpu().numpy(), cfg.topk)
-        np.testing.assert_array_equal(c.views()["topk_ids"].cpu().numpy(), ids)
 
 
 # ----------------------------------------------------------------------------- properties

@@ -199,3 +199,16 @@ def test_page_constants_fixture():
     v[0, 5] = 1e-20
     _, sc = O.quantize_act_group128(v)
     assert sc[0, 0] == O.pow2_ceil(np.float32(np.float32(gold["amax_floor"]) * np.float32(1 / 448.0)))
+
+
+def test_quantisers_read_bf16_bit_patterns_as_their_values():
+    """The weight quantisers take bf16 weights either as values or as raw bit patterns (what a
+    host copy of a bf16 tensor holds); both give the same codes and scales."""
+    w = torch.randn(256, 384, generator=torch.Generator().manual_seed(8)).to(torch.bfloat16) * 0.02
+    bits = w.view(torch.int16).numpy().view(np.uint16)
+    vals = w.double().numpy()
+    for quant in (O.quantize_weight_block128, O.quantize_mx_group32):
+        a, sa = quant(bits)
+        b, sb = quant(vals)
+        np.testing.assert_array_equal(a, b)
+        np.testing.assert_array_equal(sa, sb)

@@ -259,3 +259,56 @@ def test_forward_zero_weights_give_zero_and_linearity_in_w2():
     np.testing.assert_array_equal(b["y"], 2.0 * a["y"])         # y is linear in w2 (exact in fp64 x2)
     z = O.moe_forward(x, w13n, 0.0 * w2n, 2, logits=logits)
     assert np.all(z["out"] == 0.0)
+
+
+def test_assignment_outputs_match_dense_per_expert_outputs():
+    """One expert's outputs for chosen assignments (used to check every row of an expert on the
+    GPU without evaluating the token's other experts) = the dense torch evaluation's unweighted
+    output of that expert on that token; FP8 path with duplicate ids."""
+    cfg = inputs.make_custom_config("tiny_fp8", E=6, topk=3, H=256, I=256, fp8=True,
+                                    routing="uniform_ids", tokens=(12,))
+    w13, w2 = inputs.make_weights(cfg, 9)
+    xn = inputs.make_tokens(cfg, 12, 9).double().numpy()
+    r = inputs.make_routing(cfg, 12, 9)
+    ids = r["topk_ids"].numpy().copy()
+    ids[3] = [1, 1, 4]
+    wts = r["topk_weights"].numpy()
+    q13, s13 = O.quantize_weight_block128(w13.double().numpy())
+    q2, s2 = O.quantize_weight_block128(w2.double().numpy())
+    flat = np.array([3 * 3 + 1, 0, 35, 3 * 3 + 0, 17])          # any order, duplicates' slots included
+    got = O.assignment_outputs(xn, q13, q2, 3, flat, topk_ids=ids, topk_weights=wts, w13_scale=s13, w2_scale=s2)
+    # dense torch: every expert on every token, unweighted
+    g = torch.from_numpy(xn).reshape(12, 2, 128).float()
+    raw = torch.clamp(g.abs().amax(-1), min=1e-10) * torch.tensor(1 / 448.0)
+    sc = torch.exp2(torch.ceil(torch.log2(raw.double())))
+    xt = ((g.double() / sc[..., None]).float().to(torch.float8_e4m3fn).double() * sc[..., None]).reshape(12, 256)
+    deq = lambda c, s: torch.from_numpy(c).view(torch.float8_e4m3fn).double() * \
+        torch.from_numpy(s).double().repeat_interleave(128, -2).repeat_interleave(128, -1)
+    h = torch.einsum("th,enh->etn", xt, deq(q13, s13)).to(torch.bfloat16).double()
+    p = (F.silu(h[..., :256]).to(torch.bfloat16).double() * h[..., 256:]).to(torch.bfloat16).double()
+    pg = p.reshape(6, 12, 2, 128).float()
+    raw = torch.clamp(pg.abs().amax(-1), min=1e-10) * torch.tensor(1 / 448.0)
+    sc = torch.exp2(torch.ceil(torch.log2(raw.double())))
+    p = ((pg.double() / sc[..., None]).float().to(torch.float8_e4m3fn).double() * sc[..., None]).reshape(6, 12, 256)
+    y = torch.einsum("eti,ehi->eth", p, deq(q2, s2)).numpy()
+    ref = np.stack([y[ids.reshape(-1)[f], f // 3] for f in flat])
+    np.testing.assert_allclose(got, ref, rtol=1e-12, atol=1e-15)
+    # and it is the same y the layer evaluation uses
+    full = O.moe_forward(xn, q13, q2, 3, topk_ids=ids, topk_weights=wts, w13_scale=s13, w2_scale=s2, return_y=True)
+    np.testing.assert_array_equal(got, full["y"].reshape(36, 256)[flat])
+
+
+def test_parallel_rows_do_not_change_results_and_bf16_bit_patterns():
+    """The oracle's OpenMP loops run independent rows: one thread and all threads give the same
+    bits.  bf16 weights given as bit patterns (uint16) read as the same values as float64."""
+    cfg = inputs.CONFIGS["tiny"]
+    w13, w2 = inputs.make_weights(cfg, 11)
+    x = inputs.make_tokens(cfg, 16, 11).double().numpy()
+    logits = inputs.make_routing(cfg, 16, 11)["logits"].numpy()
+    a = O.moe_forward(x, w13.double().numpy(), w2.double().numpy(), 2, logits=logits, threads=1)
+    b = O.moe_forward(x, w13.double().numpy(), w2.double().numpy(), 2, logits=logits, threads=0)
+    np.testing.assert_array_equal(a["out"], b["out"])
+    bits13 = w13.view(torch.int16).numpy().view(np.uint16)
+    bits2 = w2.view(torch.int16).numpy().view(np.uint16)
+    c = O.moe_forward(x, bits13, bits2, 2, logits=logits)
+    np.testing.assert_array_equal(a["out"], c["out"])
