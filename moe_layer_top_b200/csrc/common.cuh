@@ -366,6 +366,13 @@ __device__ __forceinline__ void tmem_ld8(uint32_t taddr, float (&v)[8]) {
   for (int i = 0; i < 8; ++i) v[i] = __uint_as_float(r[i]);
 }
 
+__device__ __forceinline__ void tmem_ld8u(uint32_t taddr, uint32_t (&r)[8]) {
+  asm volatile(
+      "tcgen05.ld.sync.aligned.32x32b.x8.b32 {%0, %1, %2, %3, %4, %5, %6, %7}, [%8];"
+      : "=r"(r[0]), "=r"(r[1]), "=r"(r[2]), "=r"(r[3]), "=r"(r[4]), "=r"(r[5]), "=r"(r[6]), "=r"(r[7])
+      : "r"(taddr));
+}
+
 // 32 lanes x 32 consecutive 32-bit columns (raw bits)
 __device__ __forceinline__ void tmem_ld32(uint32_t taddr, uint32_t (&r)[32]) {
   asm volatile(
@@ -403,6 +410,18 @@ __device__ __forceinline__ void ffma2(uint32_t& a0, uint32_t& a1, uint32_t d0, u
       "mov.b64 {%0, %1}, ra;\n\t}"
       : "+r"(a0), "+r"(a1)
       : "r"(d0), "r"(d1), "r"(__float_as_uint(f)));
+}
+
+// float accumulators: (a0, a1) <- (d0, d1) * (f, f) + (a0, a1), d as raw fp32 words
+__device__ __forceinline__ void ffma2f(float& a0, float& a1, uint32_t d0, uint32_t d1, float f) {
+  asm("{\n\t.reg .b64 ra, rd, rf;\n\t"
+      "mov.b64 ra, {%0, %1};\n\t"
+      "mov.b64 rd, {%2, %3};\n\t"
+      "mov.b64 rf, {%4, %4};\n\t"
+      "fma.rn.f32x2 ra, rd, rf, ra;\n\t"
+      "mov.b64 {%0, %1}, ra;\n\t}"
+      : "+f"(a0), "+f"(a1)
+      : "r"(d0), "r"(d1), "f"(f));
 }
 
 // (a0, a1) <- (d0, d1) * (f, f)

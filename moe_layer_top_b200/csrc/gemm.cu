@@ -72,13 +72,20 @@ struct Cfg {
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kMmaN = kSwap ? kBM : 256;
   static constexpr int kAccCols = kSwap ? (kDown ? kBM : 2 * kBM) : 256;
-  static constexpr int kTmemCols = ceil_pow2((2 * kAccCols) < 32 ? 32 : 2 * kAccCols);
+  // TMEM accumulator buffers.  bf16: two (the whole K range of a tile accumulates in one; the
+  // next tile's MMAs use the other).  FP8: one per 128-deep K block; swap-AB accumulators are
+  // narrow, so up to eight let the MMA run that many K blocks ahead of the epilogue's
+  // promotion (a normal tile's 256 columns leave room for two).
+  static constexpr int kAccBufs = kFP8 ? ((512 / kAccCols) > 8 ? 8 : (512 / kAccCols)) : 2;
+  static constexpr int kTmemCols = ceil_pow2((kAccBufs * kAccCols) < 32 ? 32 : kAccBufs * kAccCols);
   // output columns per tile: GEMM1 -> 128 intermediate columns; GEMM2 -> H columns
   static constexpr int kTileN = kDown ? (kSwap ? 128 : 256) : 128;
   static constexpr int kHalfTok = kBM / 2;  // swap: token columns per epilogue group
   static constexpr size_t kSmemBytes = static_cast<size_t>(kStages) * kStageBytes + kSmemReserve + 1024;
   static_assert(kStages >= 2, "pipeline needs at least two stages");
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
+  static_assert(kAccBufs >= 2, "accumulators are at least double-buffered");
+  static_assert((2 * kStages + 2 * kAccBufs + 3) * 8 + 8 <= kXchgOffset, "barriers overlap the exchange buffers");
   static_assert(!kSwap || kBM == 16 || kBM == 32 || kBM == 64, "swap-AB block_m");
 };
 
@@ -155,8 +162,8 @@ __global__ void __launch_bounds__(kThreads, 1)
   uint64_t* full = reinterpret_cast<uint64_t*>(reserve);
   uint64_t* empty = full + C::kStages;
   uint64_t* acc_full = empty + C::kStages;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* xchg_bar = acc_empty + 2;
+  uint64_t* acc_empty = acc_full + C::kAccBufs;
+  uint64_t* xchg_bar = acc_empty + C::kAccBufs;
   uint64_t* drain = xchg_bar + 2;
   uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
   volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
@@ -169,11 +176,11 @@ __global__ void __launch_bounds__(kThreads, 1)
       mbar_init(&full[s], 1);
       mbar_init(&empty[s], 1);
     }
-    for (int b = 0; b < 2; ++b) {
+    for (int b = 0; b < C::kAccBufs; ++b) {
       mbar_init(&acc_full[b], 1);
       mbar_init(&acc_empty[b], kEpiWarps);
-      mbar_init(&xchg_bar[b], kEpiWarps * 32);
     }
+    for (int b = 0; b < 2; ++b) mbar_init(&xchg_bar[b], kEpiWarps * 32);
     mbar_init(drain, 1);
     *abort_flag = 0;
     fence_mbar_init();
@@ -426,8 +433,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           mma_commit(&empty[stage]);
           if constexpr (kFP8) {
             mma_commit(&acc_full[abuf]);
-            abuf ^= 1;
-            if (abuf == 0) aphase ^= 1u;
+            if (++abuf == C::kAccBufs) {
+              abuf = 0;
+              aphase ^= 1u;
+            }
           }
           if (++stage == C::kStages) {
             stage = 0;
@@ -437,8 +446,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         if (!ok) break;
         if constexpr (!kFP8) {
           mma_commit(&acc_full[abuf]);
-          abuf ^= 1;
-          if (abuf == 0) aphase ^= 1u;
+          if (++abuf == C::kAccBufs) {
+            abuf = 0;
+            aphase ^= 1u;
+          }
         }
       }
       // every MMA this thread issued has completed once `drain` flips
@@ -506,34 +517,44 @@ __global__ void __launch_bounds__(kThreads, 1)
             }
             tc_fence_after();
             const uint32_t t0 = tmem_base + lane_addr + static_cast<uint32_t>(abuf * C::kAccCols);
-            if constexpr (kDown) {
-#pragma unroll
-              for (int c = 0; c < kCols / 16; ++c) {
-                float d[16];
-                tmem_ld16(t0 + g * 128 + 16 * c, d);
-                tmem_wait_ld();
-#pragma unroll
-                for (int i = 0; i < 16; ++i) acc_a[16 * c + i] = fmaf(d[i], fa, acc_a[16 * c + i]);
+            // Promotion, software-pipelined: chunk c+1 is loaded from TMEM while chunk c is
+            // scaled into the fp32 accumulators (two lanes per instruction), and the buffer is
+            // handed back to the MMA as soon as its last chunk has landed in registers.
+            // (tcgen05.wait::ld waits for every load issued so far, so each wait comes before
+            // the next chunk's load is issued.)
+            constexpr int kChunks = kDown ? kCols / 16 : kCols / 8;
+            constexpr int kW = kDown ? 16 : 8;                   // words per chunk (per gate/up half)
+            uint32_t ba[2][kW], bb[2][kDown ? 1 : kW];
+            auto load = [&](int c) {
+              if constexpr (kDown) {
+                tmem_ld16u(t0 + g * 128 + 16 * c, ba[c & 1]);
+              } else {
+                tmem_ld8u(t0 + g * 64 + 8 * c, ba[c & 1]);
+                tmem_ld8u(t0 + 128 + g * 64 + 8 * c, bb[c & 1]);
               }
-            } else {
+            };
+            load(0);
 #pragma unroll
-              for (int c = 0; c < kCols / 16; ++c) {
-                float dg[16], du[16];
-                tmem_ld16(t0 + g * 64 + 16 * c, dg);
-                tmem_ld16(t0 + 128 + g * 64 + 16 * c, du);
-                tmem_wait_ld();
+            for (int c = 0; c < kChunks; ++c) {
+              tmem_wait_ld();                                    // chunk c is in registers
+              if (c + 1 < kChunks) {
+                load(c + 1);                                     // in flight while chunk c is scaled
+              } else {
+                tc_fence_before();
+                __syncwarp();
+                if (lane == 0) mbar_arrive(&acc_empty[abuf]);    // the MMA may reuse the buffer
+              }
 #pragma unroll
-                for (int i = 0; i < 16; ++i) {
-                  acc_a[16 * c + i] = fmaf(dg[i], fa, acc_a[16 * c + i]);
-                  acc_b[16 * c + i] = fmaf(du[i], fb, acc_b[16 * c + i]);
-                }
+              for (int i = 0; i < kW; i += 2) {
+                ffma2f(acc_a[kW * c + i], acc_a[kW * c + i + 1], ba[c & 1][i], ba[c & 1][i + 1], fa);
+                if constexpr (!kDown)
+                  ffma2f(acc_b[kW * c + i], acc_b[kW * c + i + 1], bb[c & 1][i], bb[c & 1][i + 1], fb);
               }
             }
-            tc_fence_before();
-            __syncwarp();
-            if (lane == 0) mbar_arrive(&acc_empty[abuf]);
-            abuf ^= 1;
-            if (abuf == 0) aphase ^= 1u;
+            if (++abuf == C::kAccBufs) {
+              abuf = 0;
+              aphase ^= 1u;
+            }
           }
           if (!ok) break;
         }
@@ -568,8 +589,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[abuf]);
-            abuf ^= 1;
-            if (abuf == 0) aphase ^= 1u;
+            if (++abuf == C::kAccBufs) {
+              abuf = 0;
+              aphase ^= 1u;
+            }
             uint4* dst = reinterpret_cast<uint4*>(a2 + static_cast<size_t>(grow) * I + col0);
 #pragma unroll
             for (int i = 0; i < 8; ++i)
@@ -648,8 +671,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[abuf]);
-            abuf ^= 1;
-            if (abuf == 0) aphase ^= 1u;
+            if (++abuf == C::kAccBufs) {
+              abuf = 0;
+              aphase ^= 1u;
+            }
             if (real) {
               uint4* dst = reinterpret_cast<uint4*>(yrow);
 #pragma unroll
@@ -664,6 +689,16 @@ __global__ void __launch_bounds__(kThreads, 1)
         const int tok0 = mb * kBM + g * kHT;       // first sorted row of this group
         float acc_a[kHT];                          // gate (GEMM1) or down (GEMM2)
         float acc_b[kDown ? 1 : kHT];              // up (GEMM1)
+        // GEMM2: the tokens' flat ids and routed weights, read before the K loop so that
+        // their latency is not on the tile's tail
+        int flat_j[kDown ? kHT : 1];
+        float wt_j[kDown ? kHT : 1];
+        if constexpr (kDown) {
+#pragma unroll
+          for (int j = 0; j < kHT; ++j) flat_j[j] = (*(args.sorted_ids + tok0 + j));
+#pragma unroll
+          for (int j = 0; j < kHT; ++j) wt_j[j] = flat_j[j] < args.nflat ? route_weight(args.topk_weights, flat_j[j]) : 0.f;
+        }
         // column offsets of this group's values inside one accumulator buffer
         const uint32_t col_a = static_cast<uint32_t>(g * kHT);
         const uint32_t col_b = static_cast<uint32_t>(kBM + g * kHT);
@@ -712,8 +747,10 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[abuf]);
-            abuf ^= 1;
-            if (abuf == 0) aphase ^= 1u;
+            if (++abuf == C::kAccBufs) {
+              abuf = 0;
+              aphase ^= 1u;
+            }
           }
           if (!ok) break;
         } else {
@@ -738,8 +775,10 @@ __global__ void __launch_bounds__(kThreads, 1)
           tc_fence_before();
           __syncwarp();
           if (lane == 0) mbar_arrive(&acc_empty[abuf]);
-          abuf ^= 1;
-          if (abuf == 0) aphase ^= 1u;
+          if (++abuf == C::kAccBufs) {
+            abuf = 0;
+            aphase ^= 1u;
+          }
         }
 
         if (splits > 1) {
@@ -802,11 +841,8 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int hcol = nt * 128 + row;
 #pragma unroll
           for (int j = 0; j < kHT; ++j) {
-            const int flat = (*(args.sorted_ids + tok0 + j));
-            if (flat < args.nflat) {
-              const float wt = route_weight(args.topk_weights, flat);
-              y[static_cast<size_t>(flat) * H + hcol] = __float2bfloat16_rn(acc_a[j] * wt);
-            }
+            if (flat_j[j] < args.nflat)
+              y[static_cast<size_t>(flat_j[j]) * H + hcol] = __float2bfloat16_rn(acc_a[j] * wt_j[j]);
           }
         }
       }

@@ -317,12 +317,13 @@ __global__ void __launch_bounds__(1024) route_align_small_kernel(
   } else {
     for (int i = tid; i < n; i += 1024) ids_s[i] = (*(ids_in + i));
   }
-  for (int i = tid; i < 32 * E; i += 1024) hist[i] = 0;
-  __syncthreads();
-
   const int chunk = (n + 32 * 32 - 1) / (32 * 32) * 32;  // multiple of 32
+  const int nw = (n + chunk - 1) / chunk;                 // warps that own assignments
   const int begin = warp * chunk;
   const int end = min(begin + chunk, n);
+  for (int i = tid; i < nw * E; i += 1024) hist[i] = 0;
+  __syncthreads();
+
   for (int i = begin + lane; i < end; i += 32) {
     const int g = ids_s[i];
     const int e = g - er.first;
@@ -334,7 +335,7 @@ __global__ void __launch_bounds__(1024) route_align_small_kernel(
   __syncthreads();
   for (int e = tid; e < E; e += 1024) {
     int32_t run = 0;
-    for (int w = 0; w < 32; ++w) {
+    for (int w = 0; w < nw; ++w) {
       const int32_t v = hist[w * E + e];
       hist[w * E + e] = run;
       run += v;

@@ -12,31 +12,41 @@ namespace moe {
 // ----------------------------------------------------------------------------
 // router
 // ----------------------------------------------------------------------------
+// Order-preserving 32-bit key of a finite float (larger float -> larger key;
+// -0 is folded onto +0 first so that equal logits get equal keys); 0 is below
+// every key and marks "taken / no expert".
+__device__ __forceinline__ uint32_t logit_key(float v) {
+  const uint32_t u = __float_as_uint(v + 0.0f);
+  return (u & 0x80000000u) ? ~u : (u | 0x80000000u);
+}
+__device__ __forceinline__ float key_logit(uint32_t k) {
+  return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
+}
+
 // One warp routes one token: lane r (< topk) returns the r-th chosen expert
-// and its weight.
+// and its weight.  Each selection round is two warp reductions (redux.sync):
+// the largest key, then the lowest expert index holding it -- descending
+// logit, the lower index on ties.
 template <int VPL>  // logits per lane (E <= 32 * VPL)
 __device__ __forceinline__ void route_token(const float* row, int E, int topk, int renormalize,
                                             int lane, int& out_id, float& out_w) {
-
   float v[VPL];
-  uint32_t taken = 0;
+  uint32_t key[VPL];
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = lane + 32 * i;
     v[i] = (e < E) ? (*(row + e)) : -INFINITY;
-    if (e >= E) taken |= 1u << i;
+    key[i] = (e < E) ? logit_key(v[i]) : 0u;
   }
   // softmax statistics over all experts
-  float m = -INFINITY;
+  uint32_t kmax = 0;
 #pragma unroll
-  for (int i = 0; i < VPL; ++i)
-    if (!((taken >> i) & 1u)) m = fmaxf(m, v[i]);
-#pragma unroll
-  for (int off = 16; off > 0; off >>= 1) m = fmaxf(m, __shfl_xor_sync(0xffffffffu, m, off));
+  for (int i = 0; i < VPL; ++i) kmax = max(kmax, key[i]);
+  const float m = key_logit(__reduce_max_sync(0xffffffffu, kmax));
   float z = 0.f;
 #pragma unroll
   for (int i = 0; i < VPL; ++i)
-    if (!((taken >> i) & 1u)) z += expf(v[i] - m);
+    if (lane + 32 * i < E) z += expf(v[i] - m);
 #pragma unroll
   for (int off = 16; off > 0; off >>= 1) z += __shfl_xor_sync(0xffffffffu, z, off);
 
@@ -44,29 +54,25 @@ __device__ __forceinline__ void route_token(const float* row, int E, int topk, i
   float my_logit = 0.f;
   int my_id = -1;
   for (int r = 0; r < topk; ++r) {
-    float best = -INFINITY;
-    int bi = INT_MAX;
+    uint32_t best = 0;
+    int bi = 0;
 #pragma unroll
-    for (int i = 0; i < VPL; ++i) {
-      if ((taken >> i) & 1u) continue;
-      if (bi == INT_MAX || v[i] > best) {  // ascending index inside a lane: strict > keeps the lower one
-        best = v[i];
-        bi = lane + 32 * i;
+    for (int i = 0; i < VPL; ++i)
+      if (key[i] > best) {  // ascending index inside a lane: strict > keeps the lower one
+        best = key[i];
+        bi = i;
       }
-    }
+    const uint32_t wbest = __reduce_max_sync(0xffffffffu, best);
+    const uint32_t cand = (best == wbest) ? static_cast<uint32_t>(lane + 32 * bi) : 0xffffffffu;
+    const int widx = static_cast<int>(__reduce_min_sync(0xffffffffu, cand));
+    if ((widx & 31) == lane) {
 #pragma unroll
-    for (int off = 16; off > 0; off >>= 1) {
-      const float ob = __shfl_xor_sync(0xffffffffu, best, off);
-      const int oi = __shfl_xor_sync(0xffffffffu, bi, off);
-      if (oi != INT_MAX && (bi == INT_MAX || ob > best || (ob == best && oi < bi))) {
-        best = ob;
-        bi = oi;
-      }
+      for (int i = 0; i < VPL; ++i)
+        if (i == (widx >> 5)) key[i] = 0u;
     }
-    if ((bi & 31) == lane) taken |= 1u << (bi >> 5);
     if (lane == r) {
-      my_logit = best;
-      my_id = bi;
+      my_logit = key_logit(wbest);
+      my_id = widx;
     }
   }
   const float ex = (lane < topk) ? expf(my_logit - m) : 0.f;
