@@ -505,12 +505,26 @@ __global__ void __launch_bounds__(kThreads, 1)
             sw_a = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + nt) * kb_n;
             sw_b = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + I / 128 + nt) * kb_n;
           }
-          float sa_next = (*(sa_p));
+          // the scales of K block kb are loaded two blocks ahead: their global-load latency
+          // would otherwise sit between two accumulator drains on the MMA's critical path
+          float sa0 = (*(sa_p)), swa0 = (*(sw_a)), swb0 = (*(sw_b));
+          float sa1 = 0.f, swa1 = 0.f, swb1 = 0.f;
+          if (kb_n > 1) {
+            sa1 = (*(sa_p + static_cast<size_t>(args.capacity)));
+            swa1 = (*(sw_a + 1));
+            swb1 = (*(sw_b + 1));
+          }
           for (int kb = 0; kb < kb_n; ++kb) {
-            const float sa = sa_next;
-            if (kb + 1 < kb_n) sa_next = (*(sa_p + static_cast<size_t>(kb + 1) * args.capacity));
-            const float fa = sa * (*(sw_a + kb));
-            const float fb = sa * (*(sw_b + kb));
+            const float fa = sa0 * swa0;
+            const float fb = sa0 * swb0;
+            sa0 = sa1;
+            swa0 = swa1;
+            swb0 = swb1;
+            if (kb + 2 < kb_n) {
+              sa1 = (*(sa_p + static_cast<size_t>(kb + 2) * args.capacity));
+              swa1 = (*(sw_a + kb + 2));
+              swb1 = (*(sw_b + kb + 2));
+            }
             if (!warp_wait(&acc_full[abuf], aphase, abort_flag, args.status, kWhereEpiAcc)) {
               ok = false;
               break;
@@ -691,9 +705,10 @@ __global__ void __launch_bounds__(kThreads, 1)
         float acc_b[kDown ? 1 : kHT];              // up (GEMM1)
         // GEMM2: the tokens' flat ids and routed weights, read before the K loop so that
         // their latency is not on the tile's tail
-        int flat_j[kDown ? kHT : 1];
-        float wt_j[kDown ? kHT : 1];
-        if constexpr (kDown) {
+        constexpr bool kPrefetchRows = kDown && kHT <= 16;
+        int flat_j[kPrefetchRows ? kHT : 1];
+        float wt_j[kPrefetchRows ? kHT : 1];
+        if constexpr (kPrefetchRows) {
 #pragma unroll
           for (int j = 0; j < kHT; ++j) flat_j[j] = (*(args.sorted_ids + tok0 + j));
 #pragma unroll
@@ -719,13 +734,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             sw_a = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + nt) * kb_n;
             sw_b = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + I / 128 + nt) * kb_n;
           }
-          for (int kb = ks0; kb < ks1; ++kb) {
-            const float swa = (*(sw_a + kb));
-            const float swb = (*(sw_b + kb));
-            const float* sa_p = args.a_scale_t + static_cast<size_t>(kb) * args.capacity + tok0;
-            float fa[kHT];
+          // the scales of K block kb + 1 are loaded right after block kb's drain, so their
+          // latency overlaps the wait for the next accumulator instead of following it
+          float swa = (*(sw_a + ks0)), swb = (*(sw_b + ks0));
+          float fa[kHT];
 #pragma unroll
-            for (int j = 0; j < kHT; ++j) fa[j] = (*(sa_p + j));
+          for (int j = 0; j < kHT; ++j) fa[j] = (*(args.a_scale_t + static_cast<size_t>(ks0) * args.capacity + tok0 + j));
+          for (int kb = ks0; kb < ks1; ++kb) {
             if (!warp_wait(&acc_full[abuf], aphase, abort_flag, args.status, kWhereEpiAcc)) {
               ok = false;
               break;
@@ -747,6 +762,13 @@ __global__ void __launch_bounds__(kThreads, 1)
             tc_fence_before();
             __syncwarp();
             if (lane == 0) mbar_arrive(&acc_empty[abuf]);
+            if (kb + 1 < ks1) {
+              swa = (*(sw_a + kb + 1));
+              swb = (*(sw_b + kb + 1));
+              const float* sa_p = args.a_scale_t + static_cast<size_t>(kb + 1) * args.capacity + tok0;
+#pragma unroll
+              for (int j = 0; j < kHT; ++j) fa[j] = (*(sa_p + j));
+            }
             if (++abuf == C::kAccBufs) {
               abuf = 0;
               aphase ^= 1u;
@@ -841,8 +863,15 @@ __global__ void __launch_bounds__(kThreads, 1)
           const int hcol = nt * 128 + row;
 #pragma unroll
           for (int j = 0; j < kHT; ++j) {
-            if (flat_j[j] < args.nflat)
-              y[static_cast<size_t>(flat_j[j]) * H + hcol] = __float2bfloat16_rn(acc_a[j] * wt_j[j]);
+            if constexpr (kPrefetchRows) {
+              if (flat_j[j] < args.nflat)
+                y[static_cast<size_t>(flat_j[j]) * H + hcol] = __float2bfloat16_rn(acc_a[j] * wt_j[j]);
+            } else {
+              const int flat = (*(args.sorted_ids + tok0 + j));
+              if (flat < args.nflat)
+                y[static_cast<size_t>(flat) * H + hcol] =
+                    __float2bfloat16_rn(acc_a[j] * route_weight(args.topk_weights, flat));
+            }
           }
         }
       }
