@@ -140,6 +140,24 @@ __device__ __forceinline__ void bulk_load(void* smem_dst, const void* src, uint3
       : "memory");
 }
 
+// Asynchronous bulk store of `bytes` (a multiple of 16) from shared to global
+// memory, both addresses 16-byte aligned, tracked by the issuing thread's bulk
+// groups; the shared source must be made visible to the async proxy first
+// (fence_proxy_async_smem after the generic stores that wrote it).
+__device__ __forceinline__ void bulk_store(void* dst, const void* smem_src, uint32_t bytes) {
+  asm volatile("cp.async.bulk.global.shared::cta.bulk_group [%0], [%1], %2;" ::"l"(reinterpret_cast<uint64_t>(dst)),
+               "r"(smem_u32(smem_src)), "r"(bytes)
+               : "memory");
+}
+__device__ __forceinline__ void bulk_commit() { asm volatile("cp.async.bulk.commit_group;" ::: "memory"); }
+// this thread's earlier bulk stores have finished reading shared memory
+__device__ __forceinline__ void bulk_wait_read_all() { asm volatile("cp.async.bulk.wait_group.read 0;" ::: "memory"); }
+// this thread's earlier bulk stores have completed
+__device__ __forceinline__ void bulk_wait_all() { asm volatile("cp.async.bulk.wait_group 0;" ::: "memory"); }
+__device__ __forceinline__ void fence_proxy_async_smem() {
+  asm volatile("fence.proxy.async.shared::cta;" ::: "memory");
+}
+
 // TMA gather of four rows (tile::gather4): rows y0..y3 of a 2-D tensor map whose
 // box is one row high, x the first column, into 4 consecutive box rows at
 // smem_dst (the 128-byte swizzle follows the shared-memory address, so four

@@ -68,7 +68,14 @@ struct Cfg {
   static constexpr int kTokBytes = kTokRows * 128;
   static constexpr int kWBytes = kWRows * 128;
   static constexpr int kStageBytes = kTokBytes + kWBytes;
-  static constexpr int kStagesFit = (kSmemLimit - kSmemReserve - 1024) / kStageBytes;
+  // GEMM2 FP8 normal tiles stage each output row in shared memory and write it with one
+  // asynchronous bulk copy (256 contiguous bytes per row): a thread's own row stored from
+  // registers would take 16 scattered 16-byte stores, which cost a third of the kernel.  The
+  // staging area (pitch 272 bytes: 16-byte aligned, 4-way bank spread) takes one ring stage.
+  static constexpr bool kStageY = kDown && kFP8 && !kSwap;
+  static constexpr int kYPitch = 272;
+  static constexpr int kYStageBytes = kStageY ? 256 * kYPitch : 0;
+  static constexpr int kStagesFit = (kSmemLimit - kSmemReserve - 1024 - kYStageBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
   static constexpr int kMmaN = kSwap ? kBM : 256;
   static constexpr int kAccCols = kSwap ? (kDown ? kBM : 2 * kBM) : 256;
@@ -81,8 +88,10 @@ struct Cfg {
   // output columns per tile: GEMM1 -> 128 intermediate columns; GEMM2 -> H columns
   static constexpr int kTileN = kDown ? (kSwap ? 128 : 256) : 128;
   static constexpr int kHalfTok = kBM / 2;  // swap: token columns per epilogue group
-  static constexpr size_t kSmemBytes = static_cast<size_t>(kStages) * kStageBytes + kSmemReserve + 1024;
+  static constexpr size_t kSmemBytes =
+      static_cast<size_t>(kStages) * kStageBytes + kSmemReserve + kYStageBytes + 1024;
   static_assert(kStages >= 2, "pipeline needs at least two stages");
+  static_assert(kSmemBytes <= static_cast<size_t>(kSmemLimit), "shared memory");
   static_assert(kTmemCols <= 512, "TMEM holds 512 columns");
   static_assert(kAccBufs >= 2, "accumulators are at least double-buffered");
   static_assert((2 * kStages + 2 * kAccBufs + 3) * 8 + 8 <= kXchgOffset, "barriers overlap the exchange buffers");
@@ -655,13 +664,18 @@ __global__ void __launch_bounds__(kThreads, 1)
               static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(real ? flat : 0) * H + nt * 256 + g * 128;
           if constexpr (kFP8) {
             if (real) {
+              uint8_t* st_row = reserve + kSmemReserve + static_cast<size_t>(threadIdx.x - 64) * C::kYPitch;
+              bulk_wait_read_all();   // the previous row copy from this staging slot has read it
 #pragma unroll
               for (int c = 0; c < 8; ++c) {
                 float v[16];
 #pragma unroll
                 for (int i = 0; i < 16; ++i) v[i] = acc_a[16 * c + i] * wt;
-                store_bf16x16(yrow + 16 * c, v);
+                store_bf16x16(reinterpret_cast<__nv_bfloat16*>(st_row + 32 * c), v);
               }
+              fence_proxy_async_smem();
+              bulk_store(yrow, st_row, 256);
+              bulk_commit();
             }
           } else {
             if (!warp_wait(&acc_full[abuf], aphase, abort_flag, args.status, kWhereEpiAcc)) {
@@ -876,6 +890,7 @@ __global__ void __launch_bounds__(kThreads, 1)
         }
       }
     }
+    if constexpr (C::kStageY) bulk_wait_all();   // this thread's row copies are complete
   }
 
   __syncwarp();
