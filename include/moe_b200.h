@@ -87,7 +87,7 @@ extern "C" {
 
 /* tile orientation of the two grouped GEMMs */
 #define MOE_MODE_AUTO 0    /* chosen from the expected tokens per expert */
-#define MOE_MODE_NORMAL 1  /* MMA M = 128 token rows (block_m 128), or 256 over two SMs (FP8, block_m 256), N = 256 */
+#define MOE_MODE_NORMAL 1  /* MMA M = 128 token rows (block_m 128), N = 256 weight rows */
 #define MOE_MODE_SWAP_AB 2 /* MMA M = 128 weight rows, N = block_m token rows */
 
 /* stages of moe_forward_stages, in pipeline order */
@@ -117,7 +117,7 @@ typedef struct moe_problem {
   int32_t I;            /* expert intermediate size */
   int32_t weight_dtype; /* MOE_DTYPE_* */
   int32_t mode;         /* MOE_MODE_* */
-  int32_t block_m;      /* rows per expert block: 16, 32, 64 (swap-AB); 128, or 256 for FP8 two-SM tiles (normal); 0 = auto */
+  int32_t block_m;      /* rows per expert block: 16, 32, 64 (swap-AB); 128 (normal); 0 = auto */
   int32_t renormalize;  /* router: 1 = renormalise the chosen softmax weights (default), 0 = keep them */
   int32_t split_k;      /* swap-AB GEMMs: 0 = split K when few tiles are in flight (default), 1 = never */
   /* 1 = scale each token row by its router weight before GEMM1 instead of the
@@ -170,7 +170,7 @@ typedef struct moe_workspace_layout {
   int64_t expert_offsets;   /* int32 [E + 1] */
   int64_t align_scratch;    /* int32 [chunks * E] */
   int64_t pos_of_flat;      /* int32 [T*topk]: sorted row of each assignment, -1 for a bad id or another
-                               rank's expert (FP8 / MXFP8 except two-SM tiles, and every expert-parallel call) */
+                               rank's expert (FP8 / MXFP8, and every expert-parallel call) */
   int64_t a1;               /* GEMM1 token rows.  Normal tiles: x rows in sorted order [capacity, H], bf16 or
                                E4M3 (padding rows unspecified).  Swap-AB: one row per token [T, H] -- E4M3
                                codes (FP8) or bf16(x * w) (router weight on the input) -- gathered by TMA;

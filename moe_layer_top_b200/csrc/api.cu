@@ -110,15 +110,13 @@ int validate_problem(const moe_problem* p) {
     if (p->block_m != 0 && p->block_m != 128)
       return fail(MOE_ERR_INVALID, "MXFP8 weights use block_m = 128 (got %d)", p->block_m);
   }
-  if (p->block_m == 256 && !fp8)
-    return fail(MOE_ERR_INVALID, "block_m = 256 (two-SM tiles) needs FP8 weights");
-  if (p->mode == MOE_MODE_NORMAL && p->block_m != 0 && p->block_m != 128 && p->block_m != 256)
-    return fail(MOE_ERR_INVALID, "normal mode uses block_m = 128 or 256 (got %d)", p->block_m);
+  if (p->mode == MOE_MODE_NORMAL && p->block_m != 0 && p->block_m != 128)
+    return fail(MOE_ERR_INVALID, "normal mode uses block_m = 128 (got %d)", p->block_m);
   if (p->mode == MOE_MODE_SWAP_AB && p->block_m != 0 && p->block_m != 16 && p->block_m != 32 && p->block_m != 64)
     return fail(MOE_ERR_INVALID, "swap-AB mode uses block_m in {16, 32, 64} (got %d)", p->block_m);
   if (p->mode == MOE_MODE_AUTO && p->block_m != 0 && p->block_m != 16 && p->block_m != 32 && p->block_m != 64 &&
-      p->block_m != 128 && p->block_m != 256)
-    return fail(MOE_ERR_INVALID, "block_m %d not in {16, 32, 64, 128, 256}", p->block_m);
+      p->block_m != 128)
+    return fail(MOE_ERR_INVALID, "block_m %d not in {16, 32, 64, 128}", p->block_m);
   return MOE_OK;
 }
 
@@ -145,7 +143,7 @@ void resolve(moe_problem* p) {
   }
   if (p->block_m == 0) {
     if (p->mode == MOE_MODE_NORMAL)
-      p->block_m = 128;  // the two-SM FP8 tiles (block_m 256) are opt-in: slower so far
+      p->block_m = 128;
     else
       p->block_m = avg <= 8.0 ? 16 : (avg <= 20.0 ? 32 : 64);
   }
@@ -164,7 +162,6 @@ struct Plan {
   int64_t nflat;
   bool fp8;   // 8-bit weights and activations (block-128 or MX scales)
   bool mx;    // MXFP8: E8M0 scale factors per 32 elements
-  bool pair;        // two-SM FP8 tiles
   bool tok_gather;  // swap-AB: GEMM1 gathers token rows (TMA gather4) from x or its per-token copy;
                     // normal tiles read a sorted copy a1 [capacity, H] (gather4 is too slow for 128-row tiles)
   bool ep;          // expert parallelism: some assignments go to other ranks' experts
@@ -179,7 +176,6 @@ int make_plan(const moe_problem* in, Plan* plan) {
   const moe_problem& p = plan->p;
   plan->mx = p.weight_dtype == MOE_DTYPE_MXFP8_E4M3;
   plan->fp8 = p.weight_dtype == MOE_DTYPE_FP8_E4M3 || plan->mx;
-  plan->pair = p.mode == MOE_MODE_NORMAL && p.block_m == 256;
   plan->tok_gather = p.mode == MOE_MODE_SWAP_AB;
   plan->ep = expert_parallel(&p);
   plan->er = moe::ExpertRange{p.first_expert, global_experts(&p)};
@@ -215,7 +211,7 @@ int make_plan(const moe_problem* in, Plan* plan) {
   else
     L.a1 = -1;
   // the inverse permutation: FP8 scale scatter, and the combine's mask under expert parallelism
-  L.pos_of_flat = ((plan->fp8 && !plan->pair) || plan->ep) ? take(plan->nflat * 4) : -1;
+  L.pos_of_flat = (plan->fp8 || plan->ep) ? take(plan->nflat * 4) : -1;
   // FP8: fp32 [K/128, cap]; MXFP8: E8M0 SF atoms, (cap/128) * (K/128) * 512 bytes -- the same size
   L.a1_scale = plan->fp8 ? take(cap * (p.H / 128) * 4) : -1;
   L.a2 = take(cap * p.I * elem);
@@ -367,7 +363,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
         if (e != cudaSuccess) return cuda_fail(e, "align");
         break;
       case MOE_STAGE_GATHER:
-        if (!plan.tok_gather && plan.fp8 && !plan.pair) {
+        if (!plan.tok_gather && plan.fp8) {
           // normal FP8 / MXFP8 tiles: quantise once per token into the (not yet used)
           // y region, scattering the scales to the sorted rows, then copy code rows
           void* xq = at<void>(ws, L.y);

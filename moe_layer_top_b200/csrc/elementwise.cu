@@ -1,7 +1,7 @@
 // Memory-bound helpers of the MoE pipeline: preparing GEMM1's token rows
 // (per-token FP8 / MXFP8 quantisation with scales scattered to the sorted
 // rows, the sorted copy of those code rows for normal tiles, the bf16 gather
-// for normal bf16 tiles and the two-SM tiles, the router-weight scaling), the
+// for normal bf16 tiles, the router-weight scaling), the
 // top-k combine, and the FP8 128x128 and MXFP8 weight quantisers used when
 // weights are prepared.  All move 16-byte vectors per thread.
 #include "common.cuh"

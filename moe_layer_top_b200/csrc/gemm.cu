@@ -1283,332 +1283,6 @@ __global__ void __launch_bounds__(kThreads, 1)
 }
 
 // ----------------------------------------------------------------------------
-// Normal orientation, FP8, two SMs per tile (tcgen05 cta_group::2).
-//
-// A cluster of two CTAs computes a 256 x 256 tile: CTA r holds token rows
-// [128 r, 128 r + 128) of a 256-row expert block and weight rows
-// [128 r, 128 r + 128) of the tile's 256 (GEMM1: r = 0 the gate rows, r = 1 the
-// up rows of one 128-column intermediate group; GEMM2: two 128-row halves of
-// 256 output columns).  The leader CTA (rank 0) issues the MMA (M = 256,
-// N = 256) that reads both CTAs' shared memory; each CTA's TMEM receives its
-// own 128 rows x 256 columns, so the epilogue of each CTA is the single-SM
-// one.  Per K block each SM loads 32 KB (not 48 KB) and its tensor core reads
-// half of B, which keeps the shared-memory port below its bandwidth.
-//
-// Hand-offs: both CTAs' TMA loads count their bytes on the leader's full
-// barrier; the leader's MMA commits multicast to both CTAs' empty and
-// acc_full barriers; both CTAs' epilogue warps arrive on the leader's
-// acc_empty barrier (16 arrivals).  All waits are bounded.
-// ----------------------------------------------------------------------------
-template <bool kDown>
-struct CfgPair {
-  static constexpr int kTokBytes = 128 * 128;  // this CTA's 128 token rows x 128 K bytes
-  static constexpr int kWBytes = 128 * 128;    // this CTA's 128 of the 256 weight rows
-  static constexpr int kStageBytes = kTokBytes + kWBytes;
-  static constexpr int kStages = 6;
-  static constexpr int kAccCols = 256;
-  static constexpr int kTmemCols = 512;
-  static constexpr int kTileN = kDown ? 256 : 128;  // output columns per tile
-  static constexpr size_t kSmemBytes = static_cast<size_t>(kStages) * kStageBytes + kSmemReserve + 1024;
-  static_assert(kSmemBytes <= static_cast<size_t>(kSmemLimit), "shared memory");
-};
-
-template <bool kDown>
-__global__ void __launch_bounds__(kThreads, 1)
-    moe_gemm_fp8_pair_kernel(const __grid_constant__ CUtensorMap tm_tok, const __grid_constant__ CUtensorMap tm_w,
-                             const Args args) {
-  using C = CfgPair<kDown>;
-  extern __shared__ uint8_t smem_raw[];
-  uint8_t* smem = reinterpret_cast<uint8_t*>((reinterpret_cast<uintptr_t>(smem_raw) + 1023) & ~uintptr_t(1023));
-  uint8_t* reserve = smem + static_cast<size_t>(C::kStages) * C::kStageBytes;
-  uint64_t* full = reinterpret_cast<uint64_t*>(reserve);
-  uint64_t* empty = full + C::kStages;
-  uint64_t* acc_full = empty + C::kStages;
-  uint64_t* acc_empty = acc_full + 2;
-  uint64_t* xchg_bar = acc_empty + 2;
-  uint64_t* drain = xchg_bar + 2;
-  uint32_t* tmem_slot = reinterpret_cast<uint32_t*>(drain + 1);
-  volatile int* abort_flag = reinterpret_cast<volatile int*>(tmem_slot + 1);
-  float* xchg = reinterpret_cast<float*>(reserve + kXchgOffset);
-
-  const int warp = threadIdx.x >> 5, lane = threadIdx.x & 31;
-  const uint32_t rank = cluster_ctarank();
-  const bool leader = rank == 0;
-  pdl_launch_dependents();
-  if (threadIdx.x == 0) {
-    for (int s = 0; s < C::kStages; ++s) {
-      mbar_init(&full[s], 1);
-      mbar_init(&empty[s], 1);
-    }
-    for (int b = 0; b < 2; ++b) {
-      mbar_init(&acc_full[b], 1);
-      mbar_init(&acc_empty[b], 2 * kEpiWarps);
-      mbar_init(&xchg_bar[b], kEpiWarps * 32);
-    }
-    mbar_init(drain, 1);
-    *abort_flag = 0;
-    fence_mbar_init();
-  }
-  if (warp == 0 && lane == 0) {
-    tma_prefetch_desc(&tm_tok);
-    tma_prefetch_desc(&tm_w);
-  }
-  if (warp == 1) {
-    tmem_alloc_pair(tmem_slot, C::kTmemCols);
-    tmem_relinquish_pair();
-  }
-  tc_fence_before();
-  cluster_sync();  // barriers of both CTAs initialised before any remote arrival
-  tc_fence_after();
-  const uint32_t tmem_base = *tmem_slot;
-  pdl_wait();
-
-  const int H = args.H, I = args.I;
-  const int K = kDown ? I : H;
-  const int kb_n = K / 128;
-  const int n_tiles = (kDown ? H : I) / C::kTileN;
-  const int num_tiles = ((*(args.ntpp)) / 256) * n_tiles;
-  const int cluster = blockIdx.x >> 1, n_clusters = gridDim.x >> 1;
-
-  if (warp == 0) {
-    // ------------------------------------------------------------------ producer (both CTAs)
-    if (lane == 0) {
-      const uint64_t pol_w = policy_evict_first();
-      const uint64_t pol_a = policy_evict_last();
-      int stage = 0;
-      uint32_t phase = 0;
-      long long fills = 0;
-      bool ok = true;
-      for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
-        const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
-        const int e = (*(args.expert_ids + mb));
-        const int tok_row = mb * 256 + 128 * static_cast<int>(rank);
-        const int w_row = kDown ? e * H + nt * 256 + 128 * static_cast<int>(rank)
-                                : e * 2 * I + (rank ? I : 0) + nt * 128;
-        for (int kb = 0; kb < kb_n; ++kb) {
-          if (!mbar_wait(&empty[stage], phase ^ 1u, abort_flag, args.status,
-                         MOE_STATUS_WAIT_TIMEOUT | kWhereProducer)) {
-            ok = false;
-            break;
-          }
-          uint8_t* st = smem + static_cast<size_t>(stage) * C::kStageBytes;
-          if (leader) mbar_arrive_expect_tx(&full[stage], 2 * C::kStageBytes);
-          const uint32_t bar = map_to_rank(&full[stage], 0);
-          tma_load_2d_pair(st, &tm_tok, bar, kb * 128, tok_row, pol_a);
-          tma_load_2d_pair(st + C::kTokBytes, &tm_w, bar, kb * 128, w_row, pol_w);
-          ++fills;
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      if (!ok && leader) {
-        // the leader's full barriers count both CTAs' copies: let them land
-        for (int s = 0; s < C::kStages; ++s) {
-          const long long n_s = fills / C::kStages + (s < fills % C::kStages ? 1 : 0);
-          if (n_s > 0) {
-            const uint64_t t0 = globaltimer_ns();
-            while (!mbar_try_wait(&full[s], static_cast<uint32_t>((n_s - 1) & 1)) &&
-                   globaltimer_ns() - t0 < kWaitTimeoutNs) {
-            }
-          }
-        }
-      }
-    }
-  } else if (warp == 1) {
-    // ------------------------------------------------------------------ MMA issuer (leader only)
-    if (lane == 0 && leader) {
-      constexpr uint32_t idesc = make_idesc(256, 256, true);
-      int stage = 0, abuf = 0;
-      uint32_t phase = 0, aphase = 0;
-      bool ok = true;
-      for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
-        for (int kb = 0; kb < kb_n; ++kb) {
-          if (!mbar_wait(&full[stage], phase, abort_flag, args.status, MOE_STATUS_WAIT_TIMEOUT | kWhereMma) ||
-              !mbar_wait(&acc_empty[abuf], aphase ^ 1u, abort_flag, args.status,
-                         MOE_STATUS_WAIT_TIMEOUT | kWhereMma)) {
-            ok = false;
-            break;
-          }
-          tc_fence_after();
-          const uint32_t d = tmem_base + static_cast<uint32_t>(abuf * C::kAccCols);
-          const uint32_t tok = smem_u32(smem + static_cast<size_t>(stage) * C::kStageBytes);
-          const uint32_t w = tok + C::kTokBytes;
-#pragma unroll
-          for (int k = 0; k < 4; ++k) {
-            const uint32_t koff = k * 32;
-            mma_fp8_pair(d, smem_desc_sw128(tok + koff), smem_desc_sw128(w + koff), idesc, k > 0 ? 1u : 0u);
-          }
-          mma_commit_pair(&empty[stage]);
-          mma_commit_pair(&acc_full[abuf]);
-          abuf ^= 1;
-          if (abuf == 0) aphase ^= 1u;
-          if (++stage == C::kStages) {
-            stage = 0;
-            phase ^= 1u;
-          }
-        }
-      }
-      mma_commit_pair_mask(drain, 1);  // tracks this thread's cta_group::2 MMAs
-      const uint64_t t0 = globaltimer_ns();
-      while (!mbar_try_wait(drain, 0)) {
-        if (globaltimer_ns() - t0 > kWaitTimeoutNs) {
-          report_status(args.status, MOE_STATUS_WAIT_TIMEOUT | kWhereDrain);
-          break;
-        }
-      }
-    }
-  } else {
-    // ------------------------------------------------------------------ epilogue (both CTAs)
-    const int q = warp & 3;
-    const int g = (warp - 2) >> 2;
-    const int row = 32 * q + lane;
-    const uint32_t lane_addr = static_cast<uint32_t>(32 * q) << 16;
-    const uint32_t acc_empty_leader[2] = {map_to_rank(&acc_empty[0], 0), map_to_rank(&acc_empty[1], 0)};
-    constexpr int kCols = kDown ? 128 : 64;
-    int abuf = 0, xbuf = 0;
-    uint32_t aphase = 0, xphase = 0;
-    bool ok = true;
-    for (int tile = cluster; tile < num_tiles && ok; tile += n_clusters) {
-      const int mb = tile / n_tiles, nt = tile - mb * n_tiles;
-      const int e = (*(args.expert_ids + mb));
-      const int grow = mb * 256 + 128 * static_cast<int>(rank) + row;
-      uint32_t acc_a[kCols];  // fp32 bits
-      uint32_t acc_b[kDown ? 1 : kCols];
-#pragma unroll
-      for (int i = 0; i < kCols; ++i) acc_a[i] = 0u;
-      if constexpr (!kDown) {
-#pragma unroll
-        for (int i = 0; i < kCols; ++i) acc_b[i] = 0u;
-      }
-      const float* sa_p = args.a_scale_t + grow;
-      const float* sw_a;
-      const float* sw_b;
-      if constexpr (kDown) {
-        sw_a = args.w_scale + (static_cast<size_t>(e) * (H / 128) + nt * 2 + g) * kb_n;
-        sw_b = sw_a;
-      } else {
-        sw_a = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + nt) * kb_n;
-        sw_b = args.w_scale + (static_cast<size_t>(e) * (2 * I / 128) + I / 128 + nt) * kb_n;
-      }
-      float sa_c = *sa_p, wa_c = *sw_a, wb_c = *sw_b;
-      for (int kb = 0; kb < kb_n; ++kb) {
-        float sa_n = 0.f, wa_n = 0.f, wb_n = 0.f;
-        if (kb + 1 < kb_n) {
-          sa_n = *(sa_p + static_cast<size_t>(kb + 1) * args.capacity);
-          wa_n = *(sw_a + kb + 1);
-          wb_n = *(sw_b + kb + 1);
-        }
-        const float fa = sa_c * wa_c;
-        const float fb = sa_c * wb_c;
-        if (!warp_wait(&acc_full[abuf], aphase, abort_flag, args.status, kWhereEpiAcc)) {
-          ok = false;
-          break;
-        }
-        tc_fence_after();
-        const uint32_t t0 = tmem_base + lane_addr + static_cast<uint32_t>(abuf * C::kAccCols);
-        if constexpr (kDown) {
-#pragma unroll
-          for (int c = 0; c < kCols / 16; c += 2) {
-            uint32_t d0[16], d1[16];
-            tmem_ld16u(t0 + g * 128 + 16 * c, d0);
-            tmem_ld16u(t0 + g * 128 + 16 * c + 16, d1);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              acc_a[16 * c + i] = __float_as_uint(fmaf(__uint_as_float(d0[i]), fa, __uint_as_float(acc_a[16 * c + i])));
-              acc_a[16 * c + 16 + i] =
-                  __float_as_uint(fmaf(__uint_as_float(d1[i]), fa, __uint_as_float(acc_a[16 * c + 16 + i])));
-            }
-          }
-        } else {
-#pragma unroll
-          for (int c = 0; c < kCols / 16; ++c) {
-            uint32_t dg[16], du[16];
-            tmem_ld16u(t0 + g * 64 + 16 * c, dg);
-            tmem_ld16u(t0 + 128 + g * 64 + 16 * c, du);
-            tmem_wait_ld();
-#pragma unroll
-            for (int i = 0; i < 16; ++i) {
-              acc_a[16 * c + i] = __float_as_uint(fmaf(__uint_as_float(dg[i]), fa, __uint_as_float(acc_a[16 * c + i])));
-              acc_b[16 * c + i] = __float_as_uint(fmaf(__uint_as_float(du[i]), fb, __uint_as_float(acc_b[16 * c + i])));
-            }
-          }
-        }
-        tc_fence_before();
-        __syncwarp();
-        if (lane == 0) mbar_arrive_cluster(acc_empty_leader[abuf]);
-        abuf ^= 1;
-        if (abuf == 0) aphase ^= 1u;
-        sa_c = sa_n;
-        wa_c = wa_n;
-        wb_c = wb_n;
-      }
-      if (!ok) break;
-
-      if constexpr (!kDown) {
-        // SiLU(gate) * up and the per-(row, 128) FP8 requantisation
-        float amax = 0.f;
-#pragma unroll
-        for (int i = 0; i < 64; ++i) {
-          const float p = swiglu_bf16(bf16_round(__uint_as_float(acc_a[i])), bf16_round(__uint_as_float(acc_b[i])),
-                                      args.swiglu_limit);
-          acc_a[i] = __float_as_uint(p);
-          amax = fmaxf(amax, fabsf(p));
-        }
-        float* xb = xchg + xbuf * 256;
-        xb[g * 128 + row] = amax;
-        mbar_arrive(&xchg_bar[xbuf]);
-        if (!warp_wait(&xchg_bar[xbuf], xphase, abort_flag, args.status, kWhereEpiXchg)) {
-          ok = false;
-          break;
-        }
-        amax = fmaxf(xb[row], xb[128 + row]);
-        xbuf ^= 1;
-        if (xbuf == 0) xphase ^= 1u;
-        const float scale = act_scale_from_amax(amax);
-        const float inv = pow2_recip(scale);
-        uint32_t words[16];
-#pragma unroll
-        for (int i = 0; i < 16; ++i) {
-          const float* v = reinterpret_cast<const float*>(acc_a) + 4 * i;
-          words[i] = static_cast<uint32_t>(f32x2_to_e4m3x2(v[0] * inv, v[1] * inv)) |
-                     (static_cast<uint32_t>(f32x2_to_e4m3x2(v[2] * inv, v[3] * inv)) << 16);
-        }
-        uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) + static_cast<size_t>(grow) * I +
-                                              nt * 128 + g * 64);
-#pragma unroll
-        for (int i = 0; i < 4; ++i) dst[i] = make_uint4(words[4 * i], words[4 * i + 1], words[4 * i + 2], words[4 * i + 3]);
-        if (g == 0) args.out_scale_t[static_cast<size_t>(nt) * args.capacity + grow] = scale;
-      } else {
-        const int flat = *(args.sorted_ids + grow);
-        if (flat < args.nflat) {
-          const float wt = route_weight(args.topk_weights, flat);
-          __nv_bfloat16* yrow =
-              static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(flat) * H + nt * 256 + g * 128;
-#pragma unroll
-          for (int c = 0; c < 8; ++c) {
-            float v[16];
-#pragma unroll
-            for (int i = 0; i < 16; ++i) v[i] = __uint_as_float(acc_a[16 * c + i]) * wt;
-            store_bf16x16(yrow + 16 * c, v);
-          }
-        }
-      }
-    }
-  }
-
-  __syncwarp();
-  tc_fence_before();
-  cluster_sync();  // the leader's MMAs read this CTA's shared memory: leave together
-  if (warp == 1) {
-    tc_fence_after();
-    tmem_dealloc_pair(tmem_base, C::kTmemCols);
-  }
-}
-
-// ----------------------------------------------------------------------------
 // host side
 // ----------------------------------------------------------------------------
 PFN_cuTensorMapEncodeTiled_v12000 encode_fn() {
@@ -1679,57 +1353,6 @@ cudaError_t launch_on(const GemmProblem& p, const void* tok, const void* w, cons
 }
 
 template <bool kDown>
-cudaError_t launch_fp8_pair(const GemmProblem& p, const void* tok, const void* w, const Args& args, cudaStream_t s) {
-  using C = CfgPair<kDown>;
-  auto kern = moe_gemm_fp8_pair_kernel<kDown>;
-  static bool attr_set = false;
-  if (!attr_set) {
-    cudaError_t e = cudaFuncSetAttribute(kern, cudaFuncAttributeMaxDynamicSharedMemorySize,
-                                         static_cast<int>(C::kSmemBytes));
-    if (e != cudaSuccess) return e;
-    attr_set = true;
-  }
-  const long long K = kDown ? p.I : p.H;
-  const long long wrows = kDown ? static_cast<long long>(p.E) * p.H : static_cast<long long>(p.E) * 2 * p.I;
-  CUtensorMap tm_tok, tm_w;
-  if (!make_map(&tm_tok, tok, p.capacity, K, 1, 128)) return cudaErrorInvalidValue;
-  if (!make_map(&tm_w, w, wrows, K, 1, 128)) return cudaErrorInvalidValue;
-  const int n_tiles = (kDown ? p.H : p.I) / C::kTileN;
-  const long long max_tiles = static_cast<long long>(p.capacity / 256) * n_tiles;
-  cudaLaunchConfig_t cfg = {};
-  cfg.blockDim = dim3(kThreads);
-  cfg.dynamicSmemBytes = C::kSmemBytes;
-  cfg.stream = s;
-  cudaLaunchAttribute attr[2];
-  attr[0].id = cudaLaunchAttributeProgrammaticStreamSerialization;
-  attr[0].val.programmaticStreamSerializationAllowed = 1;
-  attr[1].id = cudaLaunchAttributeClusterDimension;
-  attr[1].val.clusterDim.x = 2;
-  attr[1].val.clusterDim.y = 1;
-  attr[1].val.clusterDim.z = 1;
-  cfg.attrs = attr;
-  cfg.numAttrs = 2;
-  // The kernel is persistent: every cluster must be resident at once, or the
-  // clusters that do not fit run their whole share of tiles after the others.
-  // Not every SM can pair up (the SM count per GPC need not be even), so the
-  // grid is the number of clusters that fit, not num_sms / 2.
-  static int max_clusters = 0;
-  if (max_clusters == 0) {
-    cfg.gridDim = dim3(static_cast<unsigned>(p.num_sms / 2 * 2));
-    int n = 0;
-    cudaError_t e = cudaOccupancyMaxActiveClusters(&n, kern, &cfg);
-    if (e != cudaSuccess) return e;
-    max_clusters = n > 0 ? n : 1;
-  }
-  long long grid = 2LL * max_clusters;
-  if (grid > p.num_sms / 2 * 2) grid = p.num_sms / 2 * 2;
-  if (2 * max_tiles < grid) grid = 2 * max_tiles;
-  if (grid <= 0) return cudaSuccess;
-  cfg.gridDim = dim3(static_cast<unsigned>(grid));
-  return cudaLaunchKernelEx(&cfg, kern, tm_tok, tm_w, args);
-}
-
-template <bool kDown>
 cudaError_t launch_mx(const GemmProblem& p, const void* tok, const void* w, const Args& args, cudaStream_t s) {
   using C = CfgMx<kDown>;
   auto kern = moe_gemm_mx_kernel<kDown>;
@@ -1759,12 +1382,7 @@ cudaError_t dispatch(const GemmProblem& p, const void* tok, const void* w, const
   if constexpr (kFP8) {
     if (p.mx) return launch_mx<kDown>(p, tok, w, args, s);
   }
-  if (!p.swap) {
-    if constexpr (kFP8) {
-      if (p.block_m == 256) return launch_fp8_pair<kDown>(p, tok, w, args, s);
-    }
-    return launch_on<kDown, kFP8, false, 128>(p, tok, w, args, s);
-  }
+  if (!p.swap) return launch_on<kDown, kFP8, false, 128>(p, tok, w, args, s);
   switch (p.block_m) {
     case 16: return launch_on<kDown, kFP8, true, 16>(p, tok, w, args, s);
     case 32: return launch_on<kDown, kFP8, true, 32>(p, tok, w, args, s);

@@ -60,8 +60,6 @@ def test_resolve_problem_auto_modes(L):
     assert q.mode == ops.MODE_SWAP_AB and q.block_m == 16
     q = ops.resolve_problem(ops.problem(16384, 128, 8, 4096, 1536, fp8=True))
     assert q.mode == ops.MODE_NORMAL and q.block_m == 128
-    q = ops.resolve_problem(ops.problem(16384, 128, 8, 4096, 1536, fp8=True, block_m=256))
-    assert q.mode == ops.MODE_NORMAL and q.block_m == 256
     q = ops.resolve_problem(ops.problem(16384, 128, 8, 4096, 1536, fp8=False))
     assert q.mode == ops.MODE_NORMAL and q.block_m == 128
     q = ops.resolve_problem(ops.problem(64, 128, 8, 4096, 1536, mode=ops.MODE_NORMAL))
@@ -121,13 +119,14 @@ def test_quantize_mxfp8_argument_errors(L):
 @pytest.mark.parametrize("bad", [
     dict(T=-1), dict(E=0), dict(E=2000), dict(topk=0), dict(topk=9, E=8), dict(H=100), dict(I=0), dict(I=200),
     dict(mode=7), dict(mode=ops.MODE_NORMAL, block_m=16), dict(mode=ops.MODE_SWAP_AB, block_m=128),
-    dict(block_m=48), dict(mode=ops.MODE_NORMAL, block_m=256),
+    dict(block_m=48), dict(mode=ops.MODE_NORMAL, block_m=256), dict(block_m=256),
+    dict(block_m=256, mode=ops.MODE_NORMAL, fp8=True),
 ])
 def test_invalid_problems_are_rejected(L, bad):
     kw = dict(T=16, E=8, topk=2, H=256, I=128)
     kw.update(bad)
     p = ops.problem(kw["T"], kw["E"], kw["topk"], kw["H"], kw["I"], mode=kw.get("mode", 0),
-                    block_m=kw.get("block_m", 0))
+                    block_m=kw.get("block_m", 0), fp8=kw.get("fp8", False))
     assert L.moe_workspace_size(ctypes.byref(p)) == 0
     with pytest.raises(ops.MoeError) as ei:
         ops.resolve_problem(p)
