@@ -304,15 +304,22 @@ __global__ void __launch_bounds__(1024) route_align_small_kernel(
   int32_t* cnt = offs + E + 1;         // [E]
 
   if (logits != nullptr) {
+    // each warp routes tokens warp, warp + 32, ...; the next token's logits are loaded while the
+    // current one is routed
+    float cur[VPL], nxt[VPL];
+    if (warp < T) load_logits<VPL>(logits + static_cast<size_t>(warp) * er.e_global, er.e_global, lane, cur);
     for (int t = warp; t < T; t += 32) {
+      if (t + 32 < T) load_logits<VPL>(logits + static_cast<size_t>(t + 32) * er.e_global, er.e_global, lane, nxt);
       int id;
       float w;
-      route_token<VPL>(logits + static_cast<size_t>(t) * er.e_global, er.e_global, topk, renormalize, lane, id, w);
+      route_token_vals<VPL>(cur, er.e_global, topk, renormalize, lane, id, w);
       if (lane < topk) {
         ids_out[t * topk + lane] = id;
         weights_out[t * topk + lane] = w;
         ids_s[t * topk + lane] = id;
       }
+#pragma unroll
+      for (int i = 0; i < VPL; ++i) cur[i] = nxt[i];
     }
   } else {
     for (int i = tid; i < n; i += 1024) ids_s[i] = (*(ids_in + i));
@@ -384,18 +391,14 @@ __global__ void __launch_bounds__(1024) route_align_small_kernel(
     if (pos_of_flat && i < end) pos_of_flat[i] = dest;  // -1 for an invalid id
     __syncwarp();
   }
-  for (int p = tid; p < capacity; p += 1024) {
-    bool pad = true;
-    if (p < ntpp) {
-      const int e = owner_expert(offs, E, p);
-      pad = p >= offs[e] + cnt[e];
-    }
-    if (pad) sorted_ids[p] = n;
+  // padding: each expert's slots past its count, then everything past num_tokens_post_padded;
+  // block experts: each expert's blocks, then -1 past the used ones
+  for (int e = tid; e < E; e += 1024) {
+    for (int p = offs[e] + cnt[e]; p < offs[e + 1]; ++p) sorted_ids[p] = n;
+    for (int b = offs[e] / block_m; b < offs[e + 1] / block_m; ++b) expert_ids[b] = e;
   }
-  for (int b = tid; b < capacity / block_m; b += 1024) {
-    const int p = b * block_m;
-    expert_ids[b] = (p < ntpp) ? owner_expert(offs, E, p) : -1;
-  }
+  for (int p = ntpp + tid; p < capacity; p += 1024) sorted_ids[p] = n;
+  for (int b = ntpp / block_m + tid; b < capacity / block_m; b += 1024) expert_ids[b] = -1;
   for (int e = tid; e <= E; e += 1024) {
     offsets_out[e] = offs[e];
     if (e < E) counts_out[e] = cnt[e];

@@ -23,21 +23,27 @@ __device__ __forceinline__ float key_logit(uint32_t k) {
   return __uint_as_float((k & 0x80000000u) ? (k & 0x7FFFFFFFu) : ~k);
 }
 
-// One warp routes one token: lane r (< topk) returns the r-th chosen expert
-// and its weight.  Each selection round is two warp reductions (redux.sync):
+// One warp routes one token (route_token_vals: logits already loaded by
+// load_logits): lane r (< topk) returns the r-th chosen expert and its
+// weight.  Each selection round is two warp reductions (redux.sync):
 // the largest key, then the lowest expert index holding it -- descending
 // logit, the lower index on ties.
-template <int VPL>  // logits per lane (E <= 32 * VPL)
-__device__ __forceinline__ void route_token(const float* row, int E, int topk, int renormalize,
-                                            int lane, int& out_id, float& out_w) {
-  float v[VPL];
-  uint32_t key[VPL];
+// This lane's logits of one token: expert lane + 32 i in v[i] (-inf past E).
+template <int VPL>
+__device__ __forceinline__ void load_logits(const float* row, int E, int lane, float (&v)[VPL]) {
 #pragma unroll
   for (int i = 0; i < VPL; ++i) {
     const int e = lane + 32 * i;
     v[i] = (e < E) ? (*(row + e)) : -INFINITY;
-    key[i] = (e < E) ? logit_key(v[i]) : 0u;
   }
+}
+
+template <int VPL>  // logits per lane (E <= 32 * VPL), already in registers
+__device__ __forceinline__ void route_token_vals(const float (&v)[VPL], int E, int topk, int renormalize,
+                                                 int lane, int& out_id, float& out_w) {
+  uint32_t key[VPL];
+#pragma unroll
+  for (int i = 0; i < VPL; ++i) key[i] = (lane + 32 * i < E) ? logit_key(v[i]) : 0u;
   // softmax statistics over all experts
   uint32_t kmax = 0;
 #pragma unroll
@@ -81,6 +87,14 @@ __device__ __forceinline__ void route_token(const float* row, int E, int topk, i
   for (int off = 16; off > 0; off >>= 1) s += __shfl_xor_sync(0xffffffffu, s, off);
   out_id = my_id;
   out_w = renormalize ? __fdiv_rn(ex, s) : __fdiv_rn(ex, z);
+}
+
+template <int VPL>
+__device__ __forceinline__ void route_token(const float* row, int E, int topk, int renormalize,
+                                            int lane, int& out_id, float& out_w) {
+  float v[VPL];
+  load_logits<VPL>(row, E, lane, v);
+  route_token_vals<VPL>(v, E, topk, renormalize, lane, out_id, out_w);
 }
 
 }  // namespace moe
