@@ -72,8 +72,9 @@ struct Cfg {
   // asynchronous bulk copy (256 contiguous bytes per row): a thread's own row stored from
   // registers would take 16 scattered 16-byte stores, which cost a third of the kernel.  The
   // staging area (pitch 272 bytes: 16-byte aligned, 4-way bank spread) takes one ring stage.
-  static constexpr bool kStageY = kDown && kFP8 && !kSwap;
-  static constexpr int kYPitch = 272;
+  // GEMM1 FP8 normal tiles do the same with their 64-byte FP8 row chunks (four scattered 16-byte stores).
+  static constexpr bool kStageY = kFP8 && !kSwap;
+  static constexpr int kYPitch = kDown ? 272 : 80;
   static constexpr int kYStageBytes = kStageY ? 256 * kYPitch : 0;
   static constexpr int kStagesFit = (kSmemLimit - kSmemReserve - 1024 - kYStageBytes) / kStageBytes;
   static constexpr int kStages = kStagesFit > 8 ? 8 : kStagesFit;
@@ -648,11 +649,16 @@ __global__ void __launch_bounds__(kThreads, 1)
                          (static_cast<uint32_t>(f32x2_to_e4m3x2(acc_a[4 * i + 2] * inv, acc_a[4 * i + 3] * inv))
                           << 16);
             }
-            uint4* dst = reinterpret_cast<uint4*>(static_cast<uint8_t*>(args.out) + static_cast<size_t>(grow) * I +
-                                                  col0);
+            // the row's 64 codes go out through shared memory as one bulk copy
+            uint8_t* st_row = reserve + kSmemReserve + static_cast<size_t>(threadIdx.x - 64) * C::kYPitch;
+            bulk_wait_read_all();   // the previous copy from this staging slot has read it
 #pragma unroll
             for (int i = 0; i < 4; ++i)
-              dst[i] = make_uint4(words[4 * i], words[4 * i + 1], words[4 * i + 2], words[4 * i + 3]);
+              reinterpret_cast<uint4*>(st_row)[i] = make_uint4(words[4 * i], words[4 * i + 1], words[4 * i + 2],
+                                                               words[4 * i + 3]);
+            fence_proxy_async_smem();
+            bulk_store(static_cast<uint8_t*>(args.out) + static_cast<size_t>(grow) * I + col0, st_row, 64);
+            bulk_commit();
             if (g == 0) args.out_scale_t[static_cast<size_t>(nt) * args.capacity + grow] = scale;
           }
         } else {
