@@ -231,7 +231,9 @@ __global__ void __launch_bounds__(kThreads, 1)
       // GEMM2: the weight tiles of the first kStages fills are issued before the
       // wait (they depend only on the alignment); the a2 tiles follow after it.
       if (lane == 0) {
-        const uint64_t pol_w = policy_evict_first();
+        // weights: read once per expert by swap-AB tiles (evict first), but by every 128-row block of
+        // the expert in the normal orientation, whose blocks run in the same wave (keep in L2)
+        const uint64_t pol_w = kSwap ? policy_evict_first() : policy_evict_normal();
         const uint64_t pol_a = policy_evict_last();
         int stage = 0;
         uint32_t phase = 0;
@@ -308,7 +310,9 @@ __global__ void __launch_bounds__(kThreads, 1)
     // All 32 lanes stage the tile's token row ids (GEMM1 gathers token rows
     // from x or its quantised copy); lane 0 issues every TMA load.
     int32_t* tok_rows = reinterpret_cast<int32_t*>(reserve + kTokRowsOffset);
-    const uint64_t pol_w = policy_evict_first();
+    // weights: read once per expert by swap-AB tiles (evict first), but by every 128-row block of
+    // the expert in the normal orientation, whose blocks run in the same wave (keep in L2)
+    const uint64_t pol_w = kSwap ? policy_evict_first() : policy_evict_normal();
     const uint64_t pol_a = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
@@ -1075,7 +1079,7 @@ __global__ void __launch_bounds__(kThreads, 1)
     // All lanes stage the tile's token row ids (GEMM1 gathers code rows of
     // the per-token quantised x); lane 0 issues every copy.
     int32_t* tok_rows = reinterpret_cast<int32_t*>(reserve + kTokRowsOffset);
-    const uint64_t pol_w = policy_evict_first();
+    const uint64_t pol_w = policy_evict_normal();   // reused by every 128-row block of the expert
     const uint64_t pol_a = policy_evict_last();
     int stage = 0;
     uint32_t phase = 0;
