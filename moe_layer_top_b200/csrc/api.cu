@@ -123,6 +123,10 @@ int validate_problem(const moe_problem* p) {
 // Tile orientation and block size.  Swap-AB when an expert is expected to see
 // few tokens (the MMA M dimension is then filled by weight rows); the block
 // is the smallest of 16/32/64 that usually holds an expert's tokens whole.
+// The switch sits at 16 expected tokens per hit expert: there, with evenly
+// spread routing, swap-AB tiles are a little faster, but with skewed routing
+// the hot experts' many 16/32-row blocks each re-stream their weights and
+// the 128-row tiles win by far more; the host cannot see the skew.
 void resolve(moe_problem* p) {
   if (p->weight_dtype == MOE_DTYPE_MXFP8_E4M3) {  // block-scaled MMA: normal tiles only
     p->mode = MOE_MODE_NORMAL;
@@ -139,7 +143,7 @@ void resolve(moe_problem* p) {
     else if (p->block_m != 0 || p->H % 256)  // normal tiles need H % 256 == 0
       p->mode = MOE_MODE_SWAP_AB;
     else
-      p->mode = avg <= 40.0 ? MOE_MODE_SWAP_AB : MOE_MODE_NORMAL;
+      p->mode = avg < 16.0 ? MOE_MODE_SWAP_AB : MOE_MODE_NORMAL;
   }
   if (p->block_m == 0) {
     if (p->mode == MOE_MODE_NORMAL)

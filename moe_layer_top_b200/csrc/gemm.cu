@@ -499,6 +499,14 @@ __global__ void __launch_bounds__(kThreads, 1)
         // ---------------- normal: row = token row of the tile
         const int grow = mb * 128 + row;  // sorted row
         constexpr int kCols = kDown ? 128 : 64;  // accumulator columns per group (per gate/up half for GEMM1)
+        // GEMM2: the row's flat assignment and routed weight, read before the K loop so that
+        // their two dependent global loads are not on the tile's tail
+        int flat = 0;
+        float wt = 0.f;
+        if constexpr (kDown) {
+          flat = (*(args.sorted_ids + grow));
+          wt = flat < args.nflat ? route_weight(args.topk_weights, flat) : 0.f;
+        }
         float acc_a[kFP8 ? kCols : 1];
         float acc_b[(kFP8 && !kDown) ? kCols : 1];
         if constexpr (kFP8) {
@@ -667,9 +675,7 @@ __global__ void __launch_bounds__(kThreads, 1)
           }
         } else {
           // ---- GEMM2 epilogue: routed weight, scatter the row to y[flat]
-          const int flat = (*(args.sorted_ids + grow));
           const bool real = flat < args.nflat;
-          const float wt = real ? route_weight(args.topk_weights, flat) : 0.f;
           __nv_bfloat16* yrow =
               static_cast<__nv_bfloat16*>(args.out) + static_cast<size_t>(real ? flat : 0) * H + nt * 256 + g * 128;
           if constexpr (kFP8) {
