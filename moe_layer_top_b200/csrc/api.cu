@@ -375,8 +375,7 @@ int run_stages(const moe_problem* prob, const void* x, const float* logits, cons
                                     p.router_weight_on_input == 1 ? wts : nullptr, xq, at<void>(ws, L.a1_scale),
                                     stream);
           if (e == cudaSuccess)
-            e = moe::launch_copy_rows(xq, p.H, p.topk, nflat, at<int32_t>(ws, L.sorted_token_ids),
-                                      at<int32_t>(ws, L.num_tokens_post_padded), cap, at<void>(ws, L.a1), stream);
+            e = moe::launch_copy_rows(xq, p.H, p.topk, nflat, pos, at<void>(ws, L.a1), stream);
         } else if (!plan.tok_gather)
           e = moe::launch_gather(x, p.H, p.topk, nflat, at<int32_t>(ws, L.sorted_token_ids),
                                  at<int32_t>(ws, L.num_tokens_post_padded), cap, plan.fp8, plan.mx,

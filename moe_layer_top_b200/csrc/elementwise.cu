@@ -205,33 +205,51 @@ __global__ void __launch_bounds__(256) scale_rows_kernel(const __nv_bfloat16* x,
 }
 
 // ----------------------------------------------------------------------------
-// Sorted copy of quantised rows: a1[r] = xq[sorted_ids[r] / topk] (E4M3 bytes)
-// for the real rows r < ntpp.  With the per-token quantiser in front, x is
-// read and quantised once per token instead of once per assignment; this
-// copy then reads the L2-resident codes.
+// Sorted copy of quantised rows: a1[pos_of_flat[f]] = xq[f / topk] (E4M3 bytes)
+// for every assignment f that has a row.  With the per-token quantiser in
+// front, x is read and quantised once per token instead of once per
+// assignment; this copy then reads the L2-resident codes.  One warp per row:
+// each lane issues its 16-byte loads of a 4 KB piece of the row before any
+// store, and the 64 warps an SM holds keep that many rows in flight.
+// Padding rows are never stored (GEMM1 reads them; their outputs are dropped).
 // ----------------------------------------------------------------------------
 __global__ void __launch_bounds__(256) copy_rows_kernel(const uint8_t* xq, int H, int topk, int nflat,
-                                                        const int32_t* sorted_ids, const int32_t* ntpp_ptr,
-                                                        uint8_t* a1) {
+                                                        const int32_t* pos_of_flat, uint8_t* a1) {
   pdl_launch_dependents();
   pdl_wait();
-  const int ntpp = *ntpp_ptr;
+  constexpr int kPer = 8;  // 16-byte vectors per lane in flight
+  const int lane = threadIdx.x & 31;
+  const int warps = gridDim.x * (blockDim.x >> 5);
   const int vecs = H / 16;
-  for (int row = blockIdx.x; row < ntpp; row += gridDim.x) {
-    const int flat = (*(sorted_ids + row));
-    if (flat >= nflat) continue;  // padding rows are never stored
-    const uint4* src = reinterpret_cast<const uint4*>(xq + static_cast<size_t>(flat / topk) * H);
+  for (int f = blockIdx.x * (blockDim.x >> 5) + (threadIdx.x >> 5); f < nflat; f += warps) {
+    const int row = (*(pos_of_flat + f));
+    if (row < 0) continue;  // an invalid expert id (or another rank's expert): no row
+    const uint4* src = reinterpret_cast<const uint4*>(xq + static_cast<size_t>(f / topk) * H);
     uint4* dst = reinterpret_cast<uint4*>(a1 + static_cast<size_t>(row) * H);
-    for (int v = threadIdx.x; v < vecs; v += blockDim.x) dst[v] = (*(src + v));
+    for (int base = 0; base < vecs; base += kPer * 32) {
+      uint4 v[kPer];
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int k = base + i * 32 + lane;
+        if (k < vecs) v[i] = (*(src + k));
+      }
+#pragma unroll
+      for (int i = 0; i < kPer; ++i) {
+        const int k = base + i * 32 + lane;
+        if (k < vecs) dst[k] = v[i];
+      }
+    }
   }
 }
 
-cudaError_t launch_copy_rows(const void* xq, int H, int topk, int nflat, const int32_t* sorted_ids,
-                             const int32_t* ntpp, int capacity, void* a1, cudaStream_t stream) {
-  if (capacity == 0) return cudaSuccess;
-  const int blocks = capacity < 148 * 8 ? capacity : 148 * 8;
+cudaError_t launch_copy_rows(const void* xq, int H, int topk, int nflat, const int32_t* pos_of_flat, void* a1,
+                             cudaStream_t stream) {
+  if (nflat == 0) return cudaSuccess;
+  if (pos_of_flat == nullptr) return cudaErrorInvalidValue;
+  const int want = (nflat + 7) / 8;  // eight warps (rows) per block
+  const int blocks = want < 148 * 8 ? want : 148 * 8;
   return launch_pdl(copy_rows_kernel, blocks, 256, 0, stream, static_cast<const uint8_t*>(xq), H, topk, nflat,
-                    sorted_ids, ntpp, static_cast<uint8_t*>(a1));
+                    pos_of_flat, static_cast<uint8_t*>(a1));
 }
 
 cudaError_t launch_prepare_x(const void* x, int T, int H, int topk, bool fp8, bool mx, const int32_t* pos_of_flat,

@@ -79,9 +79,9 @@ cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32
 cudaError_t launch_prepare_x(const void* x, int T, int H, int topk, bool fp8, bool mx, const int32_t* pos_of_flat,
                              int capacity, const float* row_weight, void* xq, void* scales, cudaStream_t stream);
 
-// a1[r] = xq[sorted_ids[r] / topk] (E4M3 rows [T, H] -> sorted [capacity, H]) for real rows
-cudaError_t launch_copy_rows(const void* xq, int H, int topk, int nflat, const int32_t* sorted_ids,
-                             const int32_t* ntpp, int capacity, void* a1, cudaStream_t stream);
+// a1[pos_of_flat[f]] = xq[f / topk] (E4M3 rows [T, H] -> sorted [capacity, H]) for every row-owning f
+cudaError_t launch_copy_rows(const void* xq, int H, int topk, int nflat, const int32_t* pos_of_flat, void* a1,
+                             cudaStream_t stream);
 
 // out[t] = sum_j y[t*topk + j]; with pos_of_flat, only the assignments that
 // have a row (pos_of_flat >= 0: local experts under expert parallelism)

@@ -391,11 +391,13 @@ __global__ void __launch_bounds__(1024) route_align_small_kernel(
     if (pos_of_flat && i < end) pos_of_flat[i] = dest;  // -1 for an invalid id
     __syncwarp();
   }
-  // padding: each expert's slots past its count, then everything past num_tokens_post_padded;
-  // block experts: each expert's blocks, then -1 past the used ones
-  for (int e = tid; e < E; e += 1024) {
-    for (int p = offs[e] + cnt[e]; p < offs[e + 1]; ++p) sorted_ids[p] = n;
-    for (int b = offs[e] / block_m; b < offs[e + 1] / block_m; ++b) expert_ids[b] = e;
+  // padding: each expert's slots past its count (one warp per expert, consecutive lanes on
+  // consecutive slots), then everything past num_tokens_post_padded; block experts: each
+  // expert's blocks, then -1 past the used ones
+  for (int e = warp; e < E; e += 32) {
+    const int p1 = offs[e + 1];
+    for (int p = offs[e] + cnt[e] + lane; p < p1; p += 32) sorted_ids[p] = n;
+    for (int b = offs[e] / block_m + lane; b < p1 / block_m; b += 32) expert_ids[b] = e;
   }
   for (int p = ntpp + tid; p < capacity; p += 1024) sorted_ids[p] = n;
   for (int b = ntpp / block_m + tid; b < capacity / block_m; b += 1024) expert_ids[b] = -1;
