@@ -138,15 +138,20 @@ cudaError_t launch_gather(const void* x, int H, int topk, int nflat, const int32
 template <bool MX>
 __global__ void __launch_bounds__(256) quantize_x_kernel(const __nv_bfloat16* x, int T, int H, int topk,
                                                          const int32_t* pos_of_flat, int capacity,
-                                                         const float* row_weight, uint8_t* xq, void* scales) {
+                                                         const float* row_weight, uint8_t* xq, void* scales,
+                                                         int split) {
   pdl_launch_dependents();
   pdl_wait();
   const int vecs = H / 8;
-  const int iters = (vecs + blockDim.x - 1) / blockDim.x;
-  for (int t = blockIdx.x; t < T; t += gridDim.x) {
+  const int chunks = (vecs + blockDim.x - 1) / blockDim.x;  // 256-vector chunks of a row
+  // split = 1: a block takes whole rows; split = chunks (few rows): one chunk of a row
+  const long long items = static_cast<long long>(T) * split;
+  for (long long item = blockIdx.x; item < items; item += gridDim.x) {
+    const int t = static_cast<int>(item / split);
+    const int c0 = static_cast<int>(item - static_cast<long long>(t) * split);
     const float rw = row_weight ? (*(row_weight + static_cast<size_t>(t) * topk)) : 1.0f;
     const __nv_bfloat16* src = x + static_cast<size_t>(t) * H;
-    for (int it = 0; it < iters; ++it) {
+    for (int it = c0; it < chunks; it += split) {
       const int v = it * blockDim.x + threadIdx.x;  // uniform trip count: shuffles see full warps
       const bool in = v < vecs;
       uint4 u = make_uint4(0, 0, 0, 0);
@@ -255,16 +260,21 @@ cudaError_t launch_copy_rows(const void* xq, int H, int topk, int nflat, const i
 cudaError_t launch_prepare_x(const void* x, int T, int H, int topk, bool fp8, bool mx, const int32_t* pos_of_flat,
                              int capacity, const float* row_weight, void* xq, void* scales, cudaStream_t stream) {
   if (T == 0) return cudaSuccess;
-  const int blocks = T < 148 * 8 ? T : 148 * 8;
+  // whole rows per block when the rows alone fill the grid; else a block per 256-vector chunk of a row
+  const int chunks = (H / 8 + 255) / 256;
+  const int split = T >= 148 * 8 ? 1 : chunks;
+  const long long items = static_cast<long long>(T) * split;
+  const int blocks = items < 148 * 8 ? static_cast<int>(items) : 148 * 8;
+  const int row_blocks = T < 148 * 8 ? T : 148 * 8;  // scale_rows_kernel: one row per block
   const __nv_bfloat16* xb = static_cast<const __nv_bfloat16*>(x);
   if (mx)
     return launch_pdl(quantize_x_kernel<true>, blocks, 256, 0, stream, xb, T, H, topk, pos_of_flat, capacity,
-                      row_weight, static_cast<uint8_t*>(xq), scales);
+                      row_weight, static_cast<uint8_t*>(xq), scales, split);
   if (fp8)
     return launch_pdl(quantize_x_kernel<false>, blocks, 256, 0, stream, xb, T, H, topk, pos_of_flat, capacity,
-                      row_weight, static_cast<uint8_t*>(xq), scales);
+                      row_weight, static_cast<uint8_t*>(xq), scales, split);
   if (row_weight)
-    return launch_pdl(scale_rows_kernel, blocks, 256, 0, stream, xb, T, H, topk, row_weight,
+    return launch_pdl(scale_rows_kernel, row_blocks, 256, 0, stream, xb, T, H, topk, row_weight,
                       static_cast<__nv_bfloat16*>(xq));
   return cudaSuccess;
 }
