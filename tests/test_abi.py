@@ -68,6 +68,23 @@ def test_resolve_problem_auto_modes(L):
     assert q.mode == ops.MODE_SWAP_AB and q.block_m == 32
 
 
+@pytest.mark.parametrize("T,E,H,I,want", [
+    (255, 128, 4096, 1536, ("swap", 32)),    # 15.9 expected tokens per expert
+    (256, 128, 4096, 1536, ("normal", 128)),  # 16: the switch point
+    (128, 128, 4096, 1536, ("swap", 16)),     # 8
+    (129, 128, 4096, 1536, ("swap", 32)),     # just above 8
+    (511, 256, 7168, 2048, ("swap", 32)),
+    (512, 256, 7168, 2048, ("normal", 128)),
+    (32, 256, 7168, 2048, ("swap", 16)),
+])
+def test_resolve_problem_orientation_switch(L, T, E, H, I, want):
+    # swap-AB below 16 expected tokens per hit expert (T*k/E under even routing), 128-row tiles from 16 on
+    for fp8 in (False, True):
+        q = ops.resolve_problem(ops.problem(T, E, 8, H, I, fp8=fp8))
+        got = ("swap" if q.mode == ops.MODE_SWAP_AB else "normal", q.block_m)
+        assert got == want, (T, E, fp8, got)
+
+
 def test_resolve_problem_mxfp8_is_normal_128(L):
     for T in (1, 64, 16384):
         q = ops.resolve_problem(ops.problem(T, 128, 8, 4096, 1536, mx=True))
