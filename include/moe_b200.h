@@ -86,7 +86,7 @@ extern "C" {
  */
 
 /* tile orientation of the two grouped GEMMs */
-#define MOE_MODE_AUTO 0    /* chosen from the expected tokens per expert */
+#define MOE_MODE_AUTO 0    /* swap-AB below 16 expected tokens per hit expert (T*topk/E), else normal */
 #define MOE_MODE_NORMAL 1  /* MMA M = 128 token rows (block_m 128), N = 256 weight rows */
 #define MOE_MODE_SWAP_AB 2 /* MMA M = 128 weight rows, N = block_m token rows */
 
