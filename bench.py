@@ -16,8 +16,9 @@ own roofline and CPU baseline: the compute-bound FP8 prefill layer
 (H=4096, E=128, top-8, I=1536, T=16384) and the bf16 decode layer of the
 same shape (T = 1 ... 64).  ``--workload NAME`` times one workload alone.
 
-L2 is flushed (a 256 MiB write) before every timed step; the flush is outside
-the CUDA-event brackets.  Multi-GPU runs are independent replicas by default
+L2 is flushed before every timed step, outside the CUDA-event brackets: a
+256 MiB write, then a read of the same buffer, so that the flush's own dirty
+lines are written back before the step instead of inside it.  Multi-GPU runs are independent replicas by default
 (each rank runs the same workload; the time is the max over ranks).  With
 ``--ep N`` the layer is expert-parallel instead: each of N ranks holds E/N
 experts, runs its share of the replicated batch and the output is all-reduced
@@ -49,6 +50,15 @@ import torch  # noqa: E402
 from moe_layer_top_b200 import inputs  # noqa: E402
 
 L2_FLUSH_BYTES = 256 << 20
+
+
+def flush_l2(buf: torch.Tensor) -> None:
+    """Evict the layer's data from L2: write a buffer twice L2's size, then read
+    it back (the read pass writes the written lines back to HBM, so the step
+    starts with clean lines of an unrelated buffer rather than paying for the
+    flush's write-backs)."""
+    buf.zero_()
+    buf.sum()
 
 
 def parse_args():
@@ -421,10 +431,10 @@ def time_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor, world
 
     g_stg = capture(staged)
     for _ in range(warmup):
-        flush.zero_()
+        flush_l2(flush)
         g_fwd.replay()
         wl.collective()
-        flush.zero_()
+        flush_l2(flush)
         g_stg.replay()
     torch.cuda.synchronize()
     ev = [(torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)) for _ in range(steps)]
@@ -432,7 +442,7 @@ def time_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor, world
     torch.cuda.synchronize()
     wall0 = time.perf_counter()
     for i in range(steps):
-        flush.zero_()
+        flush_l2(flush)
         ev[i][0].record(stream)
         g_fwd.replay()
         wl.collective()     # outside the graph: no NCCL call is ever captured
@@ -443,7 +453,7 @@ def time_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor, world
     step_ms = np.array([a.elapsed_time(b) for a, b in ev])
     per_stage = []
     for i in range(steps):
-        flush.zero_()
+        flush_l2(flush)
         g_stg.replay()
         torch.cuda.synchronize()
         per_stage.append(se.elapsed())
@@ -472,12 +482,12 @@ def e2e_steps(wl: Workload, steps: int, warmup: int, flush: torch.Tensor):
         out_h.copy_(wl.out, non_blocking=True)
 
     for _ in range(warmup):
-        flush.zero_()
+        flush_l2(flush)
         one()
     torch.cuda.synchronize()
     times = []
     for _ in range(steps):
-        flush.zero_()
+        flush_l2(flush)
         a, b = torch.cuda.Event(enable_timing=True), torch.cuda.Event(enable_timing=True)
         a.record(stream)
         one()
@@ -656,7 +666,7 @@ def measure(cfg, args, world, flush, peaks, ep=None, T_only=0):
                    "global_batch": layer_copies * T_head, "tokens_per_gpu": T_head, "parallelism": parallelism,
                    "weights": ("mxfp8 e4m3 + per-32 e8m0 scales" if cfg.mx else "fp8 e4m3 + 128x128 fp32 scales")
                    if cfg.fp8 else "bf16",
-                   "routing": cfg.routing, "l2": "flushed (256 MiB write) before every step, outside the timing",
+                   "routing": cfg.routing, "l2": "flushed (256 MiB write, then read back) before every step, outside the timing",
                    "launch": ("CUDA graph of moe_fused_forward (persistent decode kernel where eligible)"
                               if args.persistent_decode else "CUDA graph of moe_fused_forward (PDL between kernels)"),
                    "layer_bytes_per_step": alg["layer_bytes"], "layer_flops_per_step": alg["flops"],
