@@ -360,14 +360,18 @@ __global__ void __launch_bounds__(1024) route_align_small_kernel(
     }
     if (lane == 31) warp_sums[warp] = incl;
     __syncthreads();
-    int32_t before = 0, total = 0;
-    for (int w = 0; w < 32; ++w) {
-      const int32_t s = warp_sums[w];
-      if (w < warp) before += s;
-      total += s;
+    // only the first ceil(E / 32) warps hold experts (E <= 256): a thread adds the sums of
+    // the warps before its own, thread 0 all of them
+    if (tid < E) {
+      int32_t before = 0;
+      for (int w = 0; w < warp; ++w) before += warp_sums[w];
+      offs[tid] = before + incl - v;
     }
-    if (tid < E) offs[tid] = before + incl - v;
-    if (tid == 0) offs[E] = total;
+    if (tid == 0) {
+      int32_t total = 0;
+      for (int w = 0; w < (E + 31) / 32; ++w) total += warp_sums[w];
+      offs[E] = total;
+    }
   }
   __syncthreads();
   const int ntpp = offs[E];
