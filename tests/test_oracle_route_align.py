@@ -126,3 +126,30 @@ def test_identity_expert_through_align_reproduces_x():
             y[s[r]] = x[s[r] // k]                  # identity expert on the gathered row
     out = (w.astype(np.float64)[:, :, None] * y.reshape(T, k, 64)).sum(1)
     np.testing.assert_allclose(out, x, rtol=1e-6, atol=1e-7)
+
+
+def test_align_random_shapes_match_brute_force():
+    """Sixty random (T, E, k, BM, id distribution) draws, including empty and single-expert cases,
+    against the counting sort written as a loop."""
+    rng = np.random.default_rng(2024)
+    for case in range(60):
+        E = int(rng.integers(1, 65))
+        k = int(rng.integers(1, min(8, E) + 1))
+        T = int(rng.integers(0, 41))
+        bm = int(rng.choice([16, 32, 64, 128]))
+        kind = case % 3
+        if kind == 0 and T > 0:
+            ids = np.stack([rng.permutation(E)[:k] for _ in range(T)])
+        elif kind == 1:
+            ids = rng.integers(0, E, (T, k))
+        else:
+            ids = np.minimum(rng.zipf(1.3, (T, k)) - 1, E - 1)
+        ids = np.asarray(ids, dtype=np.int32).reshape(T, k)
+        a = O.align(ids, E, bm)
+        ref_sorted, ref_blocks = _brute_align(ids, E, bm)
+        ntpp = a["num_tokens_post_padded"]
+        assert ntpp == len(ref_sorted), case
+        np.testing.assert_array_equal(a["sorted_token_ids"][:ntpp], ref_sorted, err_msg=str(case))
+        np.testing.assert_array_equal(a["expert_ids"][:ntpp // bm], ref_blocks, err_msg=str(case))
+        assert a["capacity"] == O.align_capacity(T, k, E, bm) >= ntpp
+        np.testing.assert_array_equal(a["expert_counts"], np.bincount(ids.reshape(-1), minlength=E))
