@@ -6,6 +6,7 @@ sort order, an off-by-one, a missing weight), compiles the copy and runs the
 oracle pins against it through ``MOE_ORACLE_LIB``: at least one pin must fail.
 The planted mistakes live only in the temporary copies."""
 
+import concurrent.futures as cf
 import os
 import shutil
 import subprocess
@@ -42,6 +43,16 @@ MUTANTS = [
      "  double r = std::ldexp(std::round(std::ldexp(x, -q)), q);"),
     ("weight_scale_448_off", "std::max(static_cast<float>(bmax), static_cast<float>(1e-10)) / 448.0f;",
      "std::max(static_cast<float>(bmax), static_cast<float>(1e-10)) / 440.0f;"),
+    ("weight_scale_one_k_block", "acc += (kE4m3.v[r[k]] * static_cast<double>(s[k / 128])) * v[k];",
+     "acc += (kE4m3.v[r[k]] * static_cast<double>(s[0])) * v[k];"),
+    ("e8m0_bias", "constexpr int kE8m0Bias = 127;", "constexpr int kE8m0Bias = 126;"),
+    ("x_not_quantised", "for (int j = 0; j < group; ++j) xh[g * group + j] = kE4m3.v[codes[j]] * scale;",
+     "for (int j = 0; j < group; ++j) xh[g * group + j] = row[g * group + j];"),
+    ("router_weight_on_input_ignored",
+     "row[k] = round_bf16(static_cast<double>(static_cast<float>(row[k]) * w));   // one fp32 product",
+     "row[k] = row[k] + 0.0 * w;"),
+    ("shard_split_rounded_up", "first[r] = static_cast<int32_t>((static_cast<int64_t>(r) * E) / world);",
+     "first[r] = static_cast<int32_t>((static_cast<int64_t>(r) * E + world - 1) / world);"),
 ]
 
 
@@ -49,20 +60,42 @@ def _cxx():
     for c in (shutil.which("g++"), os.environ.get("CXX"), "/usr/bin/g++"):
         if c and os.path.exists(c):
             return c
-    pytest.skip("no C++ compiler")
+    return None
 
 
-@pytest.mark.parametrize("name,old,new", MUTANTS, ids=[m[0] for m in MUTANTS])
-def test_pins_catch_planted_mistake(name, old, new, tmp_path):
+def _run_mutant(cxx, workdir, name, old, new):
+    """Build the copy with one planted mistake and run the pins against it: (exit code, output tail)."""
     src = open(SRC).read()
-    assert src.count(old) == 1, f"{name}: the text to mutate must occur exactly once"
-    mutated = tmp_path / "moe_oracle.cpp"
-    mutated.write_text(src.replace(old, new))
-    lib = tmp_path / "libmoe_oracle_mutant.so"
-    res = subprocess.run([_cxx(), "-O1", "-std=c++17", "-fPIC", "-shared", "-ffp-contract=off", str(mutated),
-                          "-o", str(lib)], capture_output=True, text=True)
-    assert res.returncode == 0, res.stderr
-    env = dict(os.environ, MOE_ORACLE_LIB=str(lib))
+    if src.count(old) != 1:
+        return -100, f"{name}: the text to mutate must occur exactly once"
+    d = os.path.join(workdir, name)
+    os.makedirs(d, exist_ok=True)
+    mutated = os.path.join(d, "moe_oracle.cpp")
+    with open(mutated, "w") as f:
+        f.write(src.replace(old, new))
+    lib = os.path.join(d, "libmoe_oracle_mutant.so")
+    res = subprocess.run([cxx, "-O1", "-std=c++17", "-fPIC", "-shared", "-ffp-contract=off", mutated, "-o", lib],
+                         capture_output=True, text=True)
+    if res.returncode != 0:
+        return -101, res.stderr[-2000:]
+    env = dict(os.environ, MOE_ORACLE_LIB=lib, OMP_NUM_THREADS="2")
     run = subprocess.run([sys.executable, "-m", "pytest", "-x", "-q", "-m", "not gpu", "-p", "no:cacheprovider",
                           *PINS], cwd=ROOT, env=env, capture_output=True, text=True, timeout=900)
-    assert run.returncode == 1, f"mutant {name} survived the pins:\n{run.stdout[-2000:]}"
+    return run.returncode, run.stdout[-2000:]
+
+
+@pytest.fixture(scope="module")
+def outcomes(tmp_path_factory):
+    cxx = _cxx()
+    if cxx is None:
+        pytest.skip("no C++ compiler")
+    work = str(tmp_path_factory.mktemp("mutants"))
+    with cf.ThreadPoolExecutor(max_workers=max(1, min(8, os.cpu_count() or 1))) as ex:
+        futs = {m[0]: ex.submit(_run_mutant, cxx, work, *m) for m in MUTANTS}
+        return {k: f.result() for k, f in futs.items()}
+
+
+@pytest.mark.parametrize("name", [m[0] for m in MUTANTS])
+def test_pins_catch_planted_mistake(outcomes, name):
+    rc, tail = outcomes[name]
+    assert rc == 1, f"mutant {name}: pins exit code {rc} (1 = a pin failed):\n{tail}"
