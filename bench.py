@@ -18,8 +18,9 @@ same shape (T = 1 ... 64).  ``--workload NAME`` times one workload alone.
 
 L2 is flushed before every timed step, outside the CUDA-event brackets: a
 256 MiB write, then a read of the same buffer, so that the flush's own dirty
-lines are written back before the step instead of inside it.  Multi-GPU runs are independent replicas by default
-(each rank runs the same workload; the time is the max over ranks).  With
+lines are written back before the step instead of inside it.  Multi-GPU runs
+are independent replicas by default (each rank runs the same workload; the
+time is the max over ranks).  With
 ``--ep N`` the layer is expert-parallel instead: each of N ranks holds E/N
 experts, runs its share of the replicated batch and the output is all-reduced
 over NCCL; on one GPU ``--ep N`` times one rank's share alone.
