@@ -272,27 +272,33 @@ class Workload:
     def algorithmic(self):
         """Algorithmic bytes / FLOPs of the layer and of each GEMM for this routing."""
         v = self.ops.workspace_views(self.p, self.ws)
-        counts = v["expert_counts"].cpu().numpy()
-        ntpp = int(v["num_tokens_post_padded"].item())
-        hit = int((counts > 0).sum())
-        cfg = self.cfg
-        elem = 1 if cfg.fp8 else 2
-        if cfg.mx:   # one E8M0 byte per 32 weights
-            w13_e = 2 * cfg.I * cfg.H * (1 + 1 / 32)
-            w2_e = cfg.H * cfg.I * (1 + 1 / 32)
-        else:
-            w13_e = 2 * cfg.I * cfg.H * elem + (2 * cfg.I // 128) * (cfg.H // 128) * 4 * cfg.fp8
-            w2_e = cfg.H * cfg.I * elem + (cfg.H // 128) * (cfg.I // 128) * 4 * cfg.fp8
-        nflat = self.T * cfg.topk
-        nlocal = int(counts.sum())       # assignments run here (all of them without expert parallelism)
-        route_io = self.T * cfg.E * 4 if "logits" in self.routing else nflat * 8
-        rows = ntpp
-        gemm1 = hit * w13_e + rows * cfg.H * elem + rows * cfg.I * elem
-        gemm2 = hit * w2_e + rows * cfg.I * elem + nlocal * cfg.H * 2
-        layer = hit * (w13_e + w2_e) + self.T * cfg.H * 2 * 2 + route_io
-        flops = 2.0 * nlocal * 3 * cfg.H * cfg.I
-        return {"hit_experts": hit, "padded_rows": ntpp, "layer_bytes": layer, "gemm1_bytes": gemm1,
-                "gemm2_bytes": gemm2, "flops": flops, "w13_bytes_per_expert": w13_e, "w2_bytes_per_expert": w2_e}
+        return algorithmic_counts(self.cfg, self.T, v["expert_counts"].cpu().numpy(),
+                                  int(v["num_tokens_post_padded"].item()), "logits" in self.routing)
+
+
+def algorithmic_counts(cfg, T, counts, ntpp, has_logits):
+    """Algorithmic bytes and FLOPs of one layer step: every hit expert's weights read once (with
+    their scales), x read and out written once, the routing input read; per GEMM also the padded
+    token rows it reads and the rows it writes.  FLOPs count real assignments only (2 * 3 * H * I
+    each).  counts: assignments per expert run here; ntpp: padded rows of the alignment."""
+    hit = int((counts > 0).sum())
+    elem = 1 if cfg.fp8 else 2
+    if cfg.mx:   # one E8M0 byte per 32 weights
+        w13_e = 2 * cfg.I * cfg.H * (1 + 1 / 32)
+        w2_e = cfg.H * cfg.I * (1 + 1 / 32)
+    else:
+        w13_e = 2 * cfg.I * cfg.H * elem + (2 * cfg.I // 128) * (cfg.H // 128) * 4 * cfg.fp8
+        w2_e = cfg.H * cfg.I * elem + (cfg.H // 128) * (cfg.I // 128) * 4 * cfg.fp8
+    nflat = T * cfg.topk
+    nlocal = int(counts.sum())       # assignments run here (all of them without expert parallelism)
+    route_io = T * cfg.E * 4 if has_logits else nflat * 8
+    rows = ntpp
+    gemm1 = hit * w13_e + rows * cfg.H * elem + rows * cfg.I * elem
+    gemm2 = hit * w2_e + rows * cfg.I * elem + nlocal * cfg.H * 2
+    layer = hit * (w13_e + w2_e) + T * cfg.H * 2 * 2 + route_io
+    flops = 2.0 * nlocal * 3 * cfg.H * cfg.I
+    return {"hit_experts": hit, "padded_rows": ntpp, "layer_bytes": layer, "gemm1_bytes": gemm1,
+            "gemm2_bytes": gemm2, "flops": flops, "w13_bytes_per_expert": w13_e, "w2_bytes_per_expert": w2_e}
 
 
 def kernels_per_forward(cfg, T, has_logits):
